@@ -1,0 +1,247 @@
+"""Seeded synthetic decode batches shaped like the pages' workloads.
+
+This module only draws random inputs and builds block tables and slot
+mappings (the bookkeeping a serving engine's block manager hands to the
+kernels).  It holds none of the attention arithmetic, and it is shared by
+the CUDA path's tests and bench and by the oracle's tests.
+
+The pages measure on no public suite and print no tensors: miniVLLM's demo
+runs a randomly initialised Qwen3 on two prompts repeated thirty times and
+decodes up to 256 tokens (miniVLLM review, "What main.py actually does");
+mini-sglang serves Qwen3-0.6B; tiny-vllm runs Llama 3.2 1B (tiny-vllm
+write-up, "Diem noi bat").  The configurations below stand in for those
+decode batches with their attention shapes (heads, head_dim, GQA group),
+block size 16 and seeded N(0, 1) bf16 values.
+
+All tensors are created on the CPU with a seeded ``torch.Generator``; the
+caller moves them to a device.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import torch
+
+BF16_NAN_BITS = 0x7FC0          # quiet NaN in bf16
+POISON_BLOCK_ID = 0x7FFFFFFF    # block-table padding that must never be read
+
+
+@dataclasses.dataclass(frozen=True)
+class WorkloadSpec:
+    name: str
+    seed: int
+    num_seqs: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int = 16
+    description: str = ""
+
+
+SPECS = {
+    "tiny": WorkloadSpec(
+        "tiny", 36000, 4, 8, 2, 64,
+        description="batch 4, 8 q / 2 kv heads, head_dim 64, block 16, context_lens U[1,100], "
+                    "64-block pool, block ids a seeded permutation, append 1 token/seq"),
+    "qwen3": WorkloadSpec(
+        "qwen3", 36001, 60, 16, 8, 128,
+        description="Qwen3-0.6B-shaped decode: batch 60 (2 prompts x 30, no shared blocks), "
+                    "16 q / 8 kv heads, head_dim 128, context_lens U[20,300], shuffled pool"),
+    "llama32": WorkloadSpec(
+        "llama32", 36002, 128, 32, 8, 64,
+        description="Llama-3.2-1B-shaped decode: batch 128, 32 q / 8 kv heads, head_dim 64, "
+                    "context_lens U[512,4096], blocks scattered over a pool 1.5x the need"),
+    "longskew": WorkloadSpec(
+        "longskew", 36003, 64, 32, 8, 128,
+        description="long/skewed split-KV: 32 q / 8 kv heads, head_dim 128, one 131072-token "
+                    "sequence and 63 of 1024, 1% outlier keys x8, shuffled pool"),
+    "prefix": WorkloadSpec(
+        "prefix", 36004, 256, 16, 8, 128,
+        description="prefix-shared pages: batch 256, 16 q / 8 kv heads, head_dim 128, two "
+                    "1024-token prefixes shared by 128 seqs each, private suffixes U[0,256], "
+                    "append 1 token/seq then decode"),
+}
+
+
+@dataclasses.dataclass
+class Workload:
+    spec: WorkloadSpec
+    q: torch.Tensor             # [B][Hq][D] bf16
+    k_cache: torch.Tensor       # [NB][Hkv][bs][D] bf16
+    v_cache: torch.Tensor       # [NB][Hkv][bs][D] bf16
+    block_tables: torch.Tensor  # [B][M] int32
+    context_lens: torch.Tensor  # [B] int32 (decode length, appended token included)
+    k_new: torch.Tensor         # [B][Hkv][D] bf16: the token appended this step
+    v_new: torch.Tensor         # [B][Hkv][D] bf16
+    slot_mapping: torch.Tensor  # [B] int32: slot of position context_len - 1
+    scale: float
+
+    @property
+    def dims(self):
+        B, Hq, D = self.q.shape
+        NB, Hkv, bs, _ = self.k_cache.shape
+        return dict(num_seqs=B, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D,
+                    block_size=bs, num_blocks=NB, max_blocks_per_seq=self.block_tables.shape[1])
+
+
+def _randn_bf16(gen: torch.Generator, shape) -> torch.Tensor:
+    # fp32 N(0,1) draws rounded to nearest-even bf16
+    return torch.randn(shape, generator=gen, dtype=torch.float32).to(torch.bfloat16)
+
+
+def _pages(n_tokens: torch.Tensor, bs: int) -> torch.Tensor:
+    return (n_tokens + bs - 1) // bs
+
+
+def build_tables(block_lists, max_blocks: int) -> torch.Tensor:
+    """Pack per-sequence lists of physical block ids into a [B][M] int32
+    table padded with POISON_BLOCK_ID."""
+    bt = torch.full((len(block_lists), max_blocks), POISON_BLOCK_ID, dtype=torch.int32)
+    for b, ids in enumerate(block_lists):
+        if len(ids):
+            bt[b, :len(ids)] = torch.as_tensor(ids, dtype=torch.int32)
+    return bt
+
+
+def slots_for_positions(block_tables: torch.Tensor, positions: torch.Tensor, bs: int) -> torch.Tensor:
+    """Slot of token position p of sequence b: block_tables[b][p // bs] * bs + p % bs
+    (-1 where p < 0).  This is the slot mapping a block manager passes to the
+    append."""
+    B = positions.shape[0]
+    pos = positions.to(torch.int64)
+    valid = pos >= 0
+    safe = torch.where(valid, pos, torch.zeros_like(pos))
+    blk = block_tables.to(torch.int64)[torch.arange(B), safe // bs]
+    slots = blk * bs + safe % bs
+    return torch.where(valid, slots, torch.full_like(slots, -1)).to(torch.int32)
+
+
+def make(name: str, *, poison: bool = False, seed: int | None = None,
+         context_lens=None, num_seqs: int | None = None) -> Workload:
+    """Build configuration ``name``.  ``poison`` fills every cache row no
+    sequence reads with bf16 NaN, so any read past a context shows up.
+    ``context_lens`` / ``num_seqs`` override the drawn lengths (edge cases)."""
+    spec = SPECS[name]
+    g = torch.Generator().manual_seed(spec.seed if seed is None else seed)
+    B = spec.num_seqs if num_seqs is None else num_seqs
+    Hq, Hkv, D, bs = spec.num_q_heads, spec.num_kv_heads, spec.head_dim, spec.block_size
+
+    shared_prefix_blocks = 0
+    if context_lens is not None:
+        lens = torch.as_tensor(context_lens, dtype=torch.int64)
+        B = lens.shape[0]
+    elif name == "tiny":
+        lens = torch.randint(1, 101, (B,), generator=g, dtype=torch.int64)
+    elif name == "qwen3":
+        lens = torch.randint(20, 301, (B,), generator=g, dtype=torch.int64)
+    elif name == "llama32":
+        lens = torch.randint(512, 4097, (B,), generator=g, dtype=torch.int64)
+    elif name == "longskew":
+        lens = torch.full((B,), 1024, dtype=torch.int64)
+        lens[0] = 131072
+    elif name == "prefix":
+        suffix = torch.randint(0, 257, (B,), generator=g, dtype=torch.int64)
+        lens = 1024 + suffix + 1          # shared prefix + private suffix + appended token
+        shared_prefix_blocks = 1024 // bs
+    else:
+        raise KeyError(name)
+
+    pages = _pages(lens, bs)
+    M = max(1, int(pages.max().item()) if B else 1)
+
+    # ---- physical block assignment ------------------------------------
+    if name == "prefix" and context_lens is None:
+        n_groups = 2
+        private = (pages - shared_prefix_blocks).clamp(min=0)
+        need = n_groups * shared_prefix_blocks + int(private.sum().item())
+        NB = need
+        perm = torch.randperm(NB, generator=g).tolist()
+        prefix_ids = [perm[i * shared_prefix_blocks:(i + 1) * shared_prefix_blocks]
+                      for i in range(n_groups)]
+        cursor = n_groups * shared_prefix_blocks
+        lists = []
+        for b in range(B):
+            grp = 0 if b < B // 2 else 1
+            n_priv = int(private[b].item())
+            lists.append(prefix_ids[grp] + perm[cursor:cursor + n_priv])
+            cursor += n_priv
+    else:
+        need = int(pages.sum().item())
+        if name == "tiny" and context_lens is None:
+            NB = 64
+        elif name == "llama32":
+            NB = int(math.ceil(1.5 * need))
+        else:
+            NB = max(need, 1)
+        perm = torch.randperm(NB, generator=g).tolist()
+        lists, cursor = [], 0
+        for b in range(B):
+            n = int(pages[b].item())
+            lists.append(perm[cursor:cursor + n])
+            cursor += n
+    block_tables = build_tables(lists, M)
+
+    # ---- values ----------------------------------------------------------
+    q = _randn_bf16(g, (B, Hq, D))
+    k_cache = _randn_bf16(g, (NB, Hkv, bs, D))
+    v_cache = _randn_bf16(g, (NB, Hkv, bs, D))
+    if name == "longskew":
+        # 1% of (token row, kv head) keys scaled by 8 (a power of two: exact in bf16)
+        outlier = torch.rand((NB, Hkv, bs), generator=g) < 0.01
+        k_cache = torch.where(outlier[..., None], k_cache * 8, k_cache)
+    k_new = _randn_bf16(g, (B, Hkv, D))
+    v_new = _randn_bf16(g, (B, Hkv, D))
+
+    if poison:
+        used = torch.zeros((NB, bs), dtype=torch.bool)
+        for b in range(B):
+            L = int(lens[b].item())
+            for j, blk in enumerate(lists[b]):
+                n_valid = min(bs, L - j * bs)
+                used[blk, :n_valid] = True
+        nan = torch.tensor(BF16_NAN_BITS, dtype=torch.int16).view(torch.bfloat16)
+        mask = (~used)[:, None, :, None].expand(NB, Hkv, bs, D)
+        k_cache = torch.where(mask, nan, k_cache)
+        v_cache = torch.where(mask, nan, v_cache)
+
+    slot_mapping = slots_for_positions(block_tables, lens - 1, bs)
+    return Workload(spec=spec, q=q, k_cache=k_cache.contiguous(), v_cache=v_cache.contiguous(),
+                    block_tables=block_tables, context_lens=lens.to(torch.int32),
+                    k_new=k_new, v_new=v_new, slot_mapping=slot_mapping,
+                    scale=1.0 / math.sqrt(D))
+
+
+def unique_kv_bytes(w: Workload) -> int:
+    """Bytes of distinct K and V rows the decode must read: each physical
+    (block, offset) row inside some context counts once per kv head."""
+    bs = w.spec.block_size
+    D = w.q.shape[2]
+    NB, Hkv = w.k_cache.shape[0], w.k_cache.shape[1]
+    used = torch.zeros(NB * bs, dtype=torch.bool)
+    for b, L in enumerate(w.context_lens.tolist()):
+        if L <= 0:
+            continue
+        t = torch.arange(L)
+        blk = w.block_tables[b, t // bs].to(torch.int64)
+        used[blk * bs + t % bs] = True
+    return int(used.sum().item()) * Hkv * D * 2 * 2
+
+
+def logical_kv_bytes(w: Workload) -> int:
+    """K and V bytes summed over sequences (shared rows counted per reader)."""
+    D = w.q.shape[2]
+    Hkv = w.k_cache.shape[1]
+    return int(w.context_lens.to(torch.int64).sum().item()) * Hkv * D * 2 * 2
+
+
+def qo_bytes(w: Workload) -> int:
+    """q read plus out written, bf16."""
+    return 2 * w.q.numel() * 2
+
+
+def append_bytes(w: Workload) -> int:
+    """k_new/v_new read, their cache rows written, slot ids read."""
+    n_valid = int((w.slot_mapping >= 0).sum().item())
+    per_tok = w.k_new.shape[1] * w.k_new.shape[2] * 2 * 2
+    return 2 * n_valid * per_tok + 4 * w.slot_mapping.numel()
