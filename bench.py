@@ -1,0 +1,387 @@
+"""Benchmark of one decode step of the paged-KV hot path on B200.
+
+A step is the whole path over one synthetic batch: the slot-mapped append
+of each sequence's new K/V token, then paged decode attention (partials and
+merge included).  Prints ONE JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama32]
+    python bench.py --impl reference ...   # the fp64 CPU oracle, timed on host cores
+
+Metric: effective GB/s = algorithmic bytes / device time, where the
+algorithmic bytes of a step are the distinct K/V rows the decode must read
+plus q and out, plus the append's reads and writes.  Kernel times come from
+CUDA events on the launching stream; the L2 is flushed (a 256 MB write)
+between steps, outside the timed events.  With N > 1 (torchrun) every rank
+runs an independent replica of the batch (the path has no exchange step);
+value = bytes of all ranks / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode effective KV GB/s and % of B200 HBM peak; µs per decode call"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llama32",
+                    choices=["tiny", "qwen3", "llama32", "longskew", "prefix"])
+    ap.add_argument("--impl", default="pa", choices=["pa", "reference"])
+    ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return ws, rank, local
+
+
+def _max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    dev = torch.device("cuda") if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(ws: int) -> None:
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "paged_kv_attention_36_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, or None
+    when the kernel sources changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    ent = rec.get(workload)
+    if not ent or ent.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples every 200 ms during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int, enabled: bool):
+        self.proc = None
+        self.idx = device_index
+        if enabled:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={device_index}", f"--query-gpu={self.FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "200"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except (OSError, FileNotFoundError):
+                self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _step_bytes(w):
+    from paged_kv_attention_36_b200 import workloads
+    dec = workloads.unique_kv_bytes(w) + workloads.qo_bytes(w)
+    app = workloads.append_bytes(w)
+    return dec, app
+
+
+def cpu_baseline(w, dec_bytes: int, app_bytes: int, budget_s: float = 12.0):
+    """The oracle, as it stands, on the GPU machine's host cores: full append +
+    decode steps of the same batch, repeated until about budget_s seconds."""
+    import oracle
+    from tests import paging  # bit-pattern views only
+    nthreads = oracle.default_threads()
+    kb, vb = paging.bits(w.k_cache).copy(), paging.bits(w.v_cache).copy()
+    qb = paging.bits(w.q)
+    bt, cl = w.block_tables.numpy(), w.context_lens.numpy()
+    kn, vn, sm = paging.bits(w.k_new), paging.bits(w.v_new), w.slot_mapping.numpy()
+    steps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.append(kn, vn, sm, kb, vb)
+        oracle.decode(qb, kb, vb, bt, cl, w.scale, nthreads=nthreads)
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or steps >= 50:
+            break
+    per_step = el / steps
+    return {"value": round((dec_bytes + app_bytes) / per_step / 1e9, 4), "unit": "GB/s",
+            "cores": nthreads, "kind": "oracle",
+            "sample": f"{steps} full steps (append + decode) of the '{w.spec.name}' batch, "
+                      f"{per_step * 1e3:.1f} ms each, fp64, {nthreads} threads"}
+
+
+def run_reference(args, ws, rank):
+    """--impl reference: the fp64 oracle on the host cores, rank 0 only."""
+    if rank != 0:
+        return
+    from paged_kv_attention_36_b200 import workloads
+    import oracle
+    from tests import paging
+    w = workloads.make(args.workload)
+    dec, app = _step_bytes(w)
+    nthreads = oracle.default_threads()
+    kb, vb = paging.bits(w.k_cache).copy(), paging.bits(w.v_cache).copy()
+    qb = paging.bits(w.q)
+    bt, cl = w.block_tables.numpy(), w.context_lens.numpy()
+    kn, vn, sm = paging.bits(w.k_new), paging.bits(w.v_new), w.slot_mapping.numpy()
+
+    def step():
+        oracle.append(kn, vn, sm, kb, vb)
+        oracle.decode(qb, kb, vb, bt, cl, w.scale, nthreads=nthreads)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    per = el / args.steps
+    value = (dec + app) / per / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(per * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "description": w.spec.description},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": nthreads, "kind": "oracle",
+                         "sample": f"{args.steps} full steps of the '{args.workload}' batch"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_pa(args, ws, rank, local):
+    from paged_kv_attention_36_b200 import binding as pa
+    from paged_kv_attention_36_b200 import workloads
+
+    dev = torch.device("cuda", local if ws > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+    w = workloads.make(args.workload)
+    dec_bytes, app_bytes = _step_bytes(w)
+    step_bytes = dec_bytes + app_bytes
+
+    q, kc, vc = w.q.to(dev), w.k_cache.to(dev), w.v_cache.to(dev)
+    bt, cl = w.block_tables.to(dev), w.context_lens.to(dev)
+    kn, vn, sm = w.k_new.to(dev), w.v_new.to(dev), w.slot_mapping.to(dev)
+    out = torch.empty_like(q)
+    dims = pa.make_dims(q, kc, bt)
+    wsp = pa.alloc_workspace(dims, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        pa.pa_cache_append(kn, vn, sm, kc, vc, stream=stream)
+        pa.pa_decode(q, kc, vc, bt, cl, w.scale, out, workspace=wsp, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+        flush.zero_()
+    torch.cuda.synchronize(dev)
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    clocks = ClockSampler(dev.index, enabled=not args.no_clocks)
+    _barrier(ws)
+    torch.cuda.synchronize(dev)
+    for k in range(K):
+        ev[k][0].record(stream)
+        pa.pa_cache_append(kn, vn, sm, kc, vc, stream=stream)
+        ev[k][1].record(stream)
+        pa.pa_decode(q, kc, vc, bt, cl, w.scale, out, workspace=wsp, stream=stream)
+        ev[k][2].record(stream)
+        flush.zero_()
+    torch.cuda.synchronize(dev)
+    _barrier(ws)
+    clk = clocks.stop()
+    errs = pa.pa_device_errors(clear=True)
+    if errs:
+        raise RuntimeError(f"device error bits {errs:#x} during the benchmark")
+
+    step_ms = [ev[k][0].elapsed_time(ev[k][2]) for k in range(K)]
+    app_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
+    dec_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]
+    total_ms = _max_over_ranks(sum(step_ms), ws)
+    dec_avg = _max_over_ranks(sum(dec_ms) / K, ws)
+    app_avg = _max_over_ranks(sum(app_ms) / K, ws)
+
+    # ---- end to end through the public API from pinned host buffers ----
+    host = {n: t.pin_memory() for n, t in (("q", w.q), ("bt", w.block_tables), ("cl", w.context_lens),
+                                            ("kn", w.k_new), ("vn", w.v_new), ("sm", w.slot_mapping))}
+    out_h = torch.empty(w.q.shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+    dq, dbt, dcl = torch.empty_like(q), torch.empty_like(bt), torch.empty_like(cl)
+    dkn, dvn, dsm = torch.empty_like(kn), torch.empty_like(vn), torch.empty_like(sm)
+
+    def e2e_step():
+        dq.copy_(host["q"], non_blocking=True)
+        dbt.copy_(host["bt"], non_blocking=True)
+        dcl.copy_(host["cl"], non_blocking=True)
+        dkn.copy_(host["kn"], non_blocking=True)
+        dvn.copy_(host["vn"], non_blocking=True)
+        dsm.copy_(host["sm"], non_blocking=True)
+        pa.pa_cache_append(dkn, dvn, dsm, kc, vc, stream=stream)
+        pa.pa_decode(dq, kc, vc, dbt, dcl, w.scale, out, workspace=wsp, stream=stream)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+        flush.zero_()
+    torch.cuda.synchronize(dev)
+    ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    _barrier(ws)
+    torch.cuda.synchronize(dev)
+    for k in range(K):
+        ee[k][0].record(stream)
+        e2e_step()
+        ee[k][1].record(stream)
+        flush.zero_()
+    torch.cuda.synchronize(dev)
+    _barrier(ws)
+    e2e_total = _max_over_ranks(sum(ee[k][0].elapsed_time(ee[k][1]) for k in range(K)), ws)
+
+    if rank != 0:
+        return
+    peak, peak_kind = _peaks()
+    achieved = dec_bytes / (dec_avg * 1e-3) / 1e9
+    value = ws * K * step_bytes / (total_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": ws,
+        "steps": K,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": round(total_ms / K, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "storage_dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "description": w.spec.description,
+                   "num_seqs": w.spec.num_seqs, "q_heads": w.spec.num_q_heads,
+                   "kv_heads": w.spec.num_kv_heads, "head_dim": w.spec.head_dim, "block_size": 16,
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+                   "l2": "flushed between steps (256 MB write, outside the timed events)",
+                   "unique_kv_bytes": workloads.unique_kv_bytes(w),
+                   "logical_kv_bytes": workloads.logical_kv_bytes(w)},
+        "decode_us": round(dec_avg * 1e3, 2),
+        "append_us": round(app_avg * 1e3, 2),
+        "decode_pct_of_hbm_peak": round(100 * achieved / peak, 1),
+        "decode_pct_of_8tbs_nominal": round(100 * achieved / 8000.0, 1),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                     "kernel": "pa::decode_kernel", "traffic": _traffic(args.workload),
+                     "algorithmic_bytes_per_launch": dec_bytes},
+        "e2e": {"value": round(ws * K * step_bytes / (e2e_total * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_total / K, 5)},
+        "gpu_launches": 2 * K,
+        "clocks": clk,
+    }
+    if ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, dec_bytes, app_bytes)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = _args()
+    ws, rank, local = _dist()
+    try:
+        if args.impl == "reference":
+            run_reference(args, ws, rank)
+        else:
+            if not torch.cuda.is_available():
+                raise SystemExit("bench.py needs a CUDA device for --impl pa")
+            run_pa(args, ws, rank, local)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,164 @@
+/*
+ * pa.h -- C ABI of libpa_b200.so: single-token decode attention over a
+ * paged KV cache, and the slot-mapped append of each step's new K/V token,
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The operations follow the pages' statement of the problem, which names
+ * them without a formula (miniVLLM docs index, "What is miniVLLM?": paged
+ * attention for decode, a paged KV cache; "Explore by topic": fixed-size
+ * pages, online softmax; tiny-vllm write-up, "Chi tiet": KV cache,
+ * FlashAttention-style online softmax, PagedAttention).  Written out:
+ *
+ *   for sequence b, query head h, kv head g = h / (Hq / Hkv):
+ *     K_t = k_cache[block_tables[b][t / bs]][g][t % bs][:]      (V_t likewise)
+ *     s_t = scale * dot(q[b][h], K_t)              for t < context_lens[b]
+ *     out[b][h] = sum_t softmax(s)_t * V_t        (bf16, round-to-nearest-even)
+ *
+ * computed with fp32 products, sums and online-softmax state.
+ *
+ * Conventions for every call:
+ *   - Tensor pointers are DEVICE pointers on the current CUDA device, owned
+ *     by the caller; the library never frees or keeps them.  bf16 tensors
+ *     are raw 2-byte values; all are dense, row-major, with the shapes below.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*,
+ *     NULL = legacy default stream) and never synchronise or allocate.
+ *   - Host-side checks (NULL pointers, sizes, alignment, supported shapes)
+ *     return a negative pa_status and launch nothing.
+ *   - Device-side checks (block ids, context lengths, slots) cannot be made
+ *     on the host without a sync; a violation sets a bit in the device
+ *     error word (PA_DEVERR_*), read with pa_device_errors().  The kernel
+ *     never reads or writes out of bounds and never traps; outputs of a call
+ *     that set an error bit are unspecified.
+ *
+ * Layouts:
+ *   q, out           [B][Hq][D] bf16
+ *   k_cache, v_cache [NB][Hkv][bs][D] bf16: one (block, kv head) tile is
+ *                    bs contiguous rows of D values (bs*D*2 bytes)
+ *   block_tables     [B][M] int32; entries past ceil(context_len/bs) are
+ *                    never read
+ *   context_lens     [B] int32, 0 <= L_b <= M*bs (L_b = 0 gives out = 0);
+ *                    decode needs NB >= 1 when B > 0
+ *   k_new, v_new     [T][Hkv][D] bf16
+ *   slot_mapping     [T] int32; slot s writes block s / bs, row s % bs;
+ *                    s < 0 marks padding and is skipped
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pa_status {
+    PA_OK = 0,
+    PA_ERR_NULL = -1,         /* a required pointer is NULL */
+    PA_ERR_SHAPE = -2,        /* a size is negative, zero where it must not be, or inconsistent */
+    PA_ERR_UNSUPPORTED = -3,  /* head_dim / block_size / GQA group not built into this library */
+    PA_ERR_ALIGN = -4,        /* a tensor pointer is not 16-byte aligned */
+    PA_ERR_WORKSPACE = -5,    /* workspace NULL or smaller than pa_decode_workspace_bytes() */
+    PA_ERR_CUDA = -6          /* a CUDA runtime call failed (launch, attribute, device query) */
+} pa_status;
+
+/* Bits of the device error word. */
+#define PA_DEVERR_BLOCK_ID 0x1  /* a block id inside a context was outside [0, num_blocks) */
+#define PA_DEVERR_CONTEXT 0x2   /* a context_len was outside [0, max_blocks_per_seq*block_size] */
+#define PA_DEVERR_SLOT 0x4      /* an append slot was >= num_blocks*block_size */
+#define PA_DEVERR_TIMEOUT 0x8   /* a bounded pipeline wait gave up (internal error) */
+
+typedef struct pa_dims {
+    int32_t num_seqs;           /* B */
+    int32_t num_q_heads;        /* Hq, a multiple of Hkv */
+    int32_t num_kv_heads;       /* Hkv */
+    int32_t head_dim;           /* D */
+    int32_t block_size;         /* bs, tokens per physical block */
+    int32_t num_blocks;         /* NB, physical blocks in the pool */
+    int32_t max_blocks_per_seq; /* M, width of a block_tables row */
+} pa_dims;
+
+/*
+ * Slot-mapped append ("reshape_and_cache"): for every t < num_tokens with
+ * s = slot_mapping[t] >= 0 and every kv head g,
+ *     k_cache[s / bs][g][s % bs][:] = k_new[t][g][:]    (v likewise),
+ * a bit-exact copy.  Used by decode to store the token being generated
+ * before attending over it (a KV-caching engine, miniVLLM review, "What
+ * main.py actually does").  Uses dims->num_kv_heads, head_dim, block_size,
+ * num_blocks; D must be a multiple of 8.  Slots >= NB*bs are skipped and
+ * set PA_DEVERR_SLOT.  Two tokens mapped to one slot: which one lands is
+ * unspecified.
+ */
+PA_API pa_status pa_cache_append(const void* k_new, const void* v_new, const int32_t* slot_mapping,
+                          int32_t num_tokens, void* k_cache, void* v_cache,
+                          const pa_dims* dims, void* stream);
+
+/*
+ * Device workspace pa_decode needs, in bytes, when it runs on `num_ctas`
+ * CTAs (0 = the default grid pa_decode picks on the current device).  The
+ * workspace holds split-KV partial outputs and one merge counter per
+ * (sequence, kv head).  It must be zero-filled once before its first use;
+ * every completed call leaves it ready for the next (the counters return
+ * to zero).  Calls that share one workspace must not overlap on the GPU.
+ * Returns 0 for invalid dims.
+ */
+PA_API size_t pa_decode_workspace_bytes(const pa_dims* dims, int32_t num_ctas);
+
+/* Grid size (CTAs) pa_decode uses on the current device; <= 0 on error. */
+PA_API int32_t pa_decode_default_ctas(void);
+
+/*
+ * Paged decode attention (formula at the top of this file).  One persistent
+ * CTA per SM walks an equal share of all (sequence, kv head, page) work;
+ * all GQA query heads of a kv head share each staged K/V page.  A sequence
+ * whose pages are shared between CTAs is finished by split-KV partials
+ * (flash-decoding) and a log-sum-exp merge done by the last CTA to finish
+ * its part.  Supported: block_size 16; head_dim 64 with Hq/Hkv in
+ * {1, 2, 4, 8}; head_dim 128 with Hq/Hkv in {1, 2, 4}.  q, k_cache,
+ * v_cache and out must be 16-byte aligned.
+ */
+PA_API pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, const int32_t* context_lens, float scale,
+                    void* out, const pa_dims* dims, void* workspace, size_t workspace_bytes,
+                    void* stream);
+
+/*
+ * Test hook: pa_decode on exactly `num_ctas` CTAs (which decides where
+ * contexts are split), that also records every per-CTA segment it computes:
+ * segment i covers tokens [t0, t1) of kv head g of sequence b and stores
+ *     seg_meta[i] = {b, g, t0, t1}                       int32[capacity][4]
+ *     seg_o[i][j][:]  normalised partial output          f32[capacity][G][D]
+ *     seg_m[i][j]     max logit (natural-log units)      f32[capacity][G]
+ *     seg_l[i][j]     sum_t exp(s_t - seg_m[i][j])       f32[capacity][G]
+ * for the G = Hq/Hkv query heads j of kv head g.  *seg_count (device,
+ * zeroed by the caller) receives the number of segments; entries past
+ * `capacity` are dropped.  `out` is computed as by pa_decode.  The
+ * workspace must be sized with pa_decode_workspace_bytes(dims, num_ctas).
+ */
+PA_API pa_status pa_decode_partials(const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_tables, const int32_t* context_lens,
+                             float scale, void* out, const pa_dims* dims, int32_t num_ctas,
+                             void* workspace, size_t workspace_bytes, int32_t capacity,
+                             int32_t* seg_meta, float* seg_o, float* seg_m, float* seg_l,
+                             int32_t* seg_count, void* stream);
+
+/*
+ * Reads (and, if `clear` != 0, resets) the device error word of the
+ * current device.  Synchronous: waits for all prior work on the device.
+ */
+PA_API pa_status pa_device_errors(int32_t* errors_out, int32_t clear);
+
+/* Static, human-readable name of a pa_status value. */
+PA_API const char* pa_status_string(int32_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

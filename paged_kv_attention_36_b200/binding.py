@@ -1,0 +1,205 @@
+"""ctypes binding of libpa_b200.so (the C ABI declared in include/pa.h).
+
+Argument marshalling only: every function checks the tensors' dtype,
+device and contiguity, turns them into raw pointers plus a ``pa_dims``
+struct and the current CUDA stream, calls the C entry point of the same
+name, and raises ``PaError`` on a non-zero status.  All computation runs in
+the library's CUDA kernels; if the library is missing this module raises at
+import time instead of falling back to anything else.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpa_b200.so")
+
+PA_DEVERR_BLOCK_ID = 0x1
+PA_DEVERR_CONTEXT = 0x2
+PA_DEVERR_SLOT = 0x4
+PA_DEVERR_TIMEOUT = 0x8
+
+
+class PaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {pa_status_string(code)} ({code})")
+        self.code = code
+
+
+class pa_dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "num_seqs", "num_q_heads", "num_kv_heads", "head_dim", "block_size", "num_blocks",
+        "max_blocks_per_seq")]
+
+    def __repr__(self):
+        return "pa_dims(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m paged_kv_attention_36_b200.build` "
+            "(there is no fallback implementation)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, sz, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_float
+    dp = ctypes.POINTER(pa_dims)
+    lib.pa_cache_append.argtypes = [vp, vp, vp, i32, vp, vp, dp, vp]
+    lib.pa_cache_append.restype = i32
+    lib.pa_decode_workspace_bytes.argtypes = [dp, i32]
+    lib.pa_decode_workspace_bytes.restype = sz
+    lib.pa_decode_default_ctas.argtypes = []
+    lib.pa_decode_default_ctas.restype = i32
+    lib.pa_decode.argtypes = [vp, vp, vp, vp, vp, f32, vp, dp, vp, sz, vp]
+    lib.pa_decode.restype = i32
+    lib.pa_decode_partials.argtypes = [vp, vp, vp, vp, vp, f32, vp, dp, i32, vp, sz, i32,
+                                       vp, vp, vp, vp, vp, vp]
+    lib.pa_decode_partials.restype = i32
+    lib.pa_device_errors.argtypes = [ctypes.POINTER(i32), i32]
+    lib.pa_device_errors.restype = i32
+    lib.pa_status_string.argtypes = [i32]
+    lib.pa_status_string.restype = ctypes.c_char_p
+    return lib
+
+
+lib = _load()
+
+# Every symbol include/pa.h declares.
+EXPORTS = ("pa_cache_append", "pa_decode_workspace_bytes", "pa_decode_default_ctas", "pa_decode",
+           "pa_decode_partials", "pa_device_errors", "pa_status_string")
+
+
+def pa_status_string(code: int) -> str:
+    return lib.pa_status_string(int(code)).decode()
+
+
+def _check(code: int, what: str) -> None:
+    if code != 0:
+        raise PaError(code, what)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, dtype, name, ndim=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+
+
+def make_dims(q: torch.Tensor, k_cache: torch.Tensor, block_tables: torch.Tensor) -> pa_dims:
+    """pa_dims from q [B][Hq][D], a cache [NB][Hkv][bs][D] and block_tables [B][M]."""
+    B, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_cache.shape
+    if D2 != D or block_tables.shape[0] != B:
+        raise ValueError("q, cache and block_tables shapes disagree")
+    return pa_dims(B, Hq, Hkv, D, bs, NB, block_tables.shape[1])
+
+
+def pa_decode_workspace_bytes(dims: pa_dims, num_ctas: int = 0) -> int:
+    n = lib.pa_decode_workspace_bytes(ctypes.byref(dims), int(num_ctas))
+    if n == 0:
+        raise ValueError(f"invalid dims {dims!r}")
+    return int(n)
+
+
+def pa_decode_default_ctas() -> int:
+    n = lib.pa_decode_default_ctas()
+    if n <= 0:
+        raise RuntimeError("no CUDA device")
+    return int(n)
+
+
+def alloc_workspace(dims: pa_dims, num_ctas: int = 0, device=None) -> torch.Tensor:
+    """A zero-filled device workspace (the C ABI never allocates)."""
+    return torch.zeros(pa_decode_workspace_bytes(dims, num_ctas), dtype=torch.uint8,
+                       device=device if device is not None else torch.device("cuda"))
+
+
+def pa_cache_append(k_new, v_new, slot_mapping, k_cache, v_cache, stream=None) -> None:
+    """k_cache[s // bs][g][s % bs] = k_new[t][g] (v likewise) for s = slot_mapping[t] >= 0."""
+    for t, n in ((k_new, "k_new"), (v_new, "v_new")):
+        _need(t, torch.bfloat16, n, 3)
+    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, torch.bfloat16, n, 4)
+    _need(slot_mapping, torch.int32, "slot_mapping", 1)
+    T = slot_mapping.shape[0]
+    if k_new.shape != v_new.shape or k_new.shape[0] != T or k_cache.shape != v_cache.shape:
+        raise ValueError("append shapes disagree")
+    NB, Hkv, bs, D = k_cache.shape
+    if k_new.shape[1:] != (Hkv, D):
+        raise ValueError("k_new rows must be [Hkv][D] of the cache")
+    dims = pa_dims(0, Hkv, Hkv, D, bs, NB, 0)
+    _check(lib.pa_cache_append(_ptr(k_new), _ptr(v_new), _ptr(slot_mapping), T, _ptr(k_cache),
+                               _ptr(v_cache), ctypes.byref(dims), _stream(stream)), "pa_cache_append")
+
+
+def _decode_args(q, k_cache, v_cache, block_tables, context_lens, out):
+    _need(q, torch.bfloat16, "q", 3)
+    _need(out, torch.bfloat16, "out", 3)
+    _need(k_cache, torch.bfloat16, "k_cache", 4)
+    _need(v_cache, torch.bfloat16, "v_cache", 4)
+    _need(block_tables, torch.int32, "block_tables", 2)
+    _need(context_lens, torch.int32, "context_lens", 1)
+    if out.shape != q.shape or k_cache.shape != v_cache.shape or context_lens.shape[0] != q.shape[0]:
+        raise ValueError("decode shapes disagree")
+    return make_dims(q, k_cache, block_tables)
+
+
+def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale: float, out,
+              workspace=None, stream=None) -> None:
+    """out = paged decode attention (see include/pa.h).  ``workspace`` is a
+    zero-initialised uint8 device tensor of pa_decode_workspace_bytes(dims)
+    bytes; one is allocated when omitted."""
+    dims = _decode_args(q, k_cache, v_cache, block_tables, context_lens, out)
+    if workspace is None:
+        workspace = alloc_workspace(dims, device=q.device)
+    _need(workspace, torch.uint8, "workspace", 1)
+    _check(lib.pa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                         _ptr(context_lens), float(scale), _ptr(out), ctypes.byref(dims),
+                         _ptr(workspace), workspace.numel(), _stream(stream)), "pa_decode")
+
+
+def pa_decode_partials(q, k_cache, v_cache, block_tables, context_lens, scale: float, out,
+                       num_ctas: int, workspace, capacity: int, seg_meta, seg_o, seg_m, seg_l,
+                       seg_count, stream=None) -> None:
+    """Test hook: pa_decode on ``num_ctas`` CTAs that records each segment's
+    split-KV partials (see include/pa.h)."""
+    dims = _decode_args(q, k_cache, v_cache, block_tables, context_lens, out)
+    _need(workspace, torch.uint8, "workspace", 1)
+    _need(seg_meta, torch.int32, "seg_meta", 2)
+    _need(seg_o, torch.float32, "seg_o", 3)
+    _need(seg_m, torch.float32, "seg_m", 2)
+    _need(seg_l, torch.float32, "seg_l", 2)
+    _need(seg_count, torch.int32, "seg_count", 1)
+    G = dims.num_q_heads // dims.num_kv_heads
+    if seg_meta.shape[0] < capacity or seg_o.shape[0] < capacity or seg_o.shape[1:] != (G, dims.head_dim):
+        raise ValueError("segment buffers smaller than capacity")
+    _check(lib.pa_decode_partials(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                                  _ptr(context_lens), float(scale), _ptr(out), ctypes.byref(dims),
+                                  int(num_ctas), _ptr(workspace), workspace.numel(), int(capacity),
+                                  _ptr(seg_meta), _ptr(seg_o), _ptr(seg_m), _ptr(seg_l),
+                                  _ptr(seg_count), _stream(stream)), "pa_decode_partials")
+
+
+def pa_device_errors(clear: bool = False) -> int:
+    """PA_DEVERR_* bits set on the current device since the last clear (synchronises)."""
+    v = ctypes.c_int32(0)
+    _check(lib.pa_device_errors(ctypes.byref(v), int(bool(clear))), "pa_device_errors")
+    return int(v.value)

@@ -1,0 +1,268 @@
+// pa_api.cu -- the extern "C" entry points of libpa_b200.so (declared and
+// documented in include/pa.h): host-side validation, workspace layout,
+// grid choice and kernel dispatch.  Every step of the computation runs in
+// the kernels of pa_append.cuh and pa_decode.cuh; there is no host or CPU
+// fallback.
+#include <mutex>
+
+#include "pa_append.cuh"
+#include "pa_decode.cuh"
+#include "pa_device.cuh"
+
+namespace {
+
+constexpr int kBlockSize = 16;  // tokens per physical block the decode kernels are built for
+constexpr int kMinPagesPerCta = 8;
+constexpr int kMaxDevices = 64;
+constexpr float kLog2e = 1.4426950408889634f;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// Per-shape tuning.  Registers are split between the SM's four
+// sub-partitions, so a CTA of 12 warps (11 consumers + the producer) caps a
+// thread at 168 registers and one of 8 warps at 255.  Shapes whose
+// per-warp state (q and the accumulator, 2*G*D/8 floats per lane) fits use
+// 11 consumer warps; G*D = 512 uses 7.  The ring depth R is a multiple of
+// W (each stage always feeds the same warp) holding 110-170 KB of K+V.
+template <int D, int G>
+struct Tune {
+    static constexpr int W = (G * D >= 512) ? 7 : 11;  // consumer warps
+    static constexpr int R = D == 64 ? (W == 11 ? 33 : 28) : (W == 11 ? 22 : 21);  // ring stages
+};
+
+bool supported(int D, int G) {
+    if (D == 64) return G == 1 || G == 2 || G == 4 || G == 8;
+    if (D == 128) return G == 1 || G == 2 || G == 4;
+    return false;
+}
+
+std::mutex g_mu;
+int g_sms[kMaxDevices];
+
+int current_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    return dev;
+}
+
+int sm_count() {
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return -1;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_sms[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return -1;
+        g_sms[dev] = n;
+    }
+    return g_sms[dev];
+}
+
+// Workspace layout: [counters: B*Hkv int32][part_o: grid*2*G*D f32][part_ml: grid*2*G float2]
+struct WsLayout {
+    size_t counters, part_o, part_ml, total;
+};
+
+WsLayout ws_layout(const pa_dims& d, int grid) {
+    const size_t G = size_t(d.num_q_heads / d.num_kv_heads);
+    WsLayout w;
+    w.counters = 0;
+    w.part_o = align_up(size_t(d.num_seqs) * d.num_kv_heads * 4, 256);
+    w.part_ml = align_up(w.part_o + size_t(grid) * 2 * G * d.head_dim * 4, 256);
+    w.total = align_up(w.part_ml + size_t(grid) * 2 * G * 8, 256);
+    return w;
+}
+
+bool dims_ok(const pa_dims* d) {
+    return d && d->num_seqs >= 0 && d->num_q_heads > 0 && d->num_kv_heads > 0 && d->head_dim > 0 &&
+           d->block_size > 0 && d->num_blocks >= 0 && d->max_blocks_per_seq >= 0 &&
+           d->num_q_heads % d->num_kv_heads == 0;
+}
+
+template <typename Kernel>
+bool set_smem_once(Kernel kern, int bytes, unsigned* done_mask_per_device) {
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return false;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!done_mask_per_device[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+            return false;
+        done_mask_per_device[dev] = 1;
+    }
+    return true;
+}
+
+template <int D, int G, bool DUMP>
+pa_status launch_decode(const pa::DecodeParams& p, int grid, cudaStream_t stream) {
+    constexpr int W = Tune<D, G>::W, R = Tune<D, G>::R;
+    using Cfg = pa::DecodeCfg<D, G, kBlockSize, W, R>;
+    auto kern = pa::decode_kernel<D, G, kBlockSize, W, R, DUMP>;
+    static unsigned attr_done[kMaxDevices];
+    if (!set_smem_once(kern, Cfg::kSmemBytes, attr_done)) return PA_ERR_CUDA;
+    kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <bool DUMP>
+pa_status dispatch_decode(int D, int G, const pa::DecodeParams& p, int grid, cudaStream_t s) {
+    if (D == 64) {
+        switch (G) {
+            case 1: return launch_decode<64, 1, DUMP>(p, grid, s);
+            case 2: return launch_decode<64, 2, DUMP>(p, grid, s);
+            case 4: return launch_decode<64, 4, DUMP>(p, grid, s);
+            case 8: return launch_decode<64, 8, DUMP>(p, grid, s);
+        }
+    } else if (D == 128) {
+        switch (G) {
+            case 1: return launch_decode<128, 1, DUMP>(p, grid, s);
+            case 2: return launch_decode<128, 2, DUMP>(p, grid, s);
+            case 4: return launch_decode<128, 4, DUMP>(p, grid, s);
+        }
+    }
+    return PA_ERR_UNSUPPORTED;
+}
+
+// Shared validation of pa_decode and pa_decode_partials; fills p.
+pa_status prepare_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                         const int32_t* context_lens, float scale, void* out, const pa_dims* dims, int grid,
+                         void* workspace, size_t workspace_bytes, pa::DecodeParams& p) {
+    if (!dims) return PA_ERR_NULL;
+    if (!dims_ok(dims)) return PA_ERR_SHAPE;
+    const pa_dims& d = *dims;
+    const int G = d.num_q_heads / d.num_kv_heads;
+    if (d.block_size != kBlockSize || !supported(d.head_dim, G)) return PA_ERR_UNSUPPORTED;
+    if (d.num_seqs == 0) return PA_OK;
+    // at least one block, so that a bad block id can be redirected to block 0
+    if (d.num_blocks == 0) return PA_ERR_SHAPE;
+    if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out || !workspace) return PA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(out) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned16(workspace) || !aligned4(block_tables) || !aligned4(context_lens))
+        return PA_ERR_ALIGN;
+    if (grid <= 0) return PA_ERR_CUDA;
+    const WsLayout w = ws_layout(d, grid);
+    if (workspace_bytes < w.total) return PA_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p = pa::DecodeParams{};
+    p.q = static_cast<const uint8_t*>(q);
+    p.k_cache = static_cast<const uint8_t*>(k_cache);
+    p.v_cache = static_cast<const uint8_t*>(v_cache);
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.qscale = scale * kLog2e;
+    p.B = d.num_seqs;
+    p.Hq = d.num_q_heads;
+    p.Hkv = d.num_kv_heads;
+    p.NB = d.num_blocks;
+    p.M = d.max_blocks_per_seq;
+    p.min_pages = kMinPagesPerCta;
+    p.counters = reinterpret_cast<int32_t*>(ws + w.counters);
+    p.part_o = reinterpret_cast<float*>(ws + w.part_o);
+    p.part_ml = reinterpret_cast<float2*>(ws + w.part_ml);
+    return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pa_status_string(int32_t status) {
+    switch (status) {
+        case PA_OK: return "PA_OK";
+        case PA_ERR_NULL: return "PA_ERR_NULL: a required pointer is NULL";
+        case PA_ERR_SHAPE: return "PA_ERR_SHAPE: invalid or inconsistent sizes";
+        case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED: head_dim/block_size/GQA group not built";
+        case PA_ERR_ALIGN: return "PA_ERR_ALIGN: tensor pointer not 16-byte aligned";
+        case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE: workspace missing or too small";
+        case PA_ERR_CUDA: return "PA_ERR_CUDA: CUDA runtime call failed";
+        default: return "unknown pa_status";
+    }
+}
+
+pa_status pa_cache_append(const void* k_new, const void* v_new, const int32_t* slot_mapping, int32_t num_tokens,
+                          void* k_cache, void* v_cache, const pa_dims* dims, void* stream) {
+    if (!dims) return PA_ERR_NULL;
+    const pa_dims& d = *dims;
+    if (num_tokens < 0 || d.num_kv_heads <= 0 || d.head_dim <= 0 || d.block_size <= 0 || d.num_blocks < 0)
+        return PA_ERR_SHAPE;
+    if (d.head_dim % 8 != 0) return PA_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return PA_OK;
+    if (!k_new || !v_new || !slot_mapping || !k_cache || !v_cache) return PA_ERR_NULL;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned4(slot_mapping))
+        return PA_ERR_ALIGN;
+    pa::AppendParams p;
+    p.k_new = static_cast<const uint4*>(k_new);
+    p.v_new = static_cast<const uint4*>(v_new);
+    p.slot_mapping = slot_mapping;
+    p.k_cache = static_cast<uint4*>(k_cache);
+    p.v_cache = static_cast<uint4*>(v_cache);
+    p.chunks_per_row = d.head_dim / 8;
+    p.num_chunks = int64_t(num_tokens) * d.num_kv_heads * p.chunks_per_row;
+    p.kv_heads = d.num_kv_heads;
+    p.block_size = d.block_size;
+    p.num_blocks = d.num_blocks;
+    const int64_t blocks = (p.num_chunks + pa::kAppendThreads - 1) / pa::kAppendThreads;
+    if (blocks > 0x7fffffff) return PA_ERR_SHAPE;
+    pa::append_kernel<<<unsigned(blocks), pa::kAppendThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int32_t pa_decode_default_ctas(void) { return sm_count(); }
+
+size_t pa_decode_workspace_bytes(const pa_dims* dims, int32_t num_ctas) {
+    if (!dims_ok(dims)) return 0;
+    const int grid = num_ctas > 0 ? num_ctas : sm_count();
+    if (grid <= 0) return 0;
+    return ws_layout(*dims, grid).total;
+}
+
+pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                    const int32_t* context_lens, float scale, void* out, const pa_dims* dims, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+    pa::DecodeParams p;
+    const int grid = sm_count();
+    const pa_status st = prepare_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, dims,
+                                        grid, workspace, workspace_bytes, p);
+    if (st != PA_OK || dims->num_seqs == 0) return st;
+    return dispatch_decode<false>(dims->head_dim, dims->num_q_heads / dims->num_kv_heads, p, grid,
+                                  static_cast<cudaStream_t>(stream));
+}
+
+pa_status pa_decode_partials(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                             const int32_t* context_lens, float scale, void* out, const pa_dims* dims,
+                             int32_t num_ctas, void* workspace, size_t workspace_bytes, int32_t capacity,
+                             int32_t* seg_meta, float* seg_o, float* seg_m, float* seg_l, int32_t* seg_count,
+                             void* stream) {
+    if (num_ctas <= 0 || capacity < 0) return PA_ERR_SHAPE;
+    pa::DecodeParams p;
+    const pa_status st = prepare_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, dims,
+                                        num_ctas, workspace, workspace_bytes, p);
+    if (st != PA_OK || dims->num_seqs == 0) return st;
+    if (!seg_count || (capacity > 0 && (!seg_meta || !seg_o || !seg_m || !seg_l))) return PA_ERR_NULL;
+    p.min_pages = 1;
+    p.dump_capacity = capacity;
+    p.seg_meta = seg_meta;
+    p.seg_o = seg_o;
+    p.seg_m = seg_m;
+    p.seg_l = seg_l;
+    p.seg_count = seg_count;
+    return dispatch_decode<true>(dims->head_dim, dims->num_q_heads / dims->num_kv_heads, p, num_ctas,
+                                 static_cast<cudaStream_t>(stream));
+}
+
+pa_status pa_device_errors(int32_t* errors_out, int32_t clear) {
+    if (!errors_out) return PA_ERR_NULL;
+    if (cudaDeviceSynchronize() != cudaSuccess) return PA_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, pa::g_device_errors, sizeof v) != cudaSuccess) return PA_ERR_CUDA;
+    *errors_out = int32_t(v);
+    if (clear) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(pa::g_device_errors, &zero, sizeof zero) != cudaSuccess) return PA_ERR_CUDA;
+    }
+    return PA_OK;
+}
+
+}  // extern "C"

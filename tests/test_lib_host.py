@@ -1,0 +1,106 @@
+"""CPU-side checks of the C-ABI library: it loads, exports every symbol
+include/pa.h declares, and its host-side validation rejects bad arguments
+before touching a GPU.  No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def binding():
+    from paged_kv_attention_36_b200 import build
+    build.build()
+    from paged_kv_attention_36_b200 import binding
+    return binding
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "pa.h")).read()
+    return sorted(set(re.findall(r"PA_API\s+[\w\s\*]+?\b(pa_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("pa_cache_append", "pa_decode", "pa_decode_workspace_bytes"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(binding):
+    declared = _declared()
+    assert sorted(binding.EXPORTS) == declared
+    for n in declared:
+        assert hasattr(binding.lib, n), n
+
+
+def test_status_strings(binding):
+    for code in range(0, -7, -1):
+        s = binding.pa_status_string(code)
+        assert s and "unknown" not in s
+    assert "unknown" in binding.pa_status_string(-99)
+
+
+def _dims(binding, **kw):
+    d = dict(num_seqs=4, num_q_heads=8, num_kv_heads=2, head_dim=64, block_size=16,
+             num_blocks=64, max_blocks_per_seq=7)
+    d.update(kw)
+    return binding.pa_dims(*[d[n] for n, _ in binding.pa_dims._fields_])
+
+
+def _decode(binding, dims, q=16, k=16, v=16, bt=16, cl=16, out=16, ws=16, ws_bytes=1 << 30):
+    vp = ctypes.c_void_p
+    return binding.lib.pa_decode(vp(q), vp(k), vp(v), vp(bt), vp(cl), 0.125, vp(out),
+                                 ctypes.byref(dims) if dims is not None else None, vp(ws), ws_bytes,
+                                 vp(0))
+
+
+def test_decode_host_validation(binding):
+    # fake, never-dereferenced addresses: validation fails before any CUDA call
+    assert _decode(binding, None) == -1                                   # NULL dims
+    assert _decode(binding, _dims(binding, num_q_heads=6, num_kv_heads=4)) == -2
+    assert _decode(binding, _dims(binding, head_dim=96)) == -3
+    assert _decode(binding, _dims(binding, block_size=32)) == -3
+    assert _decode(binding, _dims(binding, num_q_heads=16, num_kv_heads=1, head_dim=128)) == -3
+    assert _decode(binding, _dims(binding, num_blocks=0)) == -2
+    assert _decode(binding, _dims(binding), q=0) == -1
+    assert _decode(binding, _dims(binding), out=8) == -4                 # misaligned
+    assert _decode(binding, _dims(binding, num_seqs=0)) == 0             # nothing to do
+
+
+def test_append_host_validation(binding):
+    vp = ctypes.c_void_p
+    d = _dims(binding)
+    f = binding.lib.pa_cache_append
+    assert f(vp(16), vp(16), vp(16), 3, vp(16), vp(16), None, vp(0)) == -1
+    assert f(vp(16), vp(16), vp(16), -1, vp(16), vp(16), ctypes.byref(d), vp(0)) == -2
+    assert f(vp(16), vp(16), vp(16), 3, vp(16), vp(16), ctypes.byref(_dims(binding, head_dim=12)),
+             vp(0)) == -3
+    assert f(vp(16), vp(0), vp(16), 3, vp(16), vp(16), ctypes.byref(d), vp(0)) == -1
+    assert f(vp(16), vp(24), vp(16), 3, vp(16), vp(16), ctypes.byref(d), vp(0)) == -4
+    assert f(vp(0), vp(0), vp(0), 0, vp(0), vp(0), ctypes.byref(d), vp(0)) == 0
+
+
+def test_workspace_size_formula(binding):
+    # counters (B*Hkv int32) + per-CTA two partial slots (G*D floats + G (m, l) pairs)
+    d = _dims(binding, num_seqs=64, num_q_heads=32, num_kv_heads=8, head_dim=128)
+    n = binding.pa_decode_workspace_bytes(d, 148)
+    G = 4
+    need = 64 * 8 * 4 + 148 * 2 * G * 128 * 4 + 148 * 2 * G * 8
+    assert need <= n <= need + 3 * 256
+    with pytest.raises(ValueError):
+        binding.pa_decode_workspace_bytes(_dims(binding, num_kv_heads=3), 148)
+
+
+def test_binding_rejects_host_tensors(binding):
+    q = torch.zeros((1, 2, 64), dtype=torch.bfloat16)
+    kc = torch.zeros((1, 1, 16, 64), dtype=torch.bfloat16)
+    bt = torch.zeros((1, 1), dtype=torch.int32)
+    cl = torch.ones(1, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.pa_decode(q, kc, kc, bt, cl, 0.125, q.clone(), workspace=torch.zeros(8, dtype=torch.uint8))
+    with pytest.raises(TypeError):
+        binding.pa_decode(q.float(), kc, kc, bt, cl, 0.125, q.clone())
