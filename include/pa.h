@@ -119,9 +119,12 @@ PA_API int32_t pa_decode_default_ctas(void);
  * all GQA query heads of a kv head share each staged K/V page.  A sequence
  * whose pages are shared between CTAs is finished by split-KV partials
  * (flash-decoding) and a log-sum-exp merge done by the last CTA to finish
- * its part.  Supported: block_size 16; head_dim 64 with Hq/Hkv in
- * {1, 2, 4, 8}; head_dim 128 with Hq/Hkv in {1, 2, 4}.  q, k_cache,
- * v_cache and out must be 16-byte aligned.
+ * its part.  Supported: block_size 16, head_dim 64 or 128, Hq/Hkv in
+ * {1, 2, 4, 8}; fewer than 2^31 cache rows (NB*Hkv*bs).  q, k_cache,
+ * v_cache and out must be 16-byte aligned.  The per-page math runs on the
+ * tensor cores (mma.sync, fp32 accumulation); setting the environment
+ * variable PA_DECODE_MATH=simt before the first call selects the fp32 CUDA
+ * core variant instead (head_dim*Hq/Hkv <= 512 only).
  */
 PA_API pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
                     const int32_t* block_tables, const int32_t* context_lens, float scale,

@@ -38,12 +38,12 @@ class pa_dims(ctypes.Structure):
         return "pa_dims(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
 
 
-def _load():
-    if not os.path.exists(LIB_PATH):
+def _load(path: str = LIB_PATH):
+    if not os.path.exists(path):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m paged_kv_attention_36_b200.build` "
+            f"{path} is missing: build it with `python -m paged_kv_attention_36_b200.build` "
             "(there is no fallback implementation)")
-    lib = ctypes.CDLL(LIB_PATH)
+    lib = ctypes.CDLL(path)
     vp, i32, sz, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_float
     dp = ctypes.POINTER(pa_dims)
     lib.pa_cache_append.argtypes = [vp, vp, vp, i32, vp, vp, dp, vp]
@@ -203,3 +203,45 @@ def pa_device_errors(clear: bool = False) -> int:
     v = ctypes.c_int32(0)
     _check(lib.pa_device_errors(ctypes.byref(v), int(bool(clear))), "pa_device_errors")
     return int(v.value)
+
+
+class Prepared:
+    """A pa_cache_append / pa_decode call with its arguments marshalled
+    once: calling it re-issues the same C call on the same tensors (their
+    contents may change between calls, their storage may not).  Used where
+    per-call Python overhead would otherwise leave the GPU idle."""
+
+    def __init__(self, fn, args, what):
+        self._fn, self._args, self._what, self._keep = fn, args, what, None
+
+    def __call__(self):
+        code = self._fn(*self._args)
+        if code != 0:
+            raise PaError(code, self._what)
+
+
+def prepare_append(k_new, v_new, slot_mapping, k_cache, v_cache, stream=None) -> Prepared:
+    for t, n in ((k_new, "k_new"), (v_new, "v_new")):
+        _need(t, torch.bfloat16, n, 3)
+    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, torch.bfloat16, n, 4)
+    _need(slot_mapping, torch.int32, "slot_mapping", 1)
+    NB, Hkv, bs, D = k_cache.shape
+    dims = pa_dims(0, Hkv, Hkv, D, bs, NB, 0)
+    p = Prepared(lib.pa_cache_append,
+                 (_ptr(k_new), _ptr(v_new), _ptr(slot_mapping), slot_mapping.shape[0], _ptr(k_cache),
+                  _ptr(v_cache), ctypes.byref(dims), _stream(stream)), "pa_cache_append")
+    p._keep = (dims, k_new, v_new, slot_mapping, k_cache, v_cache)
+    return p
+
+
+def prepare_decode(q, k_cache, v_cache, block_tables, context_lens, scale: float, out, workspace,
+                   stream=None) -> Prepared:
+    dims = _decode_args(q, k_cache, v_cache, block_tables, context_lens, out)
+    _need(workspace, torch.uint8, "workspace", 1)
+    p = Prepared(lib.pa_decode,
+                 (_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+                  float(scale), _ptr(out), ctypes.byref(dims), _ptr(workspace), workspace.numel(),
+                  _stream(stream)), "pa_decode")
+    p._keep = (dims, q, k_cache, v_cache, block_tables, context_lens, out, workspace)
+    return p

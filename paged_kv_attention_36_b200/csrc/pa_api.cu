@@ -3,6 +3,10 @@
 // grid choice and kernel dispatch.  Every step of the computation runs in
 // the kernels of pa_append.cuh and pa_decode.cuh; there is no host or CPU
 // fallback.
+#include <cudaTypedefs.h>
+
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "pa_append.cuh"
@@ -20,22 +24,55 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
-// Per-shape tuning.  Registers are split between the SM's four
-// sub-partitions, so a CTA of 12 warps (11 consumers + the producer) caps a
-// thread at 168 registers and one of 8 warps at 255.  Shapes whose
-// per-warp state (q and the accumulator, 2*G*D/8 floats per lane) fits use
-// 11 consumer warps; G*D = 512 uses 7.  The ring depth R is a multiple of
-// W (each stage always feeds the same warp) holding 110-170 KB of K+V.
+// Per-shape tuning of the two math policies.
+//  SIMT: registers are split between the SM's four sub-partitions, so a CTA
+//    of 12 warps (11 consumers + the producer) caps a thread at 168
+//    registers and one of 8 warps at 255; G*D = 512 needs the latter.
+//  MMA: the per-lane state is small (2*D/16 fragment registers), 8
+//    consumer warps.
+// The ring depth R is a multiple of the consumer warps (each stage always
+// feeds the same warp) and holds 110-170 KB of K+V pages.
+enum class MathKind { kMma, kSimt };
+
+template <MathKind MK, int D, int G>
+struct Tune;
 template <int D, int G>
-struct Tune {
-    static constexpr int W = (G * D >= 512) ? 7 : 11;  // consumer warps
-    static constexpr int R = D == 64 ? (W == 11 ? 33 : 28) : (W == 11 ? 22 : 21);  // ring stages
+struct Tune<MathKind::kSimt, D, G> {
+    static constexpr int NW = (G * D >= 512) ? 7 : 11;
+    static constexpr int R = D == 64 ? (NW == 11 ? 33 : 28) : (NW == 11 ? 22 : 21);
+};
+#ifndef PA_MMA_NW
+#define PA_MMA_NW 8
+#endif
+#ifndef PA_MAX_RING
+#define PA_MAX_RING 64
+#endif
+// Deepest ring (a multiple of NW, at most PA_MAX_RING) whose CTA fits in shared memory.
+template <int D, int G, int NW>
+constexpr int ring_fit() {
+    int r = (PA_MAX_RING / NW) * NW;
+    while (r > NW && pa::DecodeCfg<D, G, kBlockSize, NW, 1>::kSmemBytes + (r - 1) * (2 * 16 * D * 2 + 16) > 232448)
+        r -= NW;
+    return r;
+}
+template <int D, int G>
+struct Tune<MathKind::kMma, D, G> {
+    static constexpr int NW = PA_MMA_NW;
+    static constexpr int R = ring_fit<D, G, NW>();
 };
 
-bool supported(int D, int G) {
-    if (D == 64) return G == 1 || G == 2 || G == 4 || G == 8;
-    if (D == 128) return G == 1 || G == 2 || G == 4;
-    return false;
+MathKind math_kind() {
+    static const MathKind k = [] {
+        const char* e = std::getenv("PA_DECODE_MATH");
+        return (e && std::strcmp(e, "simt") == 0) ? MathKind::kSimt : MathKind::kMma;
+    }();
+    return k;
+}
+
+bool supported(int D, int G, MathKind mk) {
+    if (D != 64 && D != 128) return false;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return false;
+    return mk == MathKind::kMma || G * D <= 512;
 }
 
 std::mutex g_mu;
@@ -93,34 +130,81 @@ bool set_smem_once(Kernel kern, int bytes, unsigned* done_mask_per_device) {
     return true;
 }
 
-template <int D, int G, bool DUMP>
+#ifndef PA_L2_PROMOTION
+#define PA_L2_PROMOTION CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+#endif
+
+// cuTensorMapEncodeTiled from the driver, found through the runtime.
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// A cache [NB][Hkv][bs][D] bf16 seen as a 3-D tensor {64 columns, D/64
+// panels, NB*Hkv*bs rows} (strides 128 B and D*2 B); one box is one
+// 64-column panel of one (block, kv head) tile: {64, 1, bs}, 128-byte swizzle.
+bool make_cache_map(CUtensorMap* map, const void* base, int64_t rows, int D, int bs) {
+    auto fn = encode_tiled();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {64, cuuint64_t(D / 64), cuuint64_t(rows)};
+    cuuint64_t strides[2] = {128, cuuint64_t(D) * 2};
+    cuuint32_t box[3] = {64, 1, cuuint32_t(bs)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, PA_L2_PROMOTION,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <MathKind MK, int D, int G, bool DUMP>
 pa_status launch_decode(const pa::DecodeParams& p, int grid, cudaStream_t stream) {
-    constexpr int W = Tune<D, G>::W, R = Tune<D, G>::R;
-    using Cfg = pa::DecodeCfg<D, G, kBlockSize, W, R>;
-    auto kern = pa::decode_kernel<D, G, kBlockSize, W, R, DUMP>;
+    constexpr int NW = Tune<MK, D, G>::NW, R = Tune<MK, D, G>::R;
+    using Cfg = pa::DecodeCfg<D, G, kBlockSize, NW, R>;
+    auto kern = [] {
+        if constexpr (MK == MathKind::kMma)
+            return pa::decode_kernel<D, G, kBlockSize, NW, R, DUMP, pa::MmaMath>;
+        else
+            return pa::decode_kernel<D, G, kBlockSize, NW, R, DUMP, pa::SimtMath>;
+    }();
     static unsigned attr_done[kMaxDevices];
     if (!set_smem_once(kern, Cfg::kSmemBytes, attr_done)) return PA_ERR_CUDA;
     kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-template <bool DUMP>
-pa_status dispatch_decode(int D, int G, const pa::DecodeParams& p, int grid, cudaStream_t s) {
+template <MathKind MK, bool DUMP>
+pa_status dispatch_d_g(int D, int G, const pa::DecodeParams& p, int grid, cudaStream_t s) {
     if (D == 64) {
         switch (G) {
-            case 1: return launch_decode<64, 1, DUMP>(p, grid, s);
-            case 2: return launch_decode<64, 2, DUMP>(p, grid, s);
-            case 4: return launch_decode<64, 4, DUMP>(p, grid, s);
-            case 8: return launch_decode<64, 8, DUMP>(p, grid, s);
+            case 1: return launch_decode<MK, 64, 1, DUMP>(p, grid, s);
+            case 2: return launch_decode<MK, 64, 2, DUMP>(p, grid, s);
+            case 4: return launch_decode<MK, 64, 4, DUMP>(p, grid, s);
+            case 8: return launch_decode<MK, 64, 8, DUMP>(p, grid, s);
         }
     } else if (D == 128) {
         switch (G) {
-            case 1: return launch_decode<128, 1, DUMP>(p, grid, s);
-            case 2: return launch_decode<128, 2, DUMP>(p, grid, s);
-            case 4: return launch_decode<128, 4, DUMP>(p, grid, s);
+            case 1: return launch_decode<MK, 128, 1, DUMP>(p, grid, s);
+            case 2: return launch_decode<MK, 128, 2, DUMP>(p, grid, s);
+            case 4: return launch_decode<MK, 128, 4, DUMP>(p, grid, s);
+            case 8:
+                if constexpr (MK == MathKind::kMma) return launch_decode<MK, 128, 8, DUMP>(p, grid, s);
+                break;
         }
     }
     return PA_ERR_UNSUPPORTED;
+}
+
+template <bool DUMP>
+pa_status dispatch_decode(int D, int G, const pa::DecodeParams& p, int grid, cudaStream_t s) {
+    return math_kind() == MathKind::kMma ? dispatch_d_g<MathKind::kMma, DUMP>(D, G, p, grid, s)
+                                         : dispatch_d_g<MathKind::kSimt, DUMP>(D, G, p, grid, s);
 }
 
 // Shared validation of pa_decode and pa_decode_partials; fills p.
@@ -131,7 +215,7 @@ pa_status prepare_decode(const void* q, const void* k_cache, const void* v_cache
     if (!dims_ok(dims)) return PA_ERR_SHAPE;
     const pa_dims& d = *dims;
     const int G = d.num_q_heads / d.num_kv_heads;
-    if (d.block_size != kBlockSize || !supported(d.head_dim, G)) return PA_ERR_UNSUPPORTED;
+    if (d.block_size != kBlockSize || !supported(d.head_dim, G, math_kind())) return PA_ERR_UNSUPPORTED;
     if (d.num_seqs == 0) return PA_OK;
     // at least one block, so that a bad block id can be redirected to block 0
     if (d.num_blocks == 0) return PA_ERR_SHAPE;
@@ -144,9 +228,12 @@ pa_status prepare_decode(const void* q, const void* k_cache, const void* v_cache
     if (workspace_bytes < w.total) return PA_ERR_WORKSPACE;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     p = pa::DecodeParams{};
+    const int64_t rows = int64_t(d.num_blocks) * d.num_kv_heads * d.block_size;
+    if (rows >= (int64_t(1) << 31)) return PA_ERR_SHAPE;  // TMA row coordinates are int32
+    if (!make_cache_map(&p.tmap_k, k_cache, rows, d.head_dim, d.block_size) ||
+        !make_cache_map(&p.tmap_v, v_cache, rows, d.head_dim, d.block_size))
+        return PA_ERR_CUDA;
     p.q = static_cast<const uint8_t*>(q);
-    p.k_cache = static_cast<const uint8_t*>(k_cache);
-    p.v_cache = static_cast<const uint8_t*>(v_cache);
     p.block_tables = block_tables;
     p.context_lens = context_lens;
     p.out = static_cast<__nv_bfloat16*>(out);

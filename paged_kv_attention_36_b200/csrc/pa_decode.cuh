@@ -11,36 +11,52 @@
 // merges the pieces by log-sum-exp (flash-decoding), so long or skewed
 // contexts are split exactly where the balance needs it and nowhere else.
 //
-// Inside a CTA.  Warp W (the producer) walks the CTA's share, reads block
+// Inside a CTA.  Warp NW (the producer) walks the CTA's share, reads block
 // ids from the block table and streams each (block, kv head) K tile and V
-// tile (bs*D*2 contiguous bytes each, see the cache layout in pa.h) into a
-// ring of R shared-memory stages with 1-D bulk async copies (the TMA
-// engine), completing on a per-stage mbarrier.  Per segment it also copies
-// the G query rows of kv head g (contiguous in q) into a small descriptor
-// ring.  Warps 0..W-1 (consumers) take stage i when i % W equals their
-// index, so each page is read by exactly one warp and no CTA-wide barrier
-// is needed per page.  Each consumer warp keeps its own online-softmax
-// state (running max m, running sum l, fp32 accumulator) for all G query
-// heads; at a segment end the warps combine their states through shared
-// memory.  Every wait on an mbarrier is bounded in time.
+// tile into a ring of R shared-memory stages with tiled TMA copies
+// (128-byte swizzle), completing on a per-stage mbarrier.  Per segment it
+// also copies the G query rows of kv head g (contiguous in q) into a small
+// descriptor ring.  Warps 0..NW-1 (consumers) take stage i when i % NW
+// equals their index, so each page is read by exactly one warp and no
+// CTA-wide barrier is needed per page.  Each consumer warp keeps its own
+// online-softmax state (running max m, running sum l, fp32 accumulator) for
+// all G query heads; at a segment end the warps combine their states
+// through shared memory.  Every wait on an mbarrier is bounded in time.
 //
-// Per-page math (SIMT, fp32).  Lane = 8 * tg + c: the 8 lanes of token
-// group tg share one K row; lane c owns 16-byte chunks c, c+8, ... of the
-// row, so one 128-bit shared load per lane reads 4 whole rows per warp
-// without bank conflicts.  q (pre-multiplied by scale*log2(e)) lives in
-// registers as fp32 pairs; products and sums use packed fp32 FMA
-// (__ffma2_rn); the dot product is finished with 3 xor-shuffles; the
-// softmax runs in base 2 with exp2f.
+// Staged tile layout.  A (block, kv head) tile is bs = 16 rows of D bf16.
+// TMA writes it as D/64 panels of 16 lines x 128 bytes (panel p holds
+// columns 64p .. 64p+63), with the 128-byte swizzle: the 16-byte chunk c of
+// line t sits at chunk position c ^ (t % 8).  Any 8 consecutive rows read
+// at one logical chunk therefore hit 8 different bank groups, which makes
+// both the SIMT row reads and the tensor-core ldmatrix reads conflict-free.
+//
+// Per-page math, two policies:
+//   SimtMath: lane = 8*tg + c; the 8 lanes of token group tg share one K
+//     row, lane c owning chunks c, c+8; packed fp32 FMA (__ffma2_rn) on
+//     q pre-scaled by scale*log2(e); 3 xor-shuffles finish a dot product.
+//   MmaMath: the GQA group makes each page a small dense contraction, done
+//     on the tensor cores with mma.sync m16n8k16 (bf16 in, fp32 accumulate):
+//     S^T[16 tokens x 8 heads] = K_page * Q^T, then O^T[D x 8] += V^T * P^T.
+//     Heads beyond G are zero padding.  P (in [0, 1]) is split into a bf16
+//     high part and a bf16 remainder, both multiplied, so P.V keeps ~16
+//     mantissa bits; the softmax bookkeeping stays in fp32 registers.
 #pragma once
 
 #include "pa_device.cuh"
 
+#ifndef PA_EVICT_FIRST
+#define PA_EVICT_FIRST 1  // K/V pages are read once: first candidates for L2 eviction
+#endif
+#ifndef PA_L2_PREFETCH
+#define PA_L2_PREFETCH 0  // L2-prefetch a page before waiting for its stage
+#endif
+
 namespace pa {
 
 struct DecodeParams {
+    CUtensorMap tmap_k;           // K cache as [rows = NB*Hkv*bs][D/64 panels][64] bf16
+    CUtensorMap tmap_v;           // V cache, same
     const uint8_t* q;             // [B][Hq][D] bf16
-    const uint8_t* k_cache;       // [NB][Hkv][bs][D] bf16
-    const uint8_t* v_cache;
     const int32_t* block_tables;  // [B][M]
     const int32_t* context_lens;  // [B]
     __nv_bfloat16* out;           // [B][Hq][D]
@@ -82,28 +98,10 @@ struct Split {
     }
 };
 
-template <int D, int G, int BS, int W, int R>
-struct DecodeCfg {
-    static constexpr int kRow = D * 2;              // bytes of one K or V row
-    static constexpr int kTile = BS * kRow;         // one (block, kv head) tile
-    static constexpr int kStage = 2 * kTile;        // K tile then V tile
-    static constexpr int kSegSlots = 4;
-    static constexpr int kQBytes = G * kRow;
-    static constexpr int kCombFloats = G * D + ((2 * G + 3) / 4) * 4;  // one warp's state, 16-byte padded
-    static constexpr int kThreads = (W + 1) * 32;
-
-    static constexpr int kRingOff = 0;
-    static constexpr int kQOff = kRingOff + R * kStage;
-    static constexpr int kDescOff = kQOff + kSegSlots * kQBytes;
-    static constexpr int kCombOff = kDescOff + kSegSlots * int(sizeof(SegDesc));
-    static constexpr int kBarOff = kCombOff + 2 * W * kCombFloats * 4;
-    static constexpr int kNumBars = 2 * R + 2 * kSegSlots + 1;
-    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-    static constexpr int kMiscBytes = 256;
-    static constexpr int kSmemBytes = kMiscOff + kMiscBytes;
-    static_assert(kQBytes % 16 == 0 && kTile % 16 == 0, "bulk copies need 16-byte sizes");
-    static_assert(kBarOff % 8 == 0, "mbarrier alignment");
-};
+// Byte offset of 16-byte chunk `ch` (0 .. D/8-1) of row t in a staged tile.
+__device__ __forceinline__ int tile_off(int t, int ch) {
+    return ((ch >> 3) << 11) + (t << 7) + (((ch & 7) ^ (t & 7)) << 4);
+}
 
 // Shared scalars.
 struct Misc {
@@ -118,13 +116,13 @@ struct Misc {
 };
 static_assert(sizeof(Misc) <= 256, "misc area");
 
-// ---------------------------------------------------------------------------
-// Per-page fp32 math of one consumer warp.
+// ===========================================================================
+// SIMT math policy.
 template <int D, int G, int BS>
-struct SimtState {
+struct SimtMath {
     static constexpr int NCH = D / 64;  // 16-byte chunks per lane per row
     static constexpr int ROUNDS = BS / 4;
-    static constexpr int kRow = D * 2;
+    static constexpr bool kZeroMaskedV = false;  // masked rows are skipped
     static_assert(D % 64 == 0 && BS % 4 == 0, "layout");
 
     float2 q2[G][NCH][4];
@@ -132,12 +130,13 @@ struct SimtState {
     float m[G];
     float l[G];
 
-    __device__ __forceinline__ void load_q(const uint8_t* qs, int c, float qscale) {
+    __device__ __forceinline__ void load_q(const uint8_t* qs, int lane, float qscale) {
+        const int c = lane & 7;
 #pragma unroll
         for (int h = 0; h < G; ++h)
 #pragma unroll
             for (int i = 0; i < NCH; ++i) {
-                const uint4 v = lds128(qs + h * kRow + (c + 8 * i) * 16);
+                const uint4 v = lds128(qs + h * D * 2 + (c + 8 * i) * 16);
                 const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -159,18 +158,18 @@ struct SimtState {
         }
     }
 
-    // One page: K tile kt, V tile vt (shared memory), rows >= nvalid masked.
-    __device__ __forceinline__ void page(const uint8_t* kt, const uint8_t* vt, int nvalid, int tg, int c) {
+    __device__ __forceinline__ void page(const uint8_t* kt, const uint8_t* vt, int nvalid, int lane) {
+        const int tg = lane >> 3, c = lane & 7;
         float s[ROUNDS][G];
 #pragma unroll
         for (int r = 0; r < ROUNDS; ++r) {
-            const uint8_t* row = kt + (r * 4 + tg) * kRow + c * 16;
+            const int t = r * 4 + tg;
             float2 part[G];
 #pragma unroll
             for (int h = 0; h < G; ++h) part[h] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int i = 0; i < NCH; ++i) {
-                const uint4 v = lds128(row + i * 128);
+                const uint4 v = lds128(kt + tile_off(t, c + 8 * i));
                 const float2 k0 = bf16x2_to_float2(v.x), k1 = bf16x2_to_float2(v.y);
                 const float2 k2 = bf16x2_to_float2(v.z), k3 = bf16x2_to_float2(v.w);
 #pragma unroll
@@ -184,21 +183,18 @@ struct SimtState {
 #pragma unroll
             for (int h = 0; h < G; ++h) s[r][h] = part[h].x + part[h].y;
         }
-        // finish each dot product across the 8 lanes of its token group
 #pragma unroll
         for (int off = 1; off < 8; off <<= 1)
 #pragma unroll
             for (int r = 0; r < ROUNDS; ++r)
 #pragma unroll
                 for (int h = 0; h < G; ++h) s[r][h] += __shfl_xor_sync(0xffffffffu, s[r][h], off);
-        // rows past the context contribute nothing (their bytes may be anything)
 #pragma unroll
         for (int r = 0; r < ROUNDS; ++r) {
             const bool valid = (r * 4 + tg) < nvalid;
 #pragma unroll
             for (int h = 0; h < G; ++h) s[r][h] = valid ? s[r][h] : -INFINITY;
         }
-        // online softmax: page max, rescale when the running max grows
 #pragma unroll
         for (int h = 0; h < G; ++h) {
             float pm = s[0][h];
@@ -225,14 +221,13 @@ struct SimtState {
                 pr[r][h] = exp2f(s[r][h] - m[h]);
                 l[h] += pr[r][h];
             }
-        // P.V over the valid rows
 #pragma unroll
         for (int r = 0; r < ROUNDS; ++r) {
-            if ((r * 4 + tg) < nvalid) {
-                const uint8_t* row = vt + (r * 4 + tg) * kRow + c * 16;
+            const int t = r * 4 + tg;
+            if (t < nvalid) {
 #pragma unroll
                 for (int i = 0; i < NCH; ++i) {
-                    const uint4 v = lds128(row + i * 128);
+                    const uint4 v = lds128(vt + tile_off(t, c + 8 * i));
                     const float2 v0 = bf16x2_to_float2(v.x), v1 = bf16x2_to_float2(v.y);
                     const float2 v2 = bf16x2_to_float2(v.z), v3 = bf16x2_to_float2(v.w);
 #pragma unroll
@@ -249,7 +244,7 @@ struct SimtState {
     }
 
     // Sum l and acc over the 4 token groups of the warp.
-    __device__ __forceinline__ void reduce_groups() {
+    __device__ __forceinline__ void finish() {
 #pragma unroll
         for (int off = 8; off < 32; off <<= 1) {
 #pragma unroll
@@ -266,7 +261,7 @@ struct SimtState {
         }
     }
 
-    // Warp state -> comb[G*D + 2G]: acc[h][d], then m[h], then l[h].
+    // Warp state -> comb: acc[h][d] (G*D floats), then m[h], then l[h].
     __device__ __forceinline__ void deposit(float* comb, int lane) const {
         const int tg = lane >> 3, c = lane & 7;
         if (tg == 0) {
@@ -289,7 +284,173 @@ struct SimtState {
     }
 };
 
-// ---------------------------------------------------------------------------
+// ===========================================================================
+// Tensor-core math policy (mma.sync m16n8k16, bf16 x bf16 -> fp32).
+// Lane roles in the 16x8 accumulator tiles: row = lane/4 (+8), column pair
+// 2*(lane%4) + {0, 1}.  In S^T the rows are tokens and the columns heads;
+// in O^T the rows are head-dim indices and the columns heads, so a lane
+// always owns heads h0 = 2*(lane%4) and h0 + 1.
+template <int D, int G, int BS>
+struct MmaMath {
+    static_assert(BS == 16, "one m16 tile of tokens per page");
+    static_assert(G <= 8, "heads of a group fill at most the n8 tile");
+    static constexpr int KS = D / 16;  // k-steps of Q.K = m-tiles of O^T
+    static constexpr bool kZeroMaskedV = true;  // 0 * NaN would poison the mma
+
+    uint32_t qb[KS][2];  // Q^T as B fragments (bf16 pairs)
+    float acc[KS][4];    // O^T accumulator tiles
+    float m[2], l[2];    // heads h0, h0 + 1 of this lane (l: this lane's rows only)
+    float qscale;
+
+    __device__ __forceinline__ void load_q(const uint8_t* qs, int lane, float qs_scale) {
+        qscale = qs_scale;
+        const int h = lane >> 2, kk = (lane & 3) * 2;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            if (h < G) {
+                const uint8_t* row = qs + h * D * 2;
+                qb[ks][0] = *reinterpret_cast<const uint32_t*>(row + (16 * ks + kk) * 2);
+                qb[ks][1] = *reinterpret_cast<const uint32_t*>(row + (16 * ks + kk + 8) * 2);
+            } else {
+                qb[ks][0] = qb[ks][1] = 0u;
+            }
+        }
+    }
+
+    __device__ __forceinline__ void reset() {
+        m[0] = m[1] = -INFINITY;
+        l[0] = l[1] = 0.f;
+#pragma unroll
+        for (int i = 0; i < KS; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    }
+
+    __device__ __forceinline__ void page(const uint8_t* kt, const uint8_t* vt, int nvalid, int lane) {
+        const int mi = lane >> 3, r8 = lane & 7;
+        // ---- S^T = K . Q^T ----
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+            const int t = r8 + ((mi & 1) << 3);
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                uint32_t a[4];
+                ldmatrix_x4(a, kt + tile_off(t, 2 * ks + (mi >> 1)));
+                mma_bf16_16816(s, a, qb[ks][0], qb[ks][1]);
+            }
+        }
+        const int t0 = lane >> 2;
+        const bool v0 = t0 < nvalid, v1 = (t0 + 8) < nvalid;
+        s[0] = v0 ? s[0] * qscale : -INFINITY;
+        s[1] = v0 ? s[1] * qscale : -INFINITY;
+        s[2] = v1 ? s[2] * qscale : -INFINITY;
+        s[3] = v1 ? s[3] * qscale : -INFINITY;
+        // ---- online softmax over the 16 tokens of each head column ----
+        float mx0 = fmaxf(s[0], s[2]), mx1 = fmaxf(s[1], s[3]);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+        }
+        const bool grow0 = mx0 > m[0], grow1 = mx1 > m[1];
+        if (__any_sync(0xffffffffu, grow0 || grow1)) {
+            const float n0 = fmaxf(m[0], mx0), n1 = fmaxf(m[1], mx1);
+            const float a0 = exp2f(m[0] - n0), a1 = exp2f(m[1] - n1);
+            m[0] = n0;
+            m[1] = n1;
+            l[0] *= a0;
+            l[1] *= a1;
+#pragma unroll
+            for (int i = 0; i < KS; ++i) {
+                acc[i][0] *= a0;
+                acc[i][1] *= a1;
+                acc[i][2] *= a0;
+                acc[i][3] *= a1;
+            }
+        }
+        const float p0 = exp2f(s[0] - m[0]), p1 = exp2f(s[1] - m[1]);
+        const float p2 = exp2f(s[2] - m[0]), p3 = exp2f(s[3] - m[1]);
+        l[0] += p0 + p2;
+        l[1] += p1 + p3;
+        // ---- P^T as B fragments: bf16 high part and remainder ----
+        const uint32_t h01 = float2_to_bf16x2(p0, p1), h23 = float2_to_bf16x2(p2, p3);
+        const float2 f01 = bf16x2_to_float2(h01), f23 = bf16x2_to_float2(h23);
+        const uint32_t r01 = float2_to_bf16x2(p0 - f01.x, p1 - f01.y);
+        const uint32_t r23 = float2_to_bf16x2(p2 - f23.x, p3 - f23.y);
+        const uint32_t bh0 = movmatrix_trans(h01), bh1 = movmatrix_trans(h23);
+        const uint32_t bl0 = movmatrix_trans(r01), bl1 = movmatrix_trans(r23);
+        // ---- O^T += V^T . P^T ----
+        const int tv = r8 + ((mi >> 1) << 3);
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+            uint32_t a[4];
+            ldmatrix_x4_trans(a, vt + tile_off(tv, 2 * mt + (mi & 1)));
+            mma_bf16_16816(acc[mt], a, bh0, bh1);
+            mma_bf16_16816(acc[mt], a, bl0, bl1);
+        }
+    }
+
+    // Sum l over the 8 row groups (lanes with equal lane % 4).
+    __device__ __forceinline__ void finish() {
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            l[0] += __shfl_xor_sync(0xffffffffu, l[0], off);
+            l[1] += __shfl_xor_sync(0xffffffffu, l[1], off);
+        }
+    }
+
+    __device__ __forceinline__ void deposit(float* comb, int lane) const {
+        const int h0 = (lane & 3) * 2, d0 = lane >> 2;
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+            const int d = 16 * mt + d0;
+            if (h0 < G) {
+                comb[h0 * D + d] = acc[mt][0];
+                comb[h0 * D + d + 8] = acc[mt][2];
+            }
+            if (h0 + 1 < G) {
+                comb[(h0 + 1) * D + d] = acc[mt][1];
+                comb[(h0 + 1) * D + d + 8] = acc[mt][3];
+            }
+        }
+        if (d0 == 0) {
+            if (h0 < G) {
+                comb[G * D + h0] = m[0];
+                comb[G * D + G + h0] = l[0];
+            }
+            if (h0 + 1 < G) {
+                comb[G * D + h0 + 1] = m[1];
+                comb[G * D + G + h0 + 1] = l[1];
+            }
+        }
+    }
+};
+
+// ===========================================================================
+template <int D, int G, int BS, int NW, int R>
+struct DecodeCfg {
+    static constexpr int kRow = D * 2;              // bytes of one K or V row
+    static constexpr int kTile = BS * kRow;         // one (block, kv head) tile
+    static constexpr int kPanel = BS * 128;         // one 64-column panel of a tile
+    static constexpr int kStage = 2 * kTile;        // K tile then V tile
+    static constexpr int kSegSlots = 4;
+    static constexpr int kQBytes = G * kRow;
+    static constexpr int kCombFloats = G * D + ((2 * G + 3) / 4) * 4;  // one warp's state, 16-byte padded
+    static constexpr int kThreads = (NW + 1) * 32;
+
+    // offsets from the 1024-byte aligned base
+    static constexpr int kRingOff = 0;
+    static constexpr int kQOff = kRingOff + R * kStage;
+    static constexpr int kDescOff = kQOff + kSegSlots * kQBytes;
+    static constexpr int kCombOff = kDescOff + kSegSlots * int(sizeof(SegDesc));
+    static constexpr int kBarOff = kCombOff + NW * kCombFloats * 4;
+    static constexpr int kNumBars = 2 * R + 2 * kSegSlots + 1;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    static constexpr int kMiscBytes = 256;
+    static constexpr int kSmemBytes = kMiscOff + kMiscBytes + 1024;  // + alignment slack
+    static_assert(kQBytes % 16 == 0 && kTile % 1024 == 0, "TMA tile alignment");
+    static_assert(kBarOff % 8 == 0, "mbarrier alignment");
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+};
+
 template <int BS>
 __device__ __forceinline__ int32_t clamp_len(const DecodeParams& p, int b, bool report) {
     int32_t L = __ldg(p.context_lens + b);
@@ -301,16 +462,18 @@ __device__ __forceinline__ int32_t clamp_len(const DecodeParams& p, int b, bool 
     return L;
 }
 
-template <int D, int G, int BS, int W, int R, bool DUMP>
-__global__ void __launch_bounds__((W + 1) * 32, 1) decode_kernel(const DecodeParams p) {
-    // Stage i % R always feeds warp i % W, so a warp waiting on a stage is at
+template <int D, int G, int BS, int NW, int R, bool DUMP, template <int, int, int> class Math>
+__global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
+    // Stage i % R always feeds warp i % NW, so a warp waiting on a stage is at
     // most one phase away from it and the parity waits are exact.
-    static_assert(R % W == 0, "ring depth must be a multiple of the consumer warps");
-    static_assert(W + 1 <= 16, "block reductions hold 16 warps");
-    using Cfg = DecodeCfg<D, G, BS, W, R>;
+    static_assert(R % NW == 0, "ring depth must be a multiple of the consumer warps");
+    static_assert(NW + 1 <= 16, "block reductions hold 16 warps");
+    using Cfg = DecodeCfg<D, G, BS, NW, R>;
     constexpr int S = Cfg::kSegSlots;
     constexpr int NT = Cfg::kThreads;
-    extern __shared__ __align__(128) uint8_t smem[];
+    constexpr int NPANEL = D / 64;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* ring = smem + Cfg::kRingOff;
     uint8_t* qring = smem + Cfg::kQOff;
     SegDesc* descs = reinterpret_cast<SegDesc*>(smem + Cfg::kDescOff);
@@ -332,9 +495,9 @@ __global__ void __launch_bounds__((W + 1) * 32, 1) decode_kernel(const DecodePar
         }
         for (int s = 0; s < S; ++s) {
             mbar_init(&segfull[s], 1);
-            mbar_init(&segempty[s], W);
+            mbar_init(&segempty[s], NW);
         }
-        mbar_init(consbar, W);
+        mbar_init(consbar, NW);
         misc->abort = 0;
         misc->found = 0;
         fence_mbar_init();
@@ -357,7 +520,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1) decode_kernel(const DecodePar
     __syncthreads();
     long long total = 0;
 #pragma unroll
-    for (int w = 0; w < W + 1; ++w) total += misc->red[w];
+    for (int w = 0; w < NW + 1; ++w) total += misc->red[w];
     const int64_t Wt = total * p.Hkv;  // all (b, g, page) work
     if (Wt == 0) return;
     const int64_t want = (Wt + p.min_pages - 1) / p.min_pages;
@@ -385,7 +548,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1) decode_kernel(const DecodePar
         long long before = carry;
         for (int w = 0; w < warp; ++w) before += misc->red[w];
         long long chunk_total = 0;
-        for (int w = 0; w < W + 1; ++w) chunk_total += misc->red[w];
+        for (int w = 0; w < NW + 1; ++w) chunk_total += misc->red[w];
         const long long lo = before + incl - v;
         if (v > 0 && lo <= p_start && p_start < lo + v) {
             misc->b0 = b;
@@ -397,7 +560,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1) decode_kernel(const DecodePar
         if (misc->found) break;
     }
 
-    if (warp == W) {
+    if (warp == NW) {
         // ======================= producer warp =======================
         int b = misc->b0;
         int64_t pre = misc->pre0;
@@ -410,7 +573,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1) decode_kernel(const DecodePar
         uint32_t page_i = 0, seg_i = 0;
         constexpr int C = R < 32 ? R : 32;
         bool ok = true;
-        const uint64_t pol = policy_evict_first();
+        const uint64_t pol = PA_EVICT_FIRST ? policy_evict_first() : policy_evict_normal();
         while (ok && pos < p_end) {
             const int npg = int((int64_t(np - j) < p_end - pos) ? int64_t(np - j) : p_end - pos);
             if (lane == 0) {
@@ -447,13 +610,25 @@ __global__ void __launch_bounds__((W + 1) * 32, 1) decode_kernel(const DecodePar
                     const uint32_t i = page_i + c0 + lane;
                     const int slot = int(i % R);
                     const uint32_t use = i / R;
+                    if (PA_L2_PREFETCH && use > 0) {
+                        // start the DRAM read now; the load below waits for a free stage
+#pragma unroll
+                        for (int pn = 0; pn < NPANEL; ++pn) {
+                            tma_prefetch_3d(&p.tmap_k, 0, pn, (blk * p.Hkv + g) * BS, pol);
+                            tma_prefetch_3d(&p.tmap_v, 0, pn, (blk * p.Hkv + g) * BS, pol);
+                        }
+                    }
                     if (use > 0) lane_ok = mbar_wait(&empty[slot], (use - 1) & 1, abort);
                     if (lane_ok) {
                         uint8_t* st = ring + slot * Cfg::kStage;
-                        const int64_t src = (int64_t(blk) * p.Hkv + g) * Cfg::kTile;
+                        const int row = (blk * p.Hkv + g) * BS;
                         mbar_arrive_expect_tx(&full[slot], 2 * Cfg::kTile);
-                        bulk_g2s_hint(st, p.k_cache + src, Cfg::kTile, &full[slot], pol);
-                        bulk_g2s_hint(st + Cfg::kTile, p.v_cache + src, Cfg::kTile, &full[slot], pol);
+#pragma unroll
+                        for (int pn = 0; pn < NPANEL; ++pn) {
+                            tma_load_3d(st + pn * Cfg::kPanel, &p.tmap_k, 0, pn, row, &full[slot], pol);
+                            tma_load_3d(st + Cfg::kTile + pn * Cfg::kPanel, &p.tmap_v, 0, pn, row, &full[slot],
+                                        pol);
+                        }
                     }
                 }
                 ok = __all_sync(0xffffffffu, lane_ok);
@@ -494,9 +669,8 @@ __global__ void __launch_bounds__((W + 1) * 32, 1) decode_kernel(const DecodePar
     }
 
     // ========================= consumer warps =========================
-    SimtState<D, G, BS> st;
-    const int tg = lane >> 3, c = lane & 7;
-    const int ct = threadIdx.x;  // 0 .. W*32-1
+    Math<D, G, BS> st;
+    const int ct = threadIdx.x;  // 0 .. NW*32-1
     uint32_t page_base = 0, seg_i = 0, cons_phase = 0;
 
     auto rendezvous = [&]() -> bool {
@@ -512,26 +686,40 @@ __global__ void __launch_bounds__((W + 1) * 32, 1) decode_kernel(const DecodePar
         if (!mbar_wait(&segfull[s], (seg_i / S) & 1, abort)) return;
         const SegDesc d = descs[s];
         if (d.npg == 0) break;
-        st.load_q(qring + s * Cfg::kQBytes, c, p.qscale);
+        st.load_q(qring + s * Cfg::kQBytes, lane, p.qscale);
         __syncwarp();
         if (lane == 0) mbar_arrive(&segempty[s]);
         st.reset();
 
-        for (int k = int((uint32_t(warp) + W - page_base % W) % W); k < d.npg; k += W) {
+        for (int k = int((uint32_t(warp) + NW - page_base % NW) % NW); k < d.npg; k += NW) {
             const uint32_t i = page_base + k;
             const int slot = int(i % R);
             if (!mbar_wait(&full[slot], (i / R) & 1, abort)) return;
-            const uint8_t* stg = ring + slot * Cfg::kStage;
-            const int nv = d.L - (d.j0 + k) * BS;
-            st.page(stg, stg + Cfg::kTile, nv < BS ? nv : BS, tg, c);
+            uint8_t* stg = ring + slot * Cfg::kStage;
+            const int nv_raw = d.L - (d.j0 + k) * BS;
+            const int nv = nv_raw < BS ? nv_raw : BS;
+            if (Math<D, G, BS>::kZeroMaskedV && nv < BS) {
+                // rows past the context may hold anything (NaN included): clear
+                // them in the V tile so that 0 * row stays 0 in the tensor core
+                const int per_panel = (BS - nv) * 8;  // 16-byte chunks
+                for (int x = lane; x < NPANEL * per_panel; x += 32) {
+                    const int pn = x / per_panel, rem = x - pn * per_panel;
+                    const int t = nv + (rem >> 3), cch = rem & 7;
+                    *reinterpret_cast<uint4*>(stg + Cfg::kTile + pn * Cfg::kPanel + t * 128 + cch * 16) =
+                        make_uint4(0, 0, 0, 0);
+                }
+                __syncwarp();
+                fence_proxy_async_smem();
+            }
+            st.page(stg, stg + Cfg::kTile, nv, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[slot]);
         }
         page_base += d.npg;
 
-        // ---- segment end: combine the W warp states ----
-        st.reduce_groups();
-        float* comb = combbuf + (seg_i & 1) * W * Cfg::kCombFloats;
+        // ---- segment end: combine the NW warp states ----
+        st.finish();
+        float* comb = combbuf;
         st.deposit(comb + warp * Cfg::kCombFloats, lane);
         if (!rendezvous()) return;
 
@@ -542,14 +730,14 @@ __global__ void __launch_bounds__((W + 1) * 32, 1) decode_kernel(const DecodePar
             if (!rendezvous()) return;
         }
         const int dump_idx = DUMP ? misc->dump_idx : 0;
-        for (int o = ct; o < G * D; o += W * 32) {
+        for (int o = ct; o < G * D; o += NW * 32) {
             const int h = o / D, dd = o - h * D;
             float M = -INFINITY;
 #pragma unroll
-            for (int w = 0; w < W; ++w) M = fmaxf(M, comb[w * Cfg::kCombFloats + G * D + h]);
+            for (int w = 0; w < NW; ++w) M = fmaxf(M, comb[w * Cfg::kCombFloats + G * D + h]);
             float lsum = 0.f, a = 0.f;
 #pragma unroll
-            for (int w = 0; w < W; ++w) {
+            for (int w = 0; w < NW; ++w) {
                 const float* cw = comb + w * Cfg::kCombFloats;
                 const float sc = exp2f(cw[G * D + h] - M);
                 lsum += cw[G * D + G + h] * sc;
@@ -580,7 +768,10 @@ __global__ void __launch_bounds__((W + 1) * 32, 1) decode_kernel(const DecodePar
             }
         }
 
-        if (!whole) {
+        if (whole) {
+            // every warp has read comb before any warp deposits the next segment
+            if (!rendezvous()) return;
+        } else {
             // ---- split-KV: the last CTA to finish a piece of (b, g) merges ----
             __threadfence();
             if (!rendezvous()) return;
@@ -591,7 +782,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1) decode_kernel(const DecodePar
             if (!rendezvous()) return;
             if (misc->is_last) {
                 __threadfence();
-                for (int o = ct; o < G * D; o += W * 32) {
+                for (int o = ct; o < G * D; o += NW * 32) {
                     const int h = o / D, dd = o - h * D;
                     float M = -INFINITY;
                     for (int k = d.k0; k <= d.k1; ++k) {
