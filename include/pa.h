@@ -65,7 +65,9 @@ typedef enum pa_status {
     PA_ERR_UNSUPPORTED = -3,  /* head_dim / block_size / GQA group not built into this library */
     PA_ERR_ALIGN = -4,        /* a tensor pointer is not 16-byte aligned */
     PA_ERR_WORKSPACE = -5,    /* workspace NULL or smaller than pa_decode_workspace_bytes() */
-    PA_ERR_CUDA = -6          /* a CUDA runtime call failed (launch, attribute, device query) */
+    PA_ERR_CUDA = -6,         /* a CUDA runtime call failed (launch, attribute, device query) */
+    PA_ERR_SCRATCH_LIMIT = -7 /* pa_decode_static_ws: the problem needs more scratch than
+                                 PA_STATIC_SCRATCH_BYTES */
 } pa_status;
 
 /* Bits of the device error word. */
@@ -150,6 +152,35 @@ PA_API pa_status pa_decode_partials(const void* q, const void* k_cache, const vo
                              void* workspace, size_t workspace_bytes, int32_t capacity,
                              int32_t* seg_meta, float* seg_o, float* seg_m, float* seg_l,
                              int32_t* seg_count, void* stream);
+
+/*
+ * Allocation-free decode.  No counterpart in the pages: this entry point
+ * exists for callers that cannot allocate device memory at the point where
+ * they decode -- for example code running inside a host runtime or plugin
+ * that owns every device allocation and offers no allocator, or a latency-
+ * critical loop where cudaMalloc (which may block and synchronise the
+ * device) is not acceptable.  It computes exactly what pa_decode computes,
+ * with the same arguments minus the workspace: its scratch (merge counters
+ * and split-KV partials) lives in a fixed array of PA_STATIC_SCRATCH_BYTES
+ * bytes inside the library, which every GPU that loads the library holds
+ * until the process exits.
+ *   - Nothing is allocated: no cudaMalloc/cudaFree, no allocating library call.
+ *   - A problem whose scratch (pa_decode_workspace_bytes(dims, 0)) exceeds
+ *     PA_STATIC_SCRATCH_BYTES is rejected with PA_ERR_SCRATCH_LIMIT before
+ *     anything is launched.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array and it keeps the previous
+ *     call's contents; each call clears the merge counters it needs (an
+ *     asynchronous memset on `stream`) before its kernel.  Calls that can
+ *     overlap on the GPU (different streams without ordering) race on the
+ *     array and give undefined results: order them.
+ */
+#define PA_STATIC_SCRATCH_BYTES (4u << 20)
+PA_API pa_status pa_decode_static_ws(const void* q, const void* k_cache, const void* v_cache,
+                                     const int32_t* block_tables, const int32_t* context_lens,
+                                     float scale, void* out, const pa_dims* dims, void* stream);
 
 /*
  * Reads (and, if `clear` != 0, resets) the device error word of the

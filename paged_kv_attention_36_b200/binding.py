@@ -57,6 +57,8 @@ def _load(path: str = LIB_PATH):
     lib.pa_decode_partials.argtypes = [vp, vp, vp, vp, vp, f32, vp, dp, i32, vp, sz, i32,
                                        vp, vp, vp, vp, vp, vp]
     lib.pa_decode_partials.restype = i32
+    lib.pa_decode_static_ws.argtypes = [vp, vp, vp, vp, vp, f32, vp, dp, vp]
+    lib.pa_decode_static_ws.restype = i32
     lib.pa_device_errors.argtypes = [ctypes.POINTER(i32), i32]
     lib.pa_device_errors.restype = i32
     lib.pa_status_string.argtypes = [i32]
@@ -68,7 +70,10 @@ lib = _load()
 
 # Every symbol include/pa.h declares.
 EXPORTS = ("pa_cache_append", "pa_decode_workspace_bytes", "pa_decode_default_ctas", "pa_decode",
-           "pa_decode_partials", "pa_device_errors", "pa_status_string")
+           "pa_decode_partials", "pa_decode_static_ws", "pa_device_errors", "pa_status_string")
+
+PA_ERR_SCRATCH_LIMIT = -7
+PA_STATIC_SCRATCH_BYTES = 4 << 20  # include/pa.h
 
 
 def pa_status_string(code: int) -> str:
@@ -196,6 +201,17 @@ def pa_decode_partials(q, k_cache, v_cache, block_tables, context_lens, scale: f
                                   int(num_ctas), _ptr(workspace), workspace.numel(), int(capacity),
                                   _ptr(seg_meta), _ptr(seg_o), _ptr(seg_m), _ptr(seg_l),
                                   _ptr(seg_count), _stream(stream)), "pa_decode_partials")
+
+
+def pa_decode_static_ws(q, k_cache, v_cache, block_tables, context_lens, scale: float, out,
+                        stream=None) -> None:
+    """pa_decode without a caller workspace: the library's fixed scratch array
+    is used instead, so nothing is allocated (for callers that cannot
+    allocate device memory where they decode; see include/pa.h)."""
+    dims = _decode_args(q, k_cache, v_cache, block_tables, context_lens, out)
+    _check(lib.pa_decode_static_ws(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                                   _ptr(context_lens), float(scale), _ptr(out), ctypes.byref(dims),
+                                   _stream(stream)), "pa_decode_static_ws")
 
 
 def pa_device_errors(clear: bool = False) -> int:

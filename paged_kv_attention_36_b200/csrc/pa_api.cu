@@ -252,6 +252,30 @@ pa_status prepare_decode(const void* q, const void* k_cache, const void* v_cache
 
 }  // namespace
 
+// ---- scratch for the allocation-free decode (pa_decode_static_ws) ----------
+// A fixed device array, present on every GPU that loads the library.  Host
+// code may only use the name as a symbol handle: its device address comes
+// from cudaGetSymbolAddress, looked up once per device with that device
+// current (a kernel given the host-side name would read the wrong memory).
+static __device__ __align__(256) unsigned char g_pa_static_scratch[PA_STATIC_SCRATCH_BYTES];
+
+namespace {
+void* g_static_scratch_addr[kMaxDevices];  // per device, guarded by g_mu
+
+pa_status static_scratch_address(void** addr) {
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_static_scratch_addr[dev]) {
+        void* a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_pa_static_scratch) != cudaSuccess || !a) return PA_ERR_CUDA;
+        g_static_scratch_addr[dev] = a;
+    }
+    *addr = g_static_scratch_addr[dev];
+    return PA_OK;
+}
+}  // namespace
+
 extern "C" {
 
 const char* pa_status_string(int32_t status) {
@@ -263,6 +287,8 @@ const char* pa_status_string(int32_t status) {
         case PA_ERR_ALIGN: return "PA_ERR_ALIGN: tensor pointer not 16-byte aligned";
         case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE: workspace missing or too small";
         case PA_ERR_CUDA: return "PA_ERR_CUDA: CUDA runtime call failed";
+        case PA_ERR_SCRATCH_LIMIT:
+            return "PA_ERR_SCRATCH_LIMIT: problem needs more scratch than PA_STATIC_SCRATCH_BYTES";
         default: return "unknown pa_status";
     }
 }
@@ -337,6 +363,29 @@ pa_status pa_decode_partials(const void* q, const void* k_cache, const void* v_c
     p.seg_count = seg_count;
     return dispatch_decode<true>(dims->head_dim, dims->num_q_heads / dims->num_kv_heads, p, num_ctas,
                                  static_cast<cudaStream_t>(stream));
+}
+
+pa_status pa_decode_static_ws(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                              const int32_t* context_lens, float scale, void* out, const pa_dims* dims,
+                              void* stream) {
+    if (!dims) return PA_ERR_NULL;
+    if (!dims_ok(dims)) return PA_ERR_SHAPE;
+    const int grid = sm_count();
+    if (grid <= 0) return PA_ERR_CUDA;
+    if (ws_layout(*dims, grid).total > size_t(PA_STATIC_SCRATCH_BYTES)) return PA_ERR_SCRATCH_LIMIT;
+    void* scratch = nullptr;
+    pa_status st = static_scratch_address(&scratch);
+    if (st != PA_OK) return st;
+    pa::DecodeParams p;
+    st = prepare_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, dims, grid, scratch,
+                        PA_STATIC_SCRATCH_BYTES, p);
+    if (st != PA_OK || dims->num_seqs == 0) return st;
+    // the array keeps the last call's contents: the merge counters must start at zero
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(p.counters, 0, size_t(dims->num_seqs) * dims->num_kv_heads * sizeof(int32_t), s) !=
+        cudaSuccess)
+        return PA_ERR_CUDA;
+    return dispatch_decode<false>(dims->head_dim, dims->num_q_heads / dims->num_kv_heads, p, grid, s);
 }
 
 pa_status pa_device_errors(int32_t* errors_out, int32_t clear) {

@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol(binding):
 
 
 def test_status_strings(binding):
-    for code in range(0, -7, -1):
+    for code in range(0, -8, -1):
         s = binding.pa_status_string(code)
         assert s and "unknown" not in s
     assert "unknown" in binding.pa_status_string(-99)
