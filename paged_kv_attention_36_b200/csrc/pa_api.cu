@@ -36,30 +36,51 @@ enum class MathKind { kMma, kSimt };
 
 template <MathKind MK, int D, int G>
 struct Tune;
-template <int D, int G>
-struct Tune<MathKind::kSimt, D, G> {
-    static constexpr int NW = (G * D >= 512) ? 7 : 11;
-    static constexpr int R = D == 64 ? (NW == 11 ? 33 : 28) : (NW == 11 ? 22 : 21);
-};
+
 #ifndef PA_MMA_NW
 #define PA_MMA_NW 8
 #endif
 #ifndef PA_MAX_RING
 #define PA_MAX_RING 64
 #endif
+#ifndef PA_MMA_STAGE_BYTES
+#define PA_MMA_STAGE_BYTES 8192  // pages per ring stage = this / (K+V bytes of a page)
+#endif
 // Deepest ring (a multiple of NW, at most PA_MAX_RING) whose CTA fits in shared memory.
-template <int D, int G, int NW>
+template <int D, int G, int NW, int PPS>
 constexpr int ring_fit() {
     int r = (PA_MAX_RING / NW) * NW;
-    while (r > NW && pa::DecodeCfg<D, G, kBlockSize, NW, 1>::kSmemBytes + (r - 1) * (2 * 16 * D * 2 + 16) > 232448)
+    while (r > NW && pa::DecodeCfg<D, G, kBlockSize, NW, 1, PPS>::kSmemBytes +
+                             (r - 1) * (PPS * 2 * kBlockSize * D * 2 + 16) > 232448)
         r -= NW;
     return r;
 }
 template <int D, int G>
 struct Tune<MathKind::kMma, D, G> {
     static constexpr int NW = PA_MMA_NW;
-    static constexpr int R = ring_fit<D, G, NW>();
+    static constexpr int PPS = (PA_MMA_STAGE_BYTES / (2 * kBlockSize * D * 2)) > 0
+                                   ? PA_MMA_STAGE_BYTES / (2 * kBlockSize * D * 2) : 1;
+    static constexpr int R = ring_fit<D, G, NW, PPS>();
 };
+
+template <int D, int G>
+struct Tune<MathKind::kSimt, D, G> {
+    static constexpr int NW = (G * D >= 512) ? 7 : 11;  // 8 warps: 255 registers each; 12: 168
+    static constexpr int PPS = 1;
+    static constexpr int R = ring_fit<D, G, NW, PPS>();
+};
+
+// Fixed cost of finishing a segment, expressed as K+V bytes that could be
+// streamed meanwhile (measured: ~1.5 us of a CTA's time per segment end);
+// PA_SEG_WEIGHT_BYTES overrides it.
+int32_t seg_weight_pages(int head_dim) {
+    static const long long bytes = [] {
+        const char* e = std::getenv("PA_SEG_WEIGHT_BYTES");
+        return e ? std::atoll(e) : 65536LL;
+    }();
+    const long long page = 2LL * kBlockSize * head_dim * 2;
+    return int32_t(bytes / page);
+}
 
 MathKind math_kind() {
     static const MathKind k = [] {
@@ -165,13 +186,13 @@ bool make_cache_map(CUtensorMap* map, const void* base, int64_t rows, int D, int
 
 template <MathKind MK, int D, int G, bool DUMP>
 pa_status launch_decode(const pa::DecodeParams& p, int grid, cudaStream_t stream) {
-    constexpr int NW = Tune<MK, D, G>::NW, R = Tune<MK, D, G>::R;
-    using Cfg = pa::DecodeCfg<D, G, kBlockSize, NW, R>;
+    constexpr int NW = Tune<MK, D, G>::NW, R = Tune<MK, D, G>::R, PPS = Tune<MK, D, G>::PPS;
+    using Cfg = pa::DecodeCfg<D, G, kBlockSize, NW, R, PPS>;
     auto kern = [] {
         if constexpr (MK == MathKind::kMma)
-            return pa::decode_kernel<D, G, kBlockSize, NW, R, DUMP, pa::MmaMath>;
+            return pa::decode_kernel<D, G, kBlockSize, NW, R, PPS, DUMP, pa::MmaMath>;
         else
-            return pa::decode_kernel<D, G, kBlockSize, NW, R, DUMP, pa::SimtMath>;
+            return pa::decode_kernel<D, G, kBlockSize, NW, R, PPS, DUMP, pa::SimtMath>;
     }();
     static unsigned attr_done[kMaxDevices];
     if (!set_smem_once(kern, Cfg::kSmemBytes, attr_done)) return PA_ERR_CUDA;
@@ -244,6 +265,7 @@ pa_status prepare_decode(const void* q, const void* k_cache, const void* v_cache
     p.NB = d.num_blocks;
     p.M = d.max_blocks_per_seq;
     p.min_pages = kMinPagesPerCta;
+    p.seg_weight = seg_weight_pages(d.head_dim);
     p.counters = reinterpret_cast<int32_t*>(ws + w.counters);
     p.part_o = reinterpret_cast<float*>(ws + w.part_o);
     p.part_ml = reinterpret_cast<float2*>(ws + w.part_ml);

@@ -1,11 +1,14 @@
 // pa_decode.cuh -- paged decode attention for sm_100a.
 //
 // Work decomposition.  The decode reads, for every (sequence b, kv head g),
-// the np_b = ceil(L_b / bs) pages of that sequence.  Flatten all of them in
-// (b, g, page) order into one list of W pages and give each of the
-// persistent CTAs (one per SM) an equal contiguous share.  A CTA's share is
-// a run of "segments": whole (b, g) page lists, plus at most a partial one
-// at each end.  A whole segment is finished inside the CTA and writes bf16
+// the np_b = ceil(L_b / bs) pages of that sequence.  Lay all (b, g) out in
+// order on one line, each taking np_b + X units: its pages, then X units
+// that stand for the fixed cost of finishing a segment (combining the warp
+// states and writing the output; X = seg_weight, measured in pages).  Each
+// persistent CTA (one per SM) takes an equal contiguous share of the line,
+// so a share made of many short segments gets fewer pages.  A share is a
+// run of "segments": whole (b, g) page lists, plus at most a partial one at
+// each end.  A whole segment is finished inside the CTA and writes bf16
 // output; a partial one writes an fp32 split-KV partial (normalised output,
 // max logit, exp-sum) and the last CTA to finish a piece of that (b, g)
 // merges the pieces by log-sum-exp (flash-decoding), so long or skewed
@@ -63,6 +66,7 @@ struct DecodeParams {
     float qscale;                 // scale * log2(e): logits in base-2 units
     int32_t B, Hq, Hkv, NB, M;
     int32_t min_pages;            // fewest pages worth giving a CTA
+    int32_t seg_weight;           // cost of finishing a segment, in pages (weights the split)
     int32_t* counters;            // [B*Hkv] merge tickets, zero between calls
     float* part_o;                // [grid][2][G][D] split-KV partial outputs
     float2* part_ml;              // [grid][2][G] (max logit base 2, exp-sum)
@@ -77,14 +81,12 @@ struct DecodeParams {
 
 // One segment of a CTA's share, handed from the producer to the consumers.
 struct SegDesc {
-    int64_t bg_start;  // flattened index of page 0 of (b, g)
     int32_t b, g;
     int32_t j0;        // first page of the segment within sequence b
     int32_t npg;       // pages in the segment; 0 marks the end of the share
     int32_t L;         // context length of b
     int32_t k0, k1;    // CTAs holding pages of (b, g); whole iff k0 == k1
-    int32_t first;     // this is the CTA's first segment
-    int32_t pad[6];
+    int32_t pad[9];
 };
 static_assert(sizeof(SegDesc) == 64, "descriptor size");
 
@@ -109,12 +111,13 @@ struct Misc {
     int is_last;
     int dump_idx;
     int found;
-    int b0;
-    int pad0;
-    long long pre0;
+    int b0;              // sequence where the share starts
+    int pad1;
+    long long pre0;      // weighted position of b0's first unit
     long long red[16];  // block reductions, one slot per warp (<= 16 warps)
 };
 static_assert(sizeof(Misc) <= 256, "misc area");
+
 
 // ===========================================================================
 // SIMT math policy.
@@ -137,6 +140,23 @@ struct SimtMath {
 #pragma unroll
             for (int i = 0; i < NCH; ++i) {
                 const uint4 v = lds128(qs + h * D * 2 + (c + 8 * i) * 16);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 f = bf16x2_to_float2(w[j]);
+                    q2[h][i][j] = make_float2(f.x * qscale, f.y * qscale);
+                }
+            }
+    }
+
+    // Same, from global memory (the G rows of q of one kv head).
+    __device__ __forceinline__ void load_q_global(const uint8_t* gq, int lane, float qscale) {
+        const int c = lane & 7;
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+            for (int i = 0; i < NCH; ++i) {
+                const uint4 v = __ldg(reinterpret_cast<const uint4*>(gq + h * D * 2 + (c + 8 * i) * 16));
                 const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -261,15 +281,15 @@ struct SimtMath {
         }
     }
 
-    // Warp state -> comb: acc[h][d] (G*D floats), then m[h], then l[h].
-    __device__ __forceinline__ void deposit(float* comb, int lane) const {
+    // Warp state -> dep: acc[h][d] (G*D floats), then m[h], then l[h].
+    __device__ __forceinline__ void deposit(float* dep, int lane) const {
         const int tg = lane >> 3, c = lane & 7;
         if (tg == 0) {
 #pragma unroll
             for (int h = 0; h < G; ++h)
 #pragma unroll
                 for (int i = 0; i < NCH; ++i) {
-                    float4* dst = reinterpret_cast<float4*>(comb + h * D + (c + 8 * i) * 8);
+                    float4* dst = reinterpret_cast<float4*>(dep + h * D + (c + 8 * i) * 8);
                     dst[0] = make_float4(acc[h][i][0].x, acc[h][i][0].y, acc[h][i][1].x, acc[h][i][1].y);
                     dst[1] = make_float4(acc[h][i][2].x, acc[h][i][2].y, acc[h][i][3].x, acc[h][i][3].y);
                 }
@@ -277,8 +297,8 @@ struct SimtMath {
         if (lane == 0) {
 #pragma unroll
             for (int h = 0; h < G; ++h) {
-                comb[G * D + h] = m[h];
-                comb[G * D + G + h] = l[h];
+                dep[G * D + h] = m[h];
+                dep[G * D + G + h] = l[h];
             }
         }
     }
@@ -311,6 +331,22 @@ struct MmaMath {
                 const uint8_t* row = qs + h * D * 2;
                 qb[ks][0] = *reinterpret_cast<const uint32_t*>(row + (16 * ks + kk) * 2);
                 qb[ks][1] = *reinterpret_cast<const uint32_t*>(row + (16 * ks + kk + 8) * 2);
+            } else {
+                qb[ks][0] = qb[ks][1] = 0u;
+            }
+        }
+    }
+
+    // Same, from global memory (the G rows of q of one kv head).
+    __device__ __forceinline__ void load_q_global(const uint8_t* gq, int lane, float qs_scale) {
+        qscale = qs_scale;
+        const int h = lane >> 2, kk = (lane & 3) * 2;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            if (h < G) {
+                const uint32_t* row = reinterpret_cast<const uint32_t*>(gq + h * D * 2);
+                qb[ks][0] = __ldg(row + (16 * ks + kk) / 2);
+                qb[ks][1] = __ldg(row + (16 * ks + kk + 8) / 2);
             } else {
                 qb[ks][0] = qb[ks][1] = 0u;
             }
@@ -397,40 +433,40 @@ struct MmaMath {
         }
     }
 
-    __device__ __forceinline__ void deposit(float* comb, int lane) const {
+    // Warp state -> dep: acc[h][d] (G*D floats), then m[h], then l[h].
+    __device__ __forceinline__ void deposit(float* dep, int lane) const {
         const int h0 = (lane & 3) * 2, d0 = lane >> 2;
 #pragma unroll
         for (int mt = 0; mt < KS; ++mt) {
             const int d = 16 * mt + d0;
             if (h0 < G) {
-                comb[h0 * D + d] = acc[mt][0];
-                comb[h0 * D + d + 8] = acc[mt][2];
+                dep[h0 * D + d] = acc[mt][0];
+                dep[h0 * D + d + 8] = acc[mt][2];
             }
             if (h0 + 1 < G) {
-                comb[(h0 + 1) * D + d] = acc[mt][1];
-                comb[(h0 + 1) * D + d + 8] = acc[mt][3];
+                dep[(h0 + 1) * D + d] = acc[mt][1];
+                dep[(h0 + 1) * D + d + 8] = acc[mt][3];
             }
         }
         if (d0 == 0) {
-            if (h0 < G) {
-                comb[G * D + h0] = m[0];
-                comb[G * D + G + h0] = l[0];
-            }
-            if (h0 + 1 < G) {
-                comb[G * D + h0 + 1] = m[1];
-                comb[G * D + G + h0 + 1] = l[1];
-            }
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+                if (h0 + e < G) {
+                    dep[G * D + h0 + e] = m[e];
+                    dep[G * D + G + h0 + e] = l[e];
+                }
         }
     }
 };
 
 // ===========================================================================
-template <int D, int G, int BS, int NW, int R>
+template <int D, int G, int BS, int NW, int R, int PPS>
 struct DecodeCfg {
     static constexpr int kRow = D * 2;              // bytes of one K or V row
     static constexpr int kTile = BS * kRow;         // one (block, kv head) tile
     static constexpr int kPanel = BS * 128;         // one 64-column panel of a tile
-    static constexpr int kStage = 2 * kTile;        // K tile then V tile
+    static constexpr int kPage = 2 * kTile;         // K tile then V tile
+    static constexpr int kStage = PPS * kPage;      // PPS pages of one segment
     static constexpr int kSegSlots = 4;
     static constexpr int kQBytes = G * kRow;
     static constexpr int kCombFloats = G * D + ((2 * G + 3) / 4) * 4;  // one warp's state, 16-byte padded
@@ -451,6 +487,30 @@ struct DecodeCfg {
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
+// Inclusive prefix sum of v over the NT threads of the CTA; the chunk total
+// goes to `total`.  red holds one slot per warp.
+template <int NT>
+__device__ __forceinline__ long long block_incl_scan(long long v, long long* red, long long& total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    long long incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const long long t = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += t;
+    }
+    if (lane == 31) red[warp] = incl;
+    __syncthreads();
+    long long before = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) {
+        if (w < warp) before += red[w];
+        tot += red[w];
+    }
+    __syncthreads();
+    total = tot;
+    return before + incl;
+}
+
 template <int BS>
 __device__ __forceinline__ int32_t clamp_len(const DecodeParams& p, int b, bool report) {
     int32_t L = __ldg(p.context_lens + b);
@@ -462,13 +522,13 @@ __device__ __forceinline__ int32_t clamp_len(const DecodeParams& p, int b, bool 
     return L;
 }
 
-template <int D, int G, int BS, int NW, int R, bool DUMP, template <int, int, int> class Math>
+template <int D, int G, int BS, int NW, int R, int PPS, bool DUMP, template <int, int, int> class Math>
 __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
     // Stage i % R always feeds warp i % NW, so a warp waiting on a stage is at
     // most one phase away from it and the parity waits are exact.
     static_assert(R % NW == 0, "ring depth must be a multiple of the consumer warps");
     static_assert(NW + 1 <= 16, "block reductions hold 16 warps");
-    using Cfg = DecodeCfg<D, G, BS, NW, R>;
+    using Cfg = DecodeCfg<D, G, BS, NW, R, PPS>;
     constexpr int S = Cfg::kSegSlots;
     constexpr int NT = Cfg::kThreads;
     constexpr int NPANEL = D / 64;
@@ -503,25 +563,29 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
         fence_mbar_init();
     }
 
-    // ---- pass 1: pages per kv head over all sequences; zero empty ones ----
-    long long local = 0;
-    for (int b = threadIdx.x; b < p.B; b += NT) {
-        const int32_t L = clamp_len<BS>(p, b, blockIdx.x == 0);
-        local += (L + BS - 1) / BS;
-        if (L == 0 && (b % int(gridDim.x)) == int(blockIdx.x)) {
-            uint4* o = reinterpret_cast<uint4*>(p.out + int64_t(b) * p.Hq * D);
-            for (int i = 0; i < p.Hq * D / 8; ++i) o[i] = make_uint4(0, 0, 0, 0);
+    // ---- the CTA's share: a scan of v_b = Hkv * pages(b) over the sequences;
+    // sequences with no context get zero output here.  When B fits in one
+    // chunk the same scan also locates the share's ends (no second read). ----
+    const bool one_chunk = p.B <= NT;
+    long long v_mine = 0, incl_mine = 0, Wt = 0;
+    for (int base = 0; base < p.B; base += NT) {
+        const int b = base + threadIdx.x;
+        long long v = 0;
+        if (b < p.B) {
+            const int32_t L = clamp_len<BS>(p, b, blockIdx.x == 0);
+            const int npb = (L + BS - 1) / BS;
+            v = (long long)(npb > 0 ? npb + p.seg_weight : 0) * p.Hkv;
+            if (L == 0 && (b % int(gridDim.x)) == int(blockIdx.x)) {
+                uint4* o = reinterpret_cast<uint4*>(p.out + int64_t(b) * p.Hq * D);
+                for (int i = 0; i < p.Hq * D / 8; ++i) o[i] = make_uint4(0, 0, 0, 0);
+            }
         }
+        long long chunk_total;
+        const long long incl = Wt + block_incl_scan<NT>(v, misc->red, chunk_total);  // first call also
+        Wt += chunk_total;                                                          // publishes mbar init
+        v_mine = v;
+        incl_mine = incl;
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) local += __shfl_xor_sync(0xffffffffu, local, off);
-    __syncthreads();  // also publishes the barrier initialisation
-    if (lane == 0) misc->red[warp] = local;
-    __syncthreads();
-    long long total = 0;
-#pragma unroll
-    for (int w = 0; w < NW + 1; ++w) total += misc->red[w];
-    const int64_t Wt = total * p.Hkv;  // all (b, g, page) work
     if (Wt == 0) return;
     const int64_t want = (Wt + p.min_pages - 1) / p.min_pages;
     const int64_t grid_eff = want < int64_t(gridDim.x) ? want : int64_t(gridDim.x);
@@ -529,124 +593,146 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
     const Split split{Wt / grid_eff, Wt % grid_eff};
     const int64_t p_start = split.start(blockIdx.x);
     const int64_t p_end = split.start(int64_t(blockIdx.x) + 1);
-    __syncthreads();  // misc->red reads done before reuse
 
-    // ---- pass 2: find the sequence holding p_start (chunked block scan) ----
-    long long carry = 0;
-    for (int base = 0; base < p.B; base += NT) {
-        const int b = base + threadIdx.x;
-        long long v = 0;
-        if (b < p.B) v = (long long)((clamp_len<BS>(p, b, false) + BS - 1) / BS) * p.Hkv;
-        long long incl = v;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const long long t = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += t;
-        }
-        if (lane == 31) misc->red[warp] = incl;
-        __syncthreads();
-        long long before = carry;
-        for (int w = 0; w < warp; ++w) before += misc->red[w];
-        long long chunk_total = 0;
-        for (int w = 0; w < NW + 1; ++w) chunk_total += misc->red[w];
-        const long long lo = before + incl - v;
-        if (v > 0 && lo <= p_start && p_start < lo + v) {
+    // ---- the sequence where the share starts ----
+    auto locate = [&](int b, long long v, long long incl) {
+        const long long lo = incl - v;
+        if (v > 0 && lo <= p_start && p_start < incl) {
             misc->b0 = b;
             misc->pre0 = lo;
-            misc->found = 1;
         }
-        carry += chunk_total;
-        __syncthreads();
-        if (misc->found) break;
+    };
+    if (one_chunk) {
+        locate(threadIdx.x, v_mine, incl_mine);
+    } else {
+        long long carry = 0;
+        for (int base = 0; base < p.B; base += NT) {
+            const int b = base + threadIdx.x;
+            long long v = 0;
+            if (b < p.B) {
+                const int npb = (clamp_len<BS>(p, b, false) + BS - 1) / BS;
+                v = (long long)(npb > 0 ? npb + p.seg_weight : 0) * p.Hkv;
+            }
+            long long chunk_total;
+            const long long incl = carry + block_incl_scan<NT>(v, misc->red, chunk_total);
+            locate(b, v, incl);
+            carry += chunk_total;
+        }
     }
+    __syncthreads();
 
     if (warp == NW) {
         // ======================= producer warp =======================
-        int b = misc->b0;
-        int64_t pre = misc->pre0;
-        int32_t Lb = clamp_len<BS>(p, b, false);
-        int32_t np = (Lb + BS - 1) / BS;
-        const int64_t off0 = p_start - pre;
-        int g = int(off0 / np);
-        int j = int(off0 - int64_t(g) * np);
-        int64_t pos = p_start;
-        uint32_t page_i = 0, seg_i = 0;
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_k)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_v)) : "memory");
+        }
+        uint32_t stage_i = 0, seg_i = 0;
         constexpr int C = R < 32 ? R : 32;
         bool ok = true;
         const uint64_t pol = PA_EVICT_FIRST ? policy_evict_first() : policy_evict_normal();
-        while (ok && pos < p_end) {
-            const int npg = int((int64_t(np - j) < p_end - pos) ? int64_t(np - j) : p_end - pos);
-            if (lane == 0) {
-                const int s = seg_i % S;
-                if (seg_i >= S) ok = mbar_wait(&segempty[s], ((seg_i / S) - 1) & 1, abort);
-                if (ok) {
-                    const int64_t bg_start = pre + int64_t(g) * np;
-                    SegDesc& d = descs[s];
-                    d.bg_start = bg_start;
-                    d.b = b;
-                    d.g = g;
-                    d.j0 = j;
-                    d.npg = npg;
-                    d.L = Lb;
-                    d.k0 = split.owner(bg_start);
-                    d.k1 = split.owner(bg_start + np - 1);
-                    d.first = seg_i == 0;
-                    mbar_arrive_expect_tx(&segfull[s], Cfg::kQBytes);
-                    bulk_g2s(qring + s * Cfg::kQBytes, p.q + (int64_t(b) * p.Hq + int64_t(g) * G) * Cfg::kRow,
-                             Cfg::kQBytes, &segfull[s]);
-                }
-            }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            const int32_t* bt = p.block_tables + int64_t(b) * p.M + j;
-            for (int c0 = 0; ok && c0 < npg; c0 += C) {
-                const int n = (npg - c0) < C ? (npg - c0) : C;
-                bool lane_ok = true;
-                if (lane < n) {
-                    int32_t blk = __ldg(bt + c0 + lane);
-                    if (blk < 0 || blk >= p.NB) {
-                        raise_error(PA_DEVERR_BLOCK_ID);
-                        blk = 0;
+
+        // walk the (b, g) whose units meet the share [p_start, p_end)
+        int b = misc->b0;
+        int32_t Lb = clamp_len<BS>(p, b, false);
+        int32_t np = (Lb + BS - 1) / BS;
+        int64_t unit = np + p.seg_weight;
+        int g = int((p_start - misc->pre0) / unit);
+        int64_t u0 = misc->pre0 + int64_t(g) * unit;  // line position of (b, g)'s first page
+        while (ok && u0 < p_end) {
+            const int64_t lo = p_start > u0 ? p_start : u0;
+            const int64_t hi = p_end < u0 + np ? p_end : u0 + np;
+            if (lo < hi) {
+                const int j = int(lo - u0);
+                const int npg = int(hi - lo);
+                if (lane == 0) {
+                    const int s = seg_i % S;
+                    if (seg_i >= S) ok = mbar_wait(&segempty[s], ((seg_i / S) - 1) & 1, abort);
+                    if (ok) {
+                        SegDesc& d = descs[s];
+                        d.b = b;
+                        d.g = g;
+                        d.j0 = j;
+                        d.npg = npg;
+                        d.L = Lb;
+                        d.k0 = split.owner(u0);
+                        d.k1 = split.owner(u0 + np - 1);
+                        mbar_arrive_expect_tx(&segfull[s], Cfg::kQBytes);
+                        bulk_g2s(qring + s * Cfg::kQBytes,
+                                 p.q + (int64_t(b) * p.Hq + int64_t(g) * G) * Cfg::kRow, Cfg::kQBytes,
+                                 &segfull[s]);
                     }
-                    const uint32_t i = page_i + c0 + lane;
-                    const int slot = int(i % R);
-                    const uint32_t use = i / R;
-                    if (PA_L2_PREFETCH && use > 0) {
-                        // start the DRAM read now; the load below waits for a free stage
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                // one lane per stage of PPS consecutive pages of the segment
+                const int32_t* bt = p.block_tables + int64_t(b) * p.M + j;
+                const int nst = (npg + PPS - 1) / PPS;
+                for (int c0 = 0; ok && c0 < nst; c0 += C) {
+                    const int n = (nst - c0) < C ? (nst - c0) : C;
+                    bool lane_ok = true;
+                    if (lane < n) {
+                        const int sj = (c0 + lane) * PPS;  // first page of the stage in the segment
+                        const int npst = (npg - sj) < PPS ? (npg - sj) : PPS;
+                        int32_t blk[PPS];
 #pragma unroll
-                        for (int pn = 0; pn < NPANEL; ++pn) {
-                            tma_prefetch_3d(&p.tmap_k, 0, pn, (blk * p.Hkv + g) * BS, pol);
-                            tma_prefetch_3d(&p.tmap_v, 0, pn, (blk * p.Hkv + g) * BS, pol);
+                        for (int q = 0; q < PPS; ++q) {
+                            blk[q] = 0;
+                            if (q < npst) {
+                                blk[q] = __ldg(bt + sj + q);
+                                if (blk[q] < 0 || blk[q] >= p.NB) {
+                                    raise_error(PA_DEVERR_BLOCK_ID);
+                                    blk[q] = 0;
+                                }
+                            }
+                        }
+                        const uint32_t i = stage_i + c0 + lane;
+                        const int slot = int(i % R);
+                        const uint32_t use = i / R;
+                        if (PA_L2_PREFETCH && use > 0) {
+                            // start the DRAM read now; the load below waits for a free stage
+#pragma unroll
+                            for (int q = 0; q < PPS; ++q)
+                                if (q < npst)
+#pragma unroll
+                                    for (int pn = 0; pn < NPANEL; ++pn) {
+                                        tma_prefetch_3d(&p.tmap_k, 0, pn, (blk[q] * p.Hkv + g) * BS, pol);
+                                        tma_prefetch_3d(&p.tmap_v, 0, pn, (blk[q] * p.Hkv + g) * BS, pol);
+                                    }
+                        }
+                        if (use > 0) lane_ok = mbar_wait(&empty[slot], (use - 1) & 1, abort);
+                        if (lane_ok) {
+                            uint8_t* st = ring + slot * Cfg::kStage;
+                            mbar_arrive_expect_tx(&full[slot], uint32_t(npst) * Cfg::kPage);
+#pragma unroll
+                            for (int q = 0; q < PPS; ++q) {
+                                if (q < npst) {
+                                    const int row = (blk[q] * p.Hkv + g) * BS;
+                                    uint8_t* pg = st + q * Cfg::kPage;
+#pragma unroll
+                                    for (int pn = 0; pn < NPANEL; ++pn) {
+                                        tma_load_3d(pg + pn * Cfg::kPanel, &p.tmap_k, 0, pn, row, &full[slot], pol);
+                                        tma_load_3d(pg + Cfg::kTile + pn * Cfg::kPanel, &p.tmap_v, 0, pn, row,
+                                                    &full[slot], pol);
+                                    }
+                                }
+                            }
                         }
                     }
-                    if (use > 0) lane_ok = mbar_wait(&empty[slot], (use - 1) & 1, abort);
-                    if (lane_ok) {
-                        uint8_t* st = ring + slot * Cfg::kStage;
-                        const int row = (blk * p.Hkv + g) * BS;
-                        mbar_arrive_expect_tx(&full[slot], 2 * Cfg::kTile);
-#pragma unroll
-                        for (int pn = 0; pn < NPANEL; ++pn) {
-                            tma_load_3d(st + pn * Cfg::kPanel, &p.tmap_k, 0, pn, row, &full[slot], pol);
-                            tma_load_3d(st + Cfg::kTile + pn * Cfg::kPanel, &p.tmap_v, 0, pn, row, &full[slot],
-                                        pol);
-                        }
-                    }
+                    ok = __all_sync(0xffffffffu, lane_ok);
                 }
-                ok = __all_sync(0xffffffffu, lane_ok);
+                stage_i += nst;
+                ++seg_i;
             }
-            page_i += npg;
-            ++seg_i;
-            pos += npg;
-            if (pos < p_end) {  // next (b, g)
-                j = 0;
-                if (++g == p.Hkv) {
-                    g = 0;
-                    pre += int64_t(p.Hkv) * np;
-                    do {
-                        ++b;
-                        Lb = clamp_len<BS>(p, b, false);
-                        np = (Lb + BS - 1) / BS;
-                    } while (np == 0);
-                }
+            // next (b, g) on the line (sequences without context take no units)
+            u0 += unit;
+            if (u0 < p_end && ++g == p.Hkv) {
+                g = 0;
+                do {
+                    ++b;
+                    Lb = clamp_len<BS>(p, b, false);
+                    np = (Lb + BS - 1) / BS;
+                } while (np == 0);
+                unit = np + p.seg_weight;
             }
         }
         if (ok && lane == 0) {  // end-of-share marker
@@ -661,7 +747,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
         if (!ok && lane == 0) {
             // Error path: the consumers may be gone; let every copy this warp
             // may have started land before the CTA's shared memory is freed.
-            const uint32_t last = page_i + C;
+            const uint32_t last = stage_i + C;
             for (uint32_t i = (last > R ? last - R : 0); i < last; ++i)
                 mbar_wait(&full[i % R], (i / R) & 1, nullptr, 20000000ull);
         }
@@ -671,7 +757,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
     // ========================= consumer warps =========================
     Math<D, G, BS> st;
     const int ct = threadIdx.x;  // 0 .. NW*32-1
-    uint32_t page_base = 0, seg_i = 0, cons_phase = 0;
+    uint32_t stage_base = 0, seg_i = 0, cons_phase = 0;
 
     auto rendezvous = [&]() -> bool {
         __syncwarp();
@@ -691,31 +777,38 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
         if (lane == 0) mbar_arrive(&segempty[s]);
         st.reset();
 
-        for (int k = int((uint32_t(warp) + NW - page_base % NW) % NW); k < d.npg; k += NW) {
-            const uint32_t i = page_base + k;
+        const int nst = (d.npg + PPS - 1) / PPS;
+        for (int k = int((uint32_t(warp) + NW - stage_base % NW) % NW); k < nst; k += NW) {
+            const uint32_t i = stage_base + k;
             const int slot = int(i % R);
             if (!mbar_wait(&full[slot], (i / R) & 1, abort)) return;
             uint8_t* stg = ring + slot * Cfg::kStage;
-            const int nv_raw = d.L - (d.j0 + k) * BS;
-            const int nv = nv_raw < BS ? nv_raw : BS;
-            if (Math<D, G, BS>::kZeroMaskedV && nv < BS) {
-                // rows past the context may hold anything (NaN included): clear
-                // them in the V tile so that 0 * row stays 0 in the tensor core
-                const int per_panel = (BS - nv) * 8;  // 16-byte chunks
-                for (int x = lane; x < NPANEL * per_panel; x += 32) {
-                    const int pn = x / per_panel, rem = x - pn * per_panel;
-                    const int t = nv + (rem >> 3), cch = rem & 7;
-                    *reinterpret_cast<uint4*>(stg + Cfg::kTile + pn * Cfg::kPanel + t * 128 + cch * 16) =
-                        make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int q = 0; q < PPS; ++q) {
+                const int pgi = k * PPS + q;  // page of the segment
+                if (pgi >= d.npg) break;
+                uint8_t* pg = stg + q * Cfg::kPage;
+                const int nv_raw = d.L - (d.j0 + pgi) * BS;
+                const int nv = nv_raw < BS ? nv_raw : BS;
+                if (Math<D, G, BS>::kZeroMaskedV && nv < BS) {
+                    // rows past the context may hold anything (NaN included): clear
+                    // them in the V tile so that 0 * row stays 0 in the tensor core
+                    const int per_panel = (BS - nv) * 8;  // 16-byte chunks
+                    for (int x = lane; x < NPANEL * per_panel; x += 32) {
+                        const int pn = x / per_panel, rem = x - pn * per_panel;
+                        const int t = nv + (rem >> 3), cch = rem & 7;
+                        *reinterpret_cast<uint4*>(pg + Cfg::kTile + pn * Cfg::kPanel + t * 128 + cch * 16) =
+                            make_uint4(0, 0, 0, 0);
+                    }
+                    __syncwarp();
+                    fence_proxy_async_smem();
                 }
-                __syncwarp();
-                fence_proxy_async_smem();
+                st.page(pg, pg + Cfg::kTile, nv, lane);
             }
-            st.page(stg, stg + Cfg::kTile, nv, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[slot]);
         }
-        page_base += d.npg;
+        stage_base += nst;
 
         // ---- segment end: combine the NW warp states ----
         st.finish();
@@ -724,7 +817,10 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
         if (!rendezvous()) return;
 
         const bool whole = d.k0 == d.k1;
-        const int my_slot = d.first ? 0 : 1;
+        // partial slot: the piece of the CTA that owns the segment's first page
+        // goes to slot 1 (it ends that CTA's share), any other piece to slot 0
+        // (it starts its CTA's share): at most one of each per CTA
+        const int my_slot = int(blockIdx.x) == d.k0 ? 1 : 0;
         if (DUMP) {
             if (ct == 0) misc->dump_idx = atomicAdd(p.seg_count, 1);
             if (!rendezvous()) return;
@@ -782,24 +878,53 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
             if (!rendezvous()) return;
             if (misc->is_last) {
                 __threadfence();
-                for (int o = ct; o < G * D; o += NW * 32) {
-                    const int h = o / D, dd = o - h * D;
+                // Every piece's (max, sum) goes to shared memory (the combine area
+                // is free again), then each thread merges 4 outputs with float4
+                // loads kept in flight, so the merge costs a few L2 round trips.
+                const int nk = d.k1 - d.k0 + 1;
+                float2* stage = reinterpret_cast<float2*>(comb);
+                const bool staged = nk * G * 2 <= NW * Cfg::kCombFloats;
+                if (staged) {
+                    for (int x = ct; x < nk * G; x += NW * 32) {
+                        const int k = d.k0 + x / G, h = x % G;
+                        const int64_t pk = int64_t(k) * 2 + (k == d.k0 ? 1 : 0);
+                        stage[x] = __ldcg(&p.part_ml[pk * G + h]);
+                    }
+                }
+                if (!rendezvous()) return;
+                for (int o4 = ct; o4 < G * D / 4; o4 += NW * 32) {
+                    const int h = (o4 * 4) / D, dd = o4 * 4 - h * D;
                     float M = -INFINITY;
-                    for (int k = d.k0; k <= d.k1; ++k) {
-                        const int sl = split.start(k) < d.bg_start ? 1 : 0;
-                        M = fmaxf(M, __ldcg(&p.part_ml[(int64_t(k) * 2 + sl) * G + h].x));
+                    for (int kk = 0; kk < nk; ++kk) {
+                        const int k = d.k0 + kk;
+                        const float mk =
+                            staged ? stage[kk * G + h].x
+                                   : __ldcg(&p.part_ml[(int64_t(k) * 2 + (k == d.k0 ? 1 : 0)) * G + h].x);
+                        M = fmaxf(M, mk);
                     }
-                    float lsum = 0.f, a = 0.f;
-                    for (int k = d.k0; k <= d.k1; ++k) {
-                        const int64_t ps = int64_t(k) * 2 + (split.start(k) < d.bg_start ? 1 : 0);
-                        const float2 ml = __ldcg(&p.part_ml[ps * G + h]);
+                    float lsum = 0.f;
+                    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+                    for (int kk = 0; kk < nk; ++kk) {
+                        const int k = d.k0 + kk;
+                        const int64_t pk = int64_t(k) * 2 + (k == d.k0 ? 1 : 0);
+                        const float2 ml = staged ? stage[kk * G + h] : __ldcg(&p.part_ml[pk * G + h]);
                         const float sc = ml.y * exp2f(ml.x - M);
+                        const float4 v = __ldcg(reinterpret_cast<const float4*>(&p.part_o[(pk * G + h) * D + dd]));
                         lsum += sc;
-                        a += sc * __ldcg(&p.part_o[(ps * G + h) * D + dd]);
+                        a.x += sc * v.x;
+                        a.y += sc * v.y;
+                        a.z += sc * v.z;
+                        a.w += sc * v.w;
                     }
-                    p.out[(int64_t(d.b) * p.Hq + int64_t(d.g) * G + h) * D + dd] = __float2bfloat16_rn(a / lsum);
+                    const float inv = 1.f / lsum;
+                    __nv_bfloat16* dst = p.out + (int64_t(d.b) * p.Hq + int64_t(d.g) * G + h) * D + dd;
+                    *reinterpret_cast<uint2*>(dst) =
+                        make_uint2(float2_to_bf16x2(a.x * inv, a.y * inv), float2_to_bf16x2(a.z * inv, a.w * inv));
                 }
                 if (ct == 0) p.counters[int64_t(d.b) * p.Hkv + d.g] = 0;
+                // the staged values are read before the next segment's deposit
+                if (!rendezvous()) return;
             }
         }
         ++seg_i;
