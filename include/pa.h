@@ -134,6 +134,25 @@ PA_API pa_status pa_decode(const void* q, const void* k_cache, const void* v_cac
                     void* stream);
 
 /*
+ * One decode step in one launch: the slot-mapped append of the step's new
+ * K/V rows (pa_cache_append) and then paged decode attention over the
+ * caches including those rows (pa_decode), fused.  Each CTA writes a slice
+ * of the rows, then all CTAs meet at a grid barrier (a cooperative launch,
+ * so all are resident) before any K/V page is read; the barrier wait
+ * overlaps the kernel's own set-up.  Arguments as for the two calls; the
+ * workspace as for pa_decode.  Compared with the two calls it saves the
+ * append's launch and its latency (miniVLLM docs index, "What is
+ * miniVLLM?": low-latency decode; the append and the decode of one step).
+ * After a call that set PA_DEVERR_TIMEOUT the workspace must be zero-filled
+ * again.
+ */
+PA_API pa_status pa_append_decode(const void* k_new, const void* v_new, const int32_t* slot_mapping,
+                                  int32_t num_tokens, const void* q, void* k_cache, void* v_cache,
+                                  const int32_t* block_tables, const int32_t* context_lens, float scale,
+                                  void* out, const pa_dims* dims, void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/*
  * Test hook: pa_decode on exactly `num_ctas` CTAs (which decides where
  * contexts are split), that also records every per-CTA segment it computes:
  * segment i covers tokens [t0, t1) of kv head g of sequence b and stores

@@ -57,6 +57,8 @@ def _load(path: str = LIB_PATH):
     lib.pa_decode_partials.argtypes = [vp, vp, vp, vp, vp, f32, vp, dp, i32, vp, sz, i32,
                                        vp, vp, vp, vp, vp, vp]
     lib.pa_decode_partials.restype = i32
+    lib.pa_append_decode.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, f32, vp, dp, vp, sz, vp]
+    lib.pa_append_decode.restype = i32
     lib.pa_decode_static_ws.argtypes = [vp, vp, vp, vp, vp, f32, vp, dp, vp]
     lib.pa_decode_static_ws.restype = i32
     lib.pa_device_errors.argtypes = [ctypes.POINTER(i32), i32]
@@ -70,7 +72,8 @@ lib = _load()
 
 # Every symbol include/pa.h declares.
 EXPORTS = ("pa_cache_append", "pa_decode_workspace_bytes", "pa_decode_default_ctas", "pa_decode",
-           "pa_decode_partials", "pa_decode_static_ws", "pa_device_errors", "pa_status_string")
+           "pa_append_decode", "pa_decode_partials", "pa_decode_static_ws", "pa_device_errors",
+           "pa_status_string")
 
 PA_ERR_SCRATCH_LIMIT = -7
 PA_STATIC_SCRATCH_BYTES = 4 << 20  # include/pa.h
@@ -179,6 +182,46 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale: float, out
     _check(lib.pa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                          _ptr(context_lens), float(scale), _ptr(out), ctypes.byref(dims),
                          _ptr(workspace), workspace.numel(), _stream(stream)), "pa_decode")
+
+
+def _append_args(k_new, v_new, slot_mapping, k_cache, v_cache):
+    for t, n in ((k_new, "k_new"), (v_new, "v_new")):
+        _need(t, torch.bfloat16, n, 3)
+    _need(slot_mapping, torch.int32, "slot_mapping", 1)
+    T = slot_mapping.shape[0]
+    NB, Hkv, bs, D = k_cache.shape
+    if k_new.shape != v_new.shape or k_new.shape[0] != T or k_new.shape[1:] != (Hkv, D):
+        raise ValueError("k_new/v_new must be [T][Hkv][D] of the cache")
+    return T
+
+
+def pa_append_decode(k_new, v_new, slot_mapping, q, k_cache, v_cache, block_tables, context_lens,
+                     scale: float, out, workspace=None, stream=None) -> None:
+    """One decode step in one launch: append the new K/V rows, then decode
+    (see include/pa.h)."""
+    dims = _decode_args(q, k_cache, v_cache, block_tables, context_lens, out)
+    T = _append_args(k_new, v_new, slot_mapping, k_cache, v_cache)
+    if workspace is None:
+        workspace = alloc_workspace(dims, device=q.device)
+    _need(workspace, torch.uint8, "workspace", 1)
+    _check(lib.pa_append_decode(_ptr(k_new), _ptr(v_new), _ptr(slot_mapping), T, _ptr(q),
+                                _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+                                float(scale), _ptr(out), ctypes.byref(dims), _ptr(workspace),
+                                workspace.numel(), _stream(stream)), "pa_append_decode")
+
+
+def prepare_append_decode(k_new, v_new, slot_mapping, q, k_cache, v_cache, block_tables, context_lens,
+                          scale: float, out, workspace, stream=None) -> "Prepared":
+    dims = _decode_args(q, k_cache, v_cache, block_tables, context_lens, out)
+    T = _append_args(k_new, v_new, slot_mapping, k_cache, v_cache)
+    _need(workspace, torch.uint8, "workspace", 1)
+    p = Prepared(lib.pa_append_decode,
+                 (_ptr(k_new), _ptr(v_new), _ptr(slot_mapping), T, _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                  _ptr(block_tables), _ptr(context_lens), float(scale), _ptr(out), ctypes.byref(dims),
+                  _ptr(workspace), workspace.numel(), _stream(stream)), "pa_append_decode")
+    p._keep = (dims, k_new, v_new, slot_mapping, q, k_cache, v_cache, block_tables, context_lens, out,
+               workspace)
+    return p
 
 
 def pa_decode_partials(q, k_cache, v_cache, block_tables, context_lens, scale: float, out,

@@ -118,8 +118,9 @@ int sm_count() {
 }
 
 // Workspace layout: [counters: B*Hkv int32][part_o: grid*2*G*D f32][part_ml: grid*2*G float2]
+// [grid barrier of the fused append + decode: 2 uint32]
 struct WsLayout {
-    size_t counters, part_o, part_ml, total;
+    size_t counters, part_o, part_ml, grid_bar, total;
 };
 
 WsLayout ws_layout(const pa_dims& d, int grid) {
@@ -128,7 +129,8 @@ WsLayout ws_layout(const pa_dims& d, int grid) {
     w.counters = 0;
     w.part_o = align_up(size_t(d.num_seqs) * d.num_kv_heads * 4, 256);
     w.part_ml = align_up(w.part_o + size_t(grid) * 2 * G * d.head_dim * 4, 256);
-    w.total = align_up(w.part_ml + size_t(grid) * 2 * G * 8, 256);
+    w.grid_bar = align_up(w.part_ml + size_t(grid) * 2 * G * 8, 256);
+    w.total = w.grid_bar + 256;
     return w;
 }
 
@@ -184,48 +186,63 @@ bool make_cache_map(CUtensorMap* map, const void* base, int64_t rows, int D, int
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <MathKind MK, int D, int G, bool DUMP>
+template <MathKind MK, int D, int G, bool DUMP, bool APPEND>
 pa_status launch_decode(const pa::DecodeParams& p, int grid, cudaStream_t stream) {
     constexpr int NW = Tune<MK, D, G>::NW, R = Tune<MK, D, G>::R, PPS = Tune<MK, D, G>::PPS;
     using Cfg = pa::DecodeCfg<D, G, kBlockSize, NW, R, PPS>;
     auto kern = [] {
         if constexpr (MK == MathKind::kMma)
-            return pa::decode_kernel<D, G, kBlockSize, NW, R, PPS, DUMP, pa::MmaMath>;
+            return pa::decode_kernel<D, G, kBlockSize, NW, R, PPS, DUMP, APPEND, pa::MmaMath>;
         else
-            return pa::decode_kernel<D, G, kBlockSize, NW, R, PPS, DUMP, pa::SimtMath>;
+            return pa::decode_kernel<D, G, kBlockSize, NW, R, PPS, DUMP, APPEND, pa::SimtMath>;
     }();
     static unsigned attr_done[kMaxDevices];
     if (!set_smem_once(kern, Cfg::kSmemBytes, attr_done)) return PA_ERR_CUDA;
-    kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(p);
+    if (APPEND) {
+        // the CTAs meet at a grid barrier: a cooperative launch guarantees they are all resident
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(Cfg::kThreads);
+        cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return PA_ERR_CUDA;
+    } else {
+        kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(p);
+    }
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-template <MathKind MK, bool DUMP>
+template <MathKind MK, bool DUMP, bool APPEND>
 pa_status dispatch_d_g(int D, int G, const pa::DecodeParams& p, int grid, cudaStream_t s) {
     if (D == 64) {
         switch (G) {
-            case 1: return launch_decode<MK, 64, 1, DUMP>(p, grid, s);
-            case 2: return launch_decode<MK, 64, 2, DUMP>(p, grid, s);
-            case 4: return launch_decode<MK, 64, 4, DUMP>(p, grid, s);
-            case 8: return launch_decode<MK, 64, 8, DUMP>(p, grid, s);
+            case 1: return launch_decode<MK, 64, 1, DUMP, APPEND>(p, grid, s);
+            case 2: return launch_decode<MK, 64, 2, DUMP, APPEND>(p, grid, s);
+            case 4: return launch_decode<MK, 64, 4, DUMP, APPEND>(p, grid, s);
+            case 8: return launch_decode<MK, 64, 8, DUMP, APPEND>(p, grid, s);
         }
     } else if (D == 128) {
         switch (G) {
-            case 1: return launch_decode<MK, 128, 1, DUMP>(p, grid, s);
-            case 2: return launch_decode<MK, 128, 2, DUMP>(p, grid, s);
-            case 4: return launch_decode<MK, 128, 4, DUMP>(p, grid, s);
+            case 1: return launch_decode<MK, 128, 1, DUMP, APPEND>(p, grid, s);
+            case 2: return launch_decode<MK, 128, 2, DUMP, APPEND>(p, grid, s);
+            case 4: return launch_decode<MK, 128, 4, DUMP, APPEND>(p, grid, s);
             case 8:
-                if constexpr (MK == MathKind::kMma) return launch_decode<MK, 128, 8, DUMP>(p, grid, s);
+                if constexpr (MK == MathKind::kMma) return launch_decode<MK, 128, 8, DUMP, APPEND>(p, grid, s);
                 break;
         }
     }
     return PA_ERR_UNSUPPORTED;
 }
 
-template <bool DUMP>
+template <bool DUMP, bool APPEND = false>
 pa_status dispatch_decode(int D, int G, const pa::DecodeParams& p, int grid, cudaStream_t s) {
-    return math_kind() == MathKind::kMma ? dispatch_d_g<MathKind::kMma, DUMP>(D, G, p, grid, s)
-                                         : dispatch_d_g<MathKind::kSimt, DUMP>(D, G, p, grid, s);
+    return math_kind() == MathKind::kMma ? dispatch_d_g<MathKind::kMma, DUMP, APPEND>(D, G, p, grid, s)
+                                         : dispatch_d_g<MathKind::kSimt, DUMP, APPEND>(D, G, p, grid, s);
 }
 
 // Shared validation of pa_decode and pa_decode_partials; fills p.
@@ -269,6 +286,7 @@ pa_status prepare_decode(const void* q, const void* k_cache, const void* v_cache
     p.counters = reinterpret_cast<int32_t*>(ws + w.counters);
     p.part_o = reinterpret_cast<float*>(ws + w.part_o);
     p.part_ml = reinterpret_cast<float2*>(ws + w.part_ml);
+    p.grid_bar = reinterpret_cast<unsigned int*>(ws + w.grid_bar);
     return PA_OK;
 }
 
@@ -385,6 +403,34 @@ pa_status pa_decode_partials(const void* q, const void* k_cache, const void* v_c
     p.seg_count = seg_count;
     return dispatch_decode<true>(dims->head_dim, dims->num_q_heads / dims->num_kv_heads, p, num_ctas,
                                  static_cast<cudaStream_t>(stream));
+}
+
+pa_status pa_append_decode(const void* k_new, const void* v_new, const int32_t* slot_mapping, int32_t num_tokens,
+                           const void* q, void* k_cache, void* v_cache, const int32_t* block_tables,
+                           const int32_t* context_lens, float scale, void* out, const pa_dims* dims, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+    if (!dims) return PA_ERR_NULL;
+    if (num_tokens < 0) return PA_ERR_SHAPE;
+    pa::DecodeParams p;
+    const int grid = sm_count();
+    const pa_status st = prepare_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, dims, grid,
+                                        workspace, workspace_bytes, p);
+    if (st != PA_OK) return st;
+    if (num_tokens > 0) {
+        if (!k_new || !v_new || !slot_mapping) return PA_ERR_NULL;
+        if (!aligned16(k_new) || !aligned16(v_new) || !aligned4(slot_mapping)) return PA_ERR_ALIGN;
+    }
+    if (dims->num_seqs == 0) {  // nothing to attend over: the append alone
+        return pa_cache_append(k_new, v_new, slot_mapping, num_tokens, k_cache, v_cache, dims, stream);
+    }
+    p.k_new = static_cast<const uint4*>(k_new);
+    p.v_new = static_cast<const uint4*>(v_new);
+    p.slot_mapping = slot_mapping;
+    p.app_chunks = int64_t(num_tokens) * dims->num_kv_heads * (dims->head_dim / 8);
+    p.k_cache_w = static_cast<uint4*>(k_cache);
+    p.v_cache_w = static_cast<uint4*>(v_cache);
+    return dispatch_decode<false, true>(dims->head_dim, dims->num_q_heads / dims->num_kv_heads, p, grid,
+                                        static_cast<cudaStream_t>(stream));
 }
 
 pa_status pa_decode_static_ws(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,

@@ -77,6 +77,14 @@ struct DecodeParams {
     float* seg_m;
     float* seg_l;
     int32_t* seg_count;
+    // fused append (APPEND): slot-mapped rows written before any page is read
+    const uint4* k_new;           // [T][Hkv][D] bf16 as 16-byte chunks
+    const uint4* v_new;
+    const int32_t* slot_mapping;  // [T]
+    int64_t app_chunks;           // T * Hkv * D / 8
+    uint4* k_cache_w;             // the caches, writable
+    uint4* v_cache_w;
+    unsigned int* grid_bar;       // {arrivals, departures}: zero between calls
 };
 
 // One segment of a CTA's share, handed from the producer to the consumers.
@@ -522,7 +530,7 @@ __device__ __forceinline__ int32_t clamp_len(const DecodeParams& p, int b, bool 
     return L;
 }
 
-template <int D, int G, int BS, int NW, int R, int PPS, bool DUMP, template <int, int, int> class Math>
+template <int D, int G, int BS, int NW, int R, int PPS, bool DUMP, bool APPEND, template <int, int, int> class Math>
 __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
     // Stage i % R always feeds warp i % NW, so a warp waiting on a stage is at
     // most one phase away from it and the parity waits are exact.
@@ -563,6 +571,35 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
         fence_mbar_init();
     }
 
+    if (APPEND) {
+        // This CTA's slice of the slot-mapped append (the bit copy of
+        // pa::append_kernel), then arrival at the grid barrier; the rows must
+        // be visible to the TMA loads of every CTA before any page is read.
+        const int64_t per = (p.app_chunks + gridDim.x - 1) / gridDim.x;
+        const int64_t c0 = int64_t(blockIdx.x) * per;
+        const int64_t c1 = c0 + per < p.app_chunks ? c0 + per : p.app_chunks;
+        constexpr int CPR = D / 8;  // 16-byte chunks per row
+        for (int64_t idx = c0 + threadIdx.x; idx < c1; idx += NT) {
+            const int64_t t = idx / (int64_t(p.Hkv) * CPR);
+            const int64_t rem = idx - t * p.Hkv * CPR;
+            const int32_t slot = __ldg(p.slot_mapping + t);
+            if (slot < 0) continue;
+            const int64_t block = slot / BS, offset = slot - (slot / BS) * BS;
+            if (block >= p.NB) {
+                if (rem == 0) raise_error(PA_DEVERR_SLOT);
+                continue;
+            }
+            const int64_t g = rem / CPR, c = rem - g * CPR;
+            const int64_t dst = ((block * p.Hkv + g) * BS + offset) * CPR + c;
+            p.k_cache_w[dst] = __ldg(p.k_new + idx);
+            p.v_cache_w[dst] = __ldg(p.v_new + idx);
+        }
+        fence_proxy_async_global();
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) atomicAdd(&p.grid_bar[0], 1u);
+    }
+
     // ---- the CTA's share: a scan of v_b = Hkv * pages(b) over the sequences;
     // sequences with no context get zero output here.  When B fits in one
     // chunk the same scan also locates the share's ends (no second read). ----
@@ -585,6 +622,28 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
         Wt += chunk_total;                                                          // publishes mbar init
         v_mine = v;
         incl_mine = incl;
+    }
+    if (APPEND) {
+        // wait for every CTA's rows (all CTAs are resident: a cooperative
+        // launch); the last CTA through resets the barrier for the next call
+        if (threadIdx.x == 0) {
+            const uint64_t t0 = globaltimer_ns();
+            for (uint32_t it = 0; ld_acquire_gpu(&p.grid_bar[0]) < gridDim.x; ++it) {
+                __nanosleep(32);
+                if ((it & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) {
+                    raise_error(PA_DEVERR_TIMEOUT);
+                    misc->abort = 1;
+                    break;
+                }
+            }
+            if (atomicAdd(&p.grid_bar[1], 1u) == gridDim.x - 1) {
+                p.grid_bar[0] = 0;
+                p.grid_bar[1] = 0;
+            }
+        }
+        __syncthreads();
+        fence_proxy_async_global();
+        if (misc->abort) return;
     }
     if (Wt == 0) return;
     const int64_t want = (Wt + p.min_pages - 1) / p.min_pages;

@@ -90,7 +90,7 @@ def test_workspace_size_formula(binding):
     n = binding.pa_decode_workspace_bytes(d, 148)
     G = 4
     need = 64 * 8 * 4 + 148 * 2 * G * 128 * 4 + 148 * 2 * G * 8
-    assert need <= n <= need + 3 * 256
+    assert need <= n <= need + 4 * 256  # + alignment and the fused path's grid barrier
     with pytest.raises(ValueError):
         binding.pa_decode_workspace_bytes(_dims(binding, num_kv_heads=3), 148)
 

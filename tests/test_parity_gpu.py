@@ -277,3 +277,69 @@ def test_append_skips_padding_and_touches_nothing_else(pa, oracle_lib):
     pa.pa_cache_append(kn.to(d), vn.to(d), slots.to(d), t["k_cache"], t["v_cache"])
     torch.cuda.synchronize()
     _assert_caches_equal(t, kb, vb)
+
+
+@pytest.mark.parametrize("name", ["tiny", "qwen3", "llama32", "longskew", "prefix"])
+def test_fused_append_decode_matches_oracle(pa, oracle_lib, name):
+    # one launch: every CTA appends a slice of the rows, a grid barrier, then decode
+    from paged_kv_attention_36_b200 import workloads
+    w = workloads.make(name, poison=name in ("tiny", "qwen3", "prefix"))
+    kb, vb, ref = _oracle_step(oracle_lib, w)
+    t = _to_dev(w)
+    out = torch.empty_like(t["q"])
+    pa.pa_append_decode(t["k_new"], t["v_new"], t["slot_mapping"], t["q"], t["k_cache"], t["v_cache"],
+                        t["block_tables"], t["context_lens"], w.scale, out)
+    torch.cuda.synchronize()
+    _assert_caches_equal(t, kb, vb)
+    _assert_close(out, ref)
+    assert pa.pa_device_errors(clear=True) == 0
+
+
+def test_fused_repeat_calls_reset_the_grid_barrier(pa, oracle_lib):
+    from paged_kv_attention_36_b200 import workloads
+    w = workloads.make("qwen3")
+    kb, vb, ref = _oracle_step(oracle_lib, w)
+    t = _to_dev(w)
+    dims = pa.make_dims(t["q"], t["k_cache"], t["block_tables"])
+    ws = pa.alloc_workspace(dims)
+    for _ in range(4):
+        out = torch.empty_like(t["q"])
+        pa.pa_append_decode(t["k_new"], t["v_new"], t["slot_mapping"], t["q"], t["k_cache"],
+                            t["v_cache"], t["block_tables"], t["context_lens"], w.scale, out, workspace=ws)
+        torch.cuda.synchronize()
+        _assert_close(out, ref)
+        assert int(ws[-256:].view(torch.int32).abs().sum()) == 0  # barrier counters back to zero
+    _assert_caches_equal(t, kb, vb)
+    assert pa.pa_device_errors(clear=True) == 0
+
+
+def test_fused_append_reads_rows_written_by_other_ctas(pa, oracle_lib):
+    # slots of tokens appended to sequences whose pages other CTAs read:
+    # every token goes to a different sequence's last page, in reverse order
+    from paged_kv_attention_36_b200 import workloads
+    w = workloads.make("llama32")
+    perm = torch.arange(w.q.shape[0] - 1, -1, -1)
+    w.k_new, w.v_new = w.k_new[perm].contiguous(), w.v_new[perm].contiguous()
+    w.slot_mapping = w.slot_mapping[perm].contiguous()
+    kb, vb, ref = _oracle_step(oracle_lib, w)
+    t = _to_dev(w)
+    out = torch.empty_like(t["q"])
+    pa.pa_append_decode(t["k_new"], t["v_new"], t["slot_mapping"], t["q"], t["k_cache"], t["v_cache"],
+                        t["block_tables"], t["context_lens"], w.scale, out)
+    torch.cuda.synchronize()
+    _assert_caches_equal(t, kb, vb)
+    _assert_close(out, ref)
+
+
+def test_fused_reports_bad_slot(pa):
+    d = torch.device("cuda")
+    q = torch.randn((2, 8, 64), device=d).to(torch.bfloat16)
+    kc = torch.randn((4, 2, 16, 64), device=d).to(torch.bfloat16)
+    bt = torch.tensor([[0, 1], [2, 3]], dtype=torch.int32, device=d)
+    cl = torch.tensor([20, 5], dtype=torch.int32, device=d)
+    kn = torch.randn((2, 2, 64), device=d).to(torch.bfloat16)
+    sm = torch.tensor([3, 4 * 16 + 1], dtype=torch.int32, device=d)   # second slot past the pool
+    out = torch.empty_like(q)
+    pa.pa_device_errors(clear=True)
+    pa.pa_append_decode(kn, kn, sm, q, kc, kc.clone(), bt, cl, 0.125, out)
+    assert pa.pa_device_errors(clear=True) & pa.PA_DEVERR_SLOT
