@@ -75,6 +75,7 @@ typedef enum pa_status {
 #define PA_DEVERR_CONTEXT 0x2   /* a context_len was outside [0, max_blocks_per_seq*block_size] */
 #define PA_DEVERR_SLOT 0x4      /* an append slot was >= num_blocks*block_size */
 #define PA_DEVERR_TIMEOUT 0x8   /* a bounded pipeline wait gave up (internal error) */
+#define PA_DEVERR_PREFIX 0x10   /* pa_decode_shared_prefix: a group broke its contract (see there) */
 
 typedef struct pa_dims {
     int32_t num_seqs;           /* B */
@@ -200,6 +201,53 @@ PA_API pa_status pa_decode_partials(const void* q, const void* k_cache, const vo
 PA_API pa_status pa_decode_static_ws(const void* q, const void* k_cache, const void* v_cache,
                                      const int32_t* block_tables, const int32_t* context_lens,
                                      float scale, void* out, const pa_dims* dims, void* stream);
+
+/*
+ * Shared-prefix ("cascade") decode: pa_decode (optionally fused with the
+ * append, as pa_append_decode) for a batch in which runs of consecutive
+ * sequences share the first pages of their contexts, as prefix caching
+ * leaves them (miniVLLM docs index, "What is miniVLLM?": a paged KV cache
+ * with prefix caching; Mini-SGLang write-up, "Key optimizations": Radix
+ * Cache reuse of the KV of a common prefix across requests).  The result
+ * is the formula at the top of this file; only the order of the work
+ * differs.  Group i is the sequences
+ *     b in [group_offsets[i], group_offsets[i+1])
+ * whose block_tables rows all begin with the same P_i = group_prefix_pages[i]
+ * block ids (whole blocks: P_i*bs tokens).  First the queries of all members
+ * attend to the P_i shared pages together, each page read once per group
+ * (a dense [members*G x 16] x [16 x D] tensor-core product per page), giving
+ * split-KV partials; then the decode streams only each member's own pages
+ * P_i .. ceil(L_b/bs)-1 and merges the prefix partials by log-sum-exp.
+ *   - group_offsets [num_groups+1] and group_prefix_pages [num_groups] are
+ *     DEVICE int32 arrays; offsets non-decreasing, 0 <= off[0],
+ *     off[num_groups] <= B.  Sequences outside every group, and groups with
+ *     P_i = 0, are decoded as by pa_decode.
+ *   - max_group_size >= every off[i+1] - off[i] (a host value: it sizes
+ *     the grid and the workspace).
+ *   - A member with L_b < P_i*bs, or past max_group_size in its group, is
+ *     decoded over its whole table and PA_DEVERR_PREFIX is set; so it is
+ *     for offsets out of order or range, P_i > M, and a member whose table
+ *     does not begin with the group's first member's P_i block ids (the
+ *     output of such members is unspecified).
+ *   - num_tokens > 0 also appends k_new/v_new at slot_mapping first, fused
+ *     into the decode launch as in pa_append_decode; slots must not fall in
+ *     the shared blocks (the prefix pass runs before the append).
+ *     num_tokens = 0 skips the append (k_new, v_new, slot_mapping unused).
+ *   - Supported shapes and alignment as for pa_decode.  The workspace must
+ *     be at least pa_decode_shared_prefix_workspace_bytes(dims, num_groups,
+ *     max_group_size) bytes, zero-filled before its first use, and is left
+ *     ready for the next call; calls that share it must not overlap.
+ *   - num_groups = 0 is pa_decode / pa_append_decode with this workspace.
+ */
+PA_API size_t pa_decode_shared_prefix_workspace_bytes(const pa_dims* dims, int32_t num_groups,
+                                                      int32_t max_group_size);
+PA_API pa_status pa_decode_shared_prefix(const void* k_new, const void* v_new, const int32_t* slot_mapping,
+                                         int32_t num_tokens, const void* q, void* k_cache, void* v_cache,
+                                         const int32_t* block_tables, const int32_t* context_lens, float scale,
+                                         const int32_t* group_offsets, const int32_t* group_prefix_pages,
+                                         int32_t num_groups, int32_t max_group_size, void* out,
+                                         const pa_dims* dims, void* workspace, size_t workspace_bytes,
+                                         void* stream);
 
 /*
  * Reads (and, if `clear` != 0, resets) the device error word of the

@@ -21,6 +21,7 @@ PA_DEVERR_BLOCK_ID = 0x1
 PA_DEVERR_CONTEXT = 0x2
 PA_DEVERR_SLOT = 0x4
 PA_DEVERR_TIMEOUT = 0x8
+PA_DEVERR_PREFIX = 0x10
 
 
 class PaError(RuntimeError):
@@ -59,6 +60,11 @@ def _load(path: str = LIB_PATH):
     lib.pa_decode_partials.restype = i32
     lib.pa_append_decode.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, f32, vp, dp, vp, sz, vp]
     lib.pa_append_decode.restype = i32
+    lib.pa_decode_shared_prefix_workspace_bytes.argtypes = [dp, i32, i32]
+    lib.pa_decode_shared_prefix_workspace_bytes.restype = sz
+    lib.pa_decode_shared_prefix.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, f32, vp, vp, i32, i32,
+                                            vp, dp, vp, sz, vp]
+    lib.pa_decode_shared_prefix.restype = i32
     lib.pa_decode_static_ws.argtypes = [vp, vp, vp, vp, vp, f32, vp, dp, vp]
     lib.pa_decode_static_ws.restype = i32
     lib.pa_device_errors.argtypes = [ctypes.POINTER(i32), i32]
@@ -72,7 +78,8 @@ lib = _load()
 
 # Every symbol include/pa.h declares.
 EXPORTS = ("pa_cache_append", "pa_decode_workspace_bytes", "pa_decode_default_ctas", "pa_decode",
-           "pa_append_decode", "pa_decode_partials", "pa_decode_static_ws", "pa_device_errors",
+           "pa_append_decode", "pa_decode_partials", "pa_decode_static_ws",
+           "pa_decode_shared_prefix_workspace_bytes", "pa_decode_shared_prefix", "pa_device_errors",
            "pa_status_string")
 
 PA_ERR_SCRATCH_LIMIT = -7
@@ -255,6 +262,69 @@ def pa_decode_static_ws(q, k_cache, v_cache, block_tables, context_lens, scale: 
     _check(lib.pa_decode_static_ws(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                                    _ptr(context_lens), float(scale), _ptr(out), ctypes.byref(dims),
                                    _stream(stream)), "pa_decode_static_ws")
+
+
+def pa_decode_shared_prefix_workspace_bytes(dims: pa_dims, num_groups: int, max_group_size: int) -> int:
+    n = lib.pa_decode_shared_prefix_workspace_bytes(ctypes.byref(dims), int(num_groups), int(max_group_size))
+    if n == 0:
+        raise ValueError(f"invalid dims {dims!r} / groups ({num_groups}, {max_group_size})")
+    return int(n)
+
+
+def _prefix_args(group_offsets, group_prefix_pages, max_group_size):
+    _need(group_offsets, torch.int32, "group_offsets", 1)
+    _need(group_prefix_pages, torch.int32, "group_prefix_pages", 1)
+    G = group_prefix_pages.shape[0]
+    if group_offsets.shape[0] != G + 1:
+        raise ValueError("group_offsets must have num_groups + 1 entries")
+    if G > 0 and int(max_group_size) <= 0:
+        raise ValueError("max_group_size must be positive")
+    return G
+
+
+def _shared_prefix_call(k_new, v_new, slot_mapping, q, k_cache, v_cache, block_tables, context_lens,
+                        scale, group_offsets, group_prefix_pages, max_group_size, out, workspace, stream):
+    dims = _decode_args(q, k_cache, v_cache, block_tables, context_lens, out)
+    T = 0
+    if slot_mapping is not None:
+        T = _append_args(k_new, v_new, slot_mapping, k_cache, v_cache)
+    ng = _prefix_args(group_offsets, group_prefix_pages, max_group_size)
+    if workspace is None:
+        workspace = torch.zeros(pa_decode_shared_prefix_workspace_bytes(dims, ng, max_group_size),
+                                dtype=torch.uint8, device=q.device)
+    _need(workspace, torch.uint8, "workspace", 1)
+    args = (_ptr(k_new), _ptr(v_new), _ptr(slot_mapping), T, _ptr(q), _ptr(k_cache), _ptr(v_cache),
+            _ptr(block_tables), _ptr(context_lens), float(scale), _ptr(group_offsets),
+            _ptr(group_prefix_pages), ng, int(max_group_size), _ptr(out), ctypes.byref(dims),
+            _ptr(workspace), workspace.numel(), _stream(stream))
+    keep = (dims, k_new, v_new, slot_mapping, q, k_cache, v_cache, block_tables, context_lens,
+            group_offsets, group_prefix_pages, out, workspace)
+    return args, keep
+
+
+def pa_decode_shared_prefix(q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                            group_offsets, group_prefix_pages, max_group_size: int, out,
+                            k_new=None, v_new=None, slot_mapping=None, workspace=None, stream=None) -> None:
+    """Decode of a batch whose groups of consecutive sequences share their
+    first blocks: group i = sequences [group_offsets[i], group_offsets[i+1])
+    sharing group_prefix_pages[i] blocks (see include/pa.h).  With
+    ``slot_mapping`` given, the step's new K/V rows are appended first, in
+    the same launch as the decode."""
+    args, _ = _shared_prefix_call(k_new, v_new, slot_mapping, q, k_cache, v_cache, block_tables,
+                                  context_lens, scale, group_offsets, group_prefix_pages, max_group_size,
+                                  out, workspace, stream)
+    _check(lib.pa_decode_shared_prefix(*args), "pa_decode_shared_prefix")
+
+
+def prepare_decode_shared_prefix(q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                                 group_offsets, group_prefix_pages, max_group_size: int, out, workspace,
+                                 k_new=None, v_new=None, slot_mapping=None, stream=None) -> "Prepared":
+    args, keep = _shared_prefix_call(k_new, v_new, slot_mapping, q, k_cache, v_cache, block_tables,
+                                     context_lens, scale, group_offsets, group_prefix_pages,
+                                     max_group_size, out, workspace, stream)
+    p = Prepared(lib.pa_decode_shared_prefix, args, "pa_decode_shared_prefix")
+    p._keep = keep
+    return p
 
 
 def pa_device_errors(clear: bool = False) -> int:

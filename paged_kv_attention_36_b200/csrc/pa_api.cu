@@ -1,8 +1,8 @@
 // pa_api.cu -- the extern "C" entry points of libpa_b200.so (declared and
 // documented in include/pa.h): host-side validation, workspace layout,
 // grid choice and kernel dispatch.  Every step of the computation runs in
-// the kernels of pa_append.cuh and pa_decode.cuh; there is no host or CPU
-// fallback.
+// the kernels of pa_append.cuh, pa_prefix.cuh and pa_decode.cuh; there is no
+// host or CPU fallback.
 #include <cudaTypedefs.h>
 
 #include <cstdlib>
@@ -12,6 +12,7 @@
 #include "pa_append.cuh"
 #include "pa_decode.cuh"
 #include "pa_device.cuh"
+#include "pa_prefix.cuh"
 
 namespace {
 
@@ -245,6 +246,68 @@ pa_status dispatch_decode(int D, int G, const pa::DecodeParams& p, int grid, cud
                                          : dispatch_d_g<MathKind::kSimt, DUMP, APPEND>(D, G, p, grid, s);
 }
 
+// ---- shared-prefix pass ----------------------------------------------------
+constexpr int kPrefixNW = 8;      // consumer warps: 128 query rows per CTA
+constexpr int kPrefixStages = 8;  // ring of K+V pages
+constexpr int kMaxPrefixSplits = 16;
+
+int prefix_tiles(const pa_dims& d, int max_group_size) {
+    const int64_t rows = int64_t(max_group_size) * (d.num_q_heads / d.num_kv_heads);
+    return int((rows + 16 * kPrefixNW - 1) / (16 * kPrefixNW));
+}
+
+// Key ranges per (group, row tile, kv head): enough CTAs for one wave.
+int prefix_splits(const pa_dims& d, int num_groups, int max_group_size, int sms) {
+    const int64_t base = int64_t(num_groups) * prefix_tiles(d, max_group_size) * d.num_kv_heads;
+    int64_t s = base > 0 ? sms / base : 1;
+    if (s < 1) s = 1;
+    if (s > kMaxPrefixSplits) s = kMaxPrefixSplits;
+    return int(s);
+}
+
+// The prefix partials follow the decode workspace: [o: splits*B*Hq*D f32][ml: splits*B*Hq float2]
+struct PrefixWs {
+    size_t o, ml, total;
+};
+
+PrefixWs prefix_ws(const pa_dims& d, size_t base, int splits) {
+    const size_t rows = size_t(splits) * d.num_seqs * d.num_q_heads;
+    PrefixWs w;
+    w.o = align_up(base, 256);
+    w.ml = align_up(w.o + rows * d.head_dim * 4, 256);
+    w.total = w.ml + rows * 8;
+    return w;
+}
+
+template <int D, int G>
+pa_status launch_prefix(const pa::PrefixParams& p, dim3 grid, cudaStream_t stream) {
+    using Cfg = pa::PrefixCfg<D, kPrefixNW, kPrefixStages>;
+    auto kern = pa::prefix_kernel<D, G, kPrefixNW, kPrefixStages>;
+    static unsigned attr_done[kMaxDevices];
+    if (!set_smem_once(kern, Cfg::kSmemBytes, attr_done)) return PA_ERR_CUDA;
+    kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status dispatch_prefix(int D, int G, const pa::PrefixParams& p, dim3 grid, cudaStream_t s) {
+    if (D == 64) {
+        switch (G) {
+            case 1: return launch_prefix<64, 1>(p, grid, s);
+            case 2: return launch_prefix<64, 2>(p, grid, s);
+            case 4: return launch_prefix<64, 4>(p, grid, s);
+            case 8: return launch_prefix<64, 8>(p, grid, s);
+        }
+    } else if (D == 128) {
+        switch (G) {
+            case 1: return launch_prefix<128, 1>(p, grid, s);
+            case 2: return launch_prefix<128, 2>(p, grid, s);
+            case 4: return launch_prefix<128, 4>(p, grid, s);
+            case 8: return launch_prefix<128, 8>(p, grid, s);
+        }
+    }
+    return PA_ERR_UNSUPPORTED;
+}
+
 // Shared validation of pa_decode and pa_decode_partials; fills p.
 pa_status prepare_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
                          const int32_t* context_lens, float scale, void* out, const pa_dims* dims, int grid,
@@ -431,6 +494,89 @@ pa_status pa_append_decode(const void* k_new, const void* v_new, const int32_t* 
     p.v_cache_w = static_cast<uint4*>(v_cache);
     return dispatch_decode<false, true>(dims->head_dim, dims->num_q_heads / dims->num_kv_heads, p, grid,
                                         static_cast<cudaStream_t>(stream));
+}
+
+size_t pa_decode_shared_prefix_workspace_bytes(const pa_dims* dims, int32_t num_groups, int32_t max_group_size) {
+    if (!dims_ok(dims) || num_groups < 0 || (num_groups > 0 && max_group_size <= 0)) return 0;
+    const int grid = sm_count();
+    if (grid <= 0) return 0;
+    const size_t base = ws_layout(*dims, grid).total;
+    if (num_groups == 0) return base;
+    const int mgs = max_group_size < dims->num_seqs ? max_group_size : dims->num_seqs;
+    return prefix_ws(*dims, base, prefix_splits(*dims, num_groups, mgs, grid)).total;
+}
+
+pa_status pa_decode_shared_prefix(const void* k_new, const void* v_new, const int32_t* slot_mapping,
+                                  int32_t num_tokens, const void* q, void* k_cache, void* v_cache,
+                                  const int32_t* block_tables, const int32_t* context_lens, float scale,
+                                  const int32_t* group_offsets, const int32_t* group_prefix_pages, int32_t num_groups,
+                                  int32_t max_group_size, void* out, const pa_dims* dims, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+    if (!dims) return PA_ERR_NULL;
+    if (num_tokens < 0 || num_groups < 0 || (num_groups > 0 && max_group_size <= 0)) return PA_ERR_SHAPE;
+    pa::DecodeParams p;
+    const int grid = sm_count();
+    const pa_status st = prepare_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, dims, grid,
+                                        workspace, workspace_bytes, p);
+    if (st != PA_OK) return st;
+    if (num_tokens > 0) {
+        if (!k_new || !v_new || !slot_mapping) return PA_ERR_NULL;
+        if (!aligned16(k_new) || !aligned16(v_new) || !aligned4(slot_mapping)) return PA_ERR_ALIGN;
+    }
+    const pa_dims& d = *dims;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (d.num_seqs == 0)
+        return num_tokens > 0 ? pa_cache_append(k_new, v_new, slot_mapping, num_tokens, k_cache, v_cache, dims, stream)
+                              : PA_OK;
+    const int G = d.num_q_heads / d.num_kv_heads;
+    if (num_groups > 0) {
+        if (!group_offsets || !group_prefix_pages) return PA_ERR_NULL;
+        if (!aligned4(group_offsets) || !aligned4(group_prefix_pages)) return PA_ERR_ALIGN;
+        const int mgs = max_group_size < d.num_seqs ? max_group_size : d.num_seqs;
+        const int splits = prefix_splits(d, num_groups, mgs, grid);
+        const PrefixWs w = prefix_ws(d, ws_layout(d, grid).total, splits);
+        if (workspace_bytes < w.total) return PA_ERR_WORKSPACE;
+        const int tiles = prefix_tiles(d, mgs);
+        if (int64_t(num_groups) * tiles > 0x7fffffffLL || d.num_kv_heads > 65535) return PA_ERR_SHAPE;
+        uint8_t* ws = static_cast<uint8_t*>(workspace);
+        pa::PrefixParams pp;
+        pp.tmap_k = p.tmap_k;
+        pp.tmap_v = p.tmap_v;
+        pp.q = p.q;
+        pp.block_tables = block_tables;
+        pp.context_lens = context_lens;
+        pp.group_offsets = group_offsets;
+        pp.group_prefix_pages = group_prefix_pages;
+        pp.num_groups = num_groups;
+        pp.max_group_size = mgs;
+        pp.tiles_per_group = tiles;
+        pp.B = d.num_seqs;
+        pp.Hq = d.num_q_heads;
+        pp.Hkv = d.num_kv_heads;
+        pp.NB = d.num_blocks;
+        pp.M = d.max_blocks_per_seq;
+        pp.qscale = p.qscale;
+        pp.prefix_o = reinterpret_cast<float*>(ws + w.o);
+        pp.prefix_ml = reinterpret_cast<float2*>(ws + w.ml);
+        const pa_status ps = dispatch_prefix(d.head_dim, G, pp, dim3(unsigned(num_groups * tiles),
+                                                                     unsigned(d.num_kv_heads), unsigned(splits)), s);
+        if (ps != PA_OK) return ps;
+        p.group_offsets = group_offsets;
+        p.group_prefix_pages = group_prefix_pages;
+        p.num_groups = num_groups;
+        p.max_group_size = mgs;
+        p.prefix_splits = splits;
+        p.prefix_o = pp.prefix_o;
+        p.prefix_ml = pp.prefix_ml;
+    }
+    if (num_tokens == 0) return dispatch_decode<false>(d.head_dim, G, p, grid, s);
+    p.k_new = static_cast<const uint4*>(k_new);
+    p.v_new = static_cast<const uint4*>(v_new);
+    p.slot_mapping = slot_mapping;
+    p.app_chunks = int64_t(num_tokens) * d.num_kv_heads * (d.head_dim / 8);
+    p.k_cache_w = static_cast<uint4*>(k_cache);
+    p.v_cache_w = static_cast<uint4*>(v_cache);
+    return dispatch_decode<false, true>(d.head_dim, G, p, grid, s);
 }
 
 pa_status pa_decode_static_ws(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,

@@ -46,6 +46,7 @@
 #pragma once
 
 #include "pa_device.cuh"
+#include "pa_prefix.cuh"
 
 #ifndef PA_EVICT_FIRST
 #define PA_EVICT_FIRST 1  // K/V pages are read once: first candidates for L2 eviction
@@ -85,6 +86,14 @@ struct DecodeParams {
     uint4* k_cache_w;             // the caches, writable
     uint4* v_cache_w;
     unsigned int* grid_bar;       // {arrivals, departures}: zero between calls
+    // shared prefixes (num_groups > 0): group i = sequences [off[i], off[i+1]),
+    // whose first group_prefix_pages[i] pages were attended by prefix_kernel
+    const int32_t* group_offsets;       // [num_groups + 1]
+    const int32_t* group_prefix_pages;  // [num_groups]
+    int32_t num_groups, max_group_size;
+    int32_t prefix_splits;              // key ranges of the prefix partials
+    const float* prefix_o;              // [splits][B][Hq][D]
+    const float2* prefix_ml;            // [splits][B][Hq] (max logit base 2, exp-sum)
 };
 
 // One segment of a CTA's share, handed from the producer to the consumers.
@@ -94,7 +103,8 @@ struct SegDesc {
     int32_t npg;       // pages in the segment; 0 marks the end of the share
     int32_t L;         // context length of b
     int32_t k0, k1;    // CTAs holding pages of (b, g); whole iff k0 == k1
-    int32_t pad[9];
+    int32_t P;         // shared-prefix pages of b (the line holds pages P .. ceil(L/bs)-1)
+    int32_t pad[8];
 };
 static_assert(sizeof(SegDesc) == 64, "descriptor size");
 
@@ -107,11 +117,6 @@ struct Split {
         return int32_t(pg < big ? pg / (per + 1) : rem + (pg - big) / per);
     }
 };
-
-// Byte offset of 16-byte chunk `ch` (0 .. D/8-1) of row t in a staged tile.
-__device__ __forceinline__ int tile_off(int t, int ch) {
-    return ((ch >> 3) << 11) + (t << 7) + (((ch & 7) ^ (t & 7)) << 4);
-}
 
 // Shared scalars.
 struct Misc {
@@ -268,6 +273,31 @@ struct SimtMath {
                     }
                 }
             }
+        }
+    }
+
+    // Folds a finished partial (normalised output o[G][D], (max logit base
+    // 2, exp-sum) per head) into the state, as if its tokens had been paged
+    // here.  The sums live in token group 0; every lane keeps the same m.
+    __device__ __forceinline__ void absorb(const float* o, const float2* ml, int lane) {
+        const int tg = lane >> 3, c = lane & 7;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float2 pml = __ldcg(ml + h);
+            if (!(pml.y > 0.f)) continue;
+            const float M = fmaxf(m[h], pml.x);
+            const float a_old = exp2f(m[h] - M), a_new = pml.y * exp2f(pml.x - M);
+            m[h] = M;
+            l[h] = l[h] * a_old + (tg == 0 ? a_new : 0.f);
+#pragma unroll
+            for (int i = 0; i < NCH; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float2 v = make_float2(0.f, 0.f);
+                    if (tg == 0) v = __ldcg(reinterpret_cast<const float2*>(o + h * D + (c + 8 * i) * 8 + 2 * j));
+                    acc[h][i][j] = make_float2(acc[h][i][j].x * a_old + a_new * v.x,
+                                               acc[h][i][j].y * a_old + a_new * v.y);
+                }
         }
     }
 
@@ -432,6 +462,29 @@ struct MmaMath {
         }
     }
 
+    // Folds a finished partial (normalised output o[G][D], (max logit base
+    // 2, exp-sum) per head) into the state, as if its tokens had been paged
+    // here.  l lives in row group 0 (finish() sums the row groups).
+    __device__ __forceinline__ void absorb(const float* o, const float2* ml, int lane) {
+        const int h0 = (lane & 3) * 2, d0 = lane >> 2;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int h = h0 + e;
+            if (h >= G) continue;
+            const float2 pml = __ldcg(ml + h);
+            if (!(pml.y > 0.f)) continue;
+            const float M = fmaxf(m[e], pml.x);
+            const float a_old = exp2f(m[e] - M), a_new = pml.y * exp2f(pml.x - M);
+            m[e] = M;
+            l[e] = l[e] * a_old + (d0 == 0 ? a_new : 0.f);
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+                acc[mt][e] = acc[mt][e] * a_old + a_new * __ldcg(o + h * D + 16 * mt + d0);
+                acc[mt][2 + e] = acc[mt][2 + e] * a_old + a_new * __ldcg(o + h * D + 16 * mt + d0 + 8);
+            }
+        }
+    }
+
     // Sum l over the 8 row groups (lanes with equal lane % 4).
     __device__ __forceinline__ void finish() {
 #pragma unroll
@@ -530,6 +583,37 @@ __device__ __forceinline__ int32_t clamp_len(const DecodeParams& p, int b, bool 
     return L;
 }
 
+// Sequence b's context: L tokens, of which the first P pages come from its
+// group's shared prefix (attended by prefix_kernel; 0 without groups) and
+// np = ceil(L / bs) - P pages are streamed here.  A member whose context
+// does not cover the prefix, or past max_group_size in its group, keeps all
+// its pages (prefix_kernel reports it).
+struct SeqPages {
+    int32_t L, P, np;
+};
+
+template <int BS>
+__device__ __forceinline__ SeqPages seq_pages(const DecodeParams& p, int b, bool report) {
+    SeqPages s;
+    s.L = clamp_len<BS>(p, b, report);
+    s.P = 0;
+    if (p.num_groups > 0) {
+        const int32_t* off = p.group_offsets;
+        if (b >= __ldg(off) && b < __ldg(off + p.num_groups)) {
+            int lo = 0, hi = p.num_groups;  // off[lo] <= b < off[hi]
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (__ldg(off + mid) <= b) lo = mid;
+                else hi = mid;
+            }
+            const int32_t P = __ldg(p.group_prefix_pages + lo);
+            if (P > 0 && int64_t(P) * BS <= s.L && b - __ldg(off + lo) < p.max_group_size) s.P = P;
+        }
+    }
+    s.np = (s.L + BS - 1) / BS - s.P;
+    return s;
+}
+
 template <int D, int G, int BS, int NW, int R, int PPS, bool DUMP, bool APPEND, template <int, int, int> class Math>
 __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
     // Stage i % R always feeds warp i % NW, so a warp waiting on a stage is at
@@ -609,10 +693,9 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
         const int b = base + threadIdx.x;
         long long v = 0;
         if (b < p.B) {
-            const int32_t L = clamp_len<BS>(p, b, blockIdx.x == 0);
-            const int npb = (L + BS - 1) / BS;
-            v = (long long)(npb > 0 ? npb + p.seg_weight : 0) * p.Hkv;
-            if (L == 0 && (b % int(gridDim.x)) == int(blockIdx.x)) {
+            const SeqPages sp = seq_pages<BS>(p, b, blockIdx.x == 0);
+            v = (long long)(sp.np > 0 ? sp.np + p.seg_weight : 0) * p.Hkv;
+            if (sp.L == 0 && (b % int(gridDim.x)) == int(blockIdx.x)) {
                 uint4* o = reinterpret_cast<uint4*>(p.out + int64_t(b) * p.Hq * D);
                 for (int i = 0; i < p.Hq * D / 8; ++i) o[i] = make_uint4(0, 0, 0, 0);
             }
@@ -645,6 +728,30 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
         fence_proxy_async_global();
         if (misc->abort) return;
     }
+    if (p.num_groups > 0) {
+        // Sequences whose whole context is their group's shared prefix take no
+        // units: their output is the merge of the prefix partials alone.
+        for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
+            const SeqPages sp = seq_pages<BS>(p, b, false);
+            if (sp.P == 0 || sp.np != 0) continue;
+            const int per = prefix_split_pages(sp.P, p.prefix_splits);
+            const int nz = (sp.P + per - 1) / per;
+            for (int o = threadIdx.x; o < p.Hq * D; o += NT) {
+                const int h = o / D;
+                float M = -INFINITY;
+                for (int z = 0; z < nz; ++z) M = fmaxf(M, __ldcg(&p.prefix_ml[(int64_t(z) * p.B + b) * p.Hq + h]).x);
+                float lsum = 0.f, a = 0.f;
+                for (int z = 0; z < nz; ++z) {
+                    const int64_t idx = (int64_t(z) * p.B + b) * p.Hq + h;
+                    const float2 ml = __ldcg(&p.prefix_ml[idx]);
+                    const float w = ml.y * exp2f(ml.x - M);
+                    lsum += w;
+                    a += w * __ldcg(&p.prefix_o[idx * D + (o - h * D)]);
+                }
+                p.out[int64_t(b) * p.Hq * D + o] = __float2bfloat16_rn(a / lsum);
+            }
+        }
+    }
     if (Wt == 0) return;
     const int64_t want = (Wt + p.min_pages - 1) / p.min_pages;
     const int64_t grid_eff = want < int64_t(gridDim.x) ? want : int64_t(gridDim.x);
@@ -669,7 +776,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
             const int b = base + threadIdx.x;
             long long v = 0;
             if (b < p.B) {
-                const int npb = (clamp_len<BS>(p, b, false) + BS - 1) / BS;
+                const int32_t npb = seq_pages<BS>(p, b, false).np;
                 v = (long long)(npb > 0 ? npb + p.seg_weight : 0) * p.Hkv;
             }
             long long chunk_total;
@@ -693,8 +800,8 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
 
         // walk the (b, g) whose units meet the share [p_start, p_end)
         int b = misc->b0;
-        int32_t Lb = clamp_len<BS>(p, b, false);
-        int32_t np = (Lb + BS - 1) / BS;
+        SeqPages sp = seq_pages<BS>(p, b, false);
+        int32_t Lb = sp.L, Pb = sp.P, np = sp.np;  // the line holds b's pages Pb .. Pb+np-1
         int64_t unit = np + p.seg_weight;
         int g = int((p_start - misc->pre0) / unit);
         int64_t u0 = misc->pre0 + int64_t(g) * unit;  // line position of (b, g)'s first page
@@ -702,7 +809,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
             const int64_t lo = p_start > u0 ? p_start : u0;
             const int64_t hi = p_end < u0 + np ? p_end : u0 + np;
             if (lo < hi) {
-                const int j = int(lo - u0);
+                const int j = Pb + int(lo - u0);  // first page of the segment in b's table
                 const int npg = int(hi - lo);
                 if (lane == 0) {
                     const int s = seg_i % S;
@@ -716,6 +823,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
                         d.L = Lb;
                         d.k0 = split.owner(u0);
                         d.k1 = split.owner(u0 + np - 1);
+                        d.P = Pb;
                         mbar_arrive_expect_tx(&segfull[s], Cfg::kQBytes);
                         bulk_g2s(qring + s * Cfg::kQBytes,
                                  p.q + (int64_t(b) * p.Hq + int64_t(g) * G) * Cfg::kRow, Cfg::kQBytes,
@@ -788,9 +896,11 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
                 g = 0;
                 do {
                     ++b;
-                    Lb = clamp_len<BS>(p, b, false);
-                    np = (Lb + BS - 1) / BS;
-                } while (np == 0);
+                    sp = seq_pages<BS>(p, b, false);
+                } while (sp.np == 0);
+                Lb = sp.L;
+                Pb = sp.P;
+                np = sp.np;
                 unit = np + p.seg_weight;
             }
         }
@@ -835,6 +945,16 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
         __syncwarp();
         if (lane == 0) mbar_arrive(&segempty[s]);
         st.reset();
+        if (d.P > 0 && d.j0 == d.P) {
+            // the piece that starts at b's first own page carries the shared
+            // prefix: its partials are folded in, one key range per warp
+            const int per = prefix_split_pages(d.P, p.prefix_splits);
+            const int nz = (d.P + per - 1) / per;
+            for (int z = warp; z < nz; z += NW) {
+                const int64_t idx = (int64_t(z) * p.B + d.b) * p.Hq + int64_t(d.g) * G;
+                st.absorb(p.prefix_o + idx * D, p.prefix_ml + idx, lane);
+            }
+        }
 
         const int nst = (d.npg + PPS - 1) / PPS;
         for (int k = int((uint32_t(warp) + NW - stage_base % NW) % NW); k < nst; k += NW) {

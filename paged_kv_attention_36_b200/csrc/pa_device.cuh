@@ -158,6 +158,13 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Byte offset of 16-byte chunk `ch` (0 .. D/8-1) of row t in a staged
+// (block, kv head) tile: D/64 panels of 16 rows x 128 bytes, written by TMA
+// with the 128-byte swizzle (chunk c of row t sits at position c ^ (t % 8)).
+__device__ __forceinline__ int tile_off(int t, int ch) {
+    return ((ch >> 3) << 11) + (t << 7) + (((ch & 7) ^ (t & 7)) << 4);
+}
+
 // ---- warp-level tensor-core fragments (mma.sync family) --------------------
 __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void* smem_row) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"

@@ -76,6 +76,20 @@ class Workload:
     v_new: torch.Tensor         # [B][Hkv][D] bf16
     slot_mapping: torch.Tensor  # [B] int32: slot of position context_len - 1
     scale: float
+    # shared prefixes: group i = sequences [group_offsets[i], group_offsets[i+1])
+    # whose tables begin with the same group_prefix_pages[i] blocks
+    group_offsets: torch.Tensor = None       # [num_groups + 1] int32
+    group_prefix_pages: torch.Tensor = None  # [num_groups] int32
+
+    @property
+    def num_groups(self) -> int:
+        return 0 if self.group_prefix_pages is None else int(self.group_prefix_pages.shape[0])
+
+    @property
+    def max_group_size(self) -> int:
+        if self.num_groups == 0:
+            return 0
+        return int((self.group_offsets[1:] - self.group_offsets[:-1]).max().item())
 
     @property
     def dims(self):
@@ -181,6 +195,20 @@ def make(name: str, *, poison: bool = False, seed: int | None = None,
             lists.append(perm[cursor:cursor + n])
             cursor += n
     block_tables = build_tables(lists, M)
+    w = _fill(spec, g, lens, lists, block_tables, NB, poison)
+    if name == "prefix" and context_lens is None:
+        w.group_offsets = torch.tensor([0, B // 2, B], dtype=torch.int32)
+        w.group_prefix_pages = torch.tensor([shared_prefix_blocks] * 2, dtype=torch.int32)
+    return w
+
+
+def _fill(spec: WorkloadSpec, g: torch.Generator, lens: torch.Tensor, lists, block_tables: torch.Tensor,
+          NB: int, poison: bool, num_seqs: int | None = None) -> Workload:
+    """Draws q, the caches and the appended rows for a batch whose tables are
+    built, poisons unread rows if asked, and derives the slot mapping."""
+    B = lens.shape[0]
+    Hq, Hkv, D, bs = spec.num_q_heads, spec.num_kv_heads, spec.head_dim, spec.block_size
+    name = spec.name
 
     # ---- values ----------------------------------------------------------
     q = _randn_bf16(g, (B, Hq, D))
@@ -245,3 +273,52 @@ def append_bytes(w: Workload) -> int:
     n_valid = int((w.slot_mapping >= 0).sum().item())
     per_tok = w.k_new.shape[1] * w.k_new.shape[2] * 2 * 2
     return 2 * n_valid * per_tok + 4 * w.slot_mapping.numel()
+
+
+def make_grouped(name: str, groups, suffix_lens, *, tail_lens=(), seed: int | None = None,
+                 poison: bool = False, heads=None) -> Workload:
+    """A batch with the head shapes of configuration ``name`` in which runs of
+    consecutive sequences share their first blocks, as prefix caching
+    leaves them.  ``groups`` = [(members, prefix_pages), ...]; member b of
+    the groups has context prefix_pages * bs + suffix_lens[b] (0 makes the
+    whole context the shared prefix); then one sequence in no group per
+    entry of ``tail_lens``.  Block ids are a seeded permutation of a pool
+    that holds exactly the needed blocks.  ``heads`` = (Hq, Hkv, D)
+    overrides the configuration's head shapes."""
+    spec = SPECS[name]
+    if heads is not None:
+        spec = dataclasses.replace(spec, num_q_heads=heads[0], num_kv_heads=heads[1], head_dim=heads[2])
+    g = torch.Generator().manual_seed(spec.seed + 1000 if seed is None else seed)
+    bs = spec.block_size
+    n_members = sum(m for m, _ in groups)
+    if len(suffix_lens) != n_members:
+        raise ValueError("one suffix length per group member")
+    lens, prefix_of = [], []
+    for gi, (m, P) in enumerate(groups):
+        for _ in range(m):
+            prefix_of.append(gi)
+    for b, sfx in enumerate(suffix_lens):
+        lens.append(groups[prefix_of[b]][1] * bs + int(sfx))
+    lens += [int(L) for L in tail_lens]
+    lens_t = torch.tensor(lens, dtype=torch.int64)
+    pages = _pages(lens_t, bs)
+    private = [int(pages[b]) - (groups[prefix_of[b]][1] if b < n_members else 0) for b in range(len(lens))]
+    NB = max(1, sum(P for _, P in groups) + sum(private))
+    perm = torch.randperm(NB, generator=g).tolist()
+    cursor, prefix_ids = 0, []
+    for _, P in groups:
+        prefix_ids.append(perm[cursor:cursor + P])
+        cursor += P
+    lists = []
+    for b in range(len(lens)):
+        shared = prefix_ids[prefix_of[b]] if b < n_members else []
+        lists.append(shared + perm[cursor:cursor + private[b]])
+        cursor += private[b]
+    M = max(1, int(pages.max().item()) if len(lens) else 1)
+    w = _fill(spec, g, lens_t, lists, build_tables(lists, M), NB, poison)
+    offsets = [0]
+    for m, _ in groups:
+        offsets.append(offsets[-1] + m)
+    w.group_offsets = torch.tensor(offsets, dtype=torch.int32)
+    w.group_prefix_pages = torch.tensor([P for _, P in groups], dtype=torch.int32)
+    return w
