@@ -14,7 +14,10 @@ CUDA events on the launching stream.  L2: each step reads one of several
 copies of the paged cache, rotated so that a copy is untouched by at least
 400 MB of other traffic before it is read again (inputs larger than the
 126 MB L2); batches too small for that flush L2 with a 256 MB write between
-steps, outside the timed events.  With N > 1 (torchrun) every rank runs an
+steps, outside the timed events.  A batch whose sequences share prefix
+blocks (the prefix-shared workload) runs the shared-prefix path: one prefix
+attention launch per step before the fused append + decode; the same steps
+on the plain path are timed beside it.  With N > 1 (torchrun) every rank runs an
 independent replica of the batch (the path has no exchange step); value =
 bytes of all ranks / the slowest rank's time.
 """
@@ -258,13 +261,29 @@ def run_pa(args, ws, rank, local):
     caches = [(w.k_cache.to(dev), w.v_cache.to(dev)) for _ in range(ncopies)]
     out = torch.empty_like(q)
     dims = pa.make_dims(q, caches[0][0], bt)
-    wsp = pa.alloc_workspace(dims, device=dev)
+    grouped = w.num_groups > 0
+    if grouped:
+        go, gp, mgs = w.group_offsets.to(dev), w.group_prefix_pages.to(dev), w.max_group_size
+        wsp = torch.zeros(pa.pa_decode_shared_prefix_workspace_bytes(dims, w.num_groups, mgs),
+                          dtype=torch.uint8, device=dev)
+    else:
+        wsp = pa.alloc_workspace(dims, device=dev)
     flush = None if rotate else torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     app = [pa.prepare_append(kn, vn, sm, kc, vc, stream=stream) for kc, vc in caches]
-    dec = [pa.prepare_decode(q, kc, vc, bt, cl, w.scale, out, wsp, stream=stream) for kc, vc in caches]
-    fused = [pa.prepare_append_decode(kn, vn, sm, q, kc, vc, bt, cl, w.scale, out, wsp, stream=stream)
+    plain = [pa.prepare_append_decode(kn, vn, sm, q, kc, vc, bt, cl, w.scale, out, wsp, stream=stream)
              for kc, vc in caches]
+    if grouped:
+        # one prefix-attention launch, then the fused append + decode of the members' own pages
+        fused = [pa.prepare_decode_shared_prefix(q, kc, vc, bt, cl, w.scale, go, gp, mgs, out, wsp, k_new=kn,
+                                                 v_new=vn, slot_mapping=sm, stream=stream) for kc, vc in caches]
+        dec = [pa.prepare_decode_shared_prefix(q, kc, vc, bt, cl, w.scale, go, gp, mgs, out, wsp, stream=stream)
+               for kc, vc in caches]
+        launches = 2
+    else:
+        fused = plain
+        dec = [pa.prepare_decode(q, kc, vc, bt, cl, w.scale, out, wsp, stream=stream) for kc, vc in caches]
+        launches = 1
 
     def between():
         if flush is not None:
@@ -314,13 +333,34 @@ def run_pa(args, ws, rank, local):
     app_avg = _max_over_ranks(sum(ev2[k][0].elapsed_time(ev2[k][1]) for k in range(K)) / K, ws)
     dec_avg = _max_over_ranks(sum(ev2[k][1].elapsed_time(ev2[k][2]) for k in range(K)) / K, ws)
 
+    plain_avg = None
+    if grouped:
+        # ---- the same steps on the plain path (every member streams the shared pages) ----
+        for k in range(W_):
+            plain[k % ncopies]()
+            between()
+        ev3 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+        torch.cuda.synchronize(dev)
+        for k in range(K):
+            ev3[k][0].record(stream)
+            plain[k % ncopies]()
+            ev3[k][1].record(stream)
+            between()
+        torch.cuda.synchronize(dev)
+        plain_avg = _max_over_ranks(sum(ev3[k][0].elapsed_time(ev3[k][1]) for k in range(K)) / K, ws)
+
     # ---- end to end through the public API from pinned host buffers ----
-    host = {n: t.pin_memory() for n, t in (("q", w.q), ("bt", w.block_tables), ("cl", w.context_lens),
-                                            ("kn", w.k_new), ("vn", w.v_new), ("sm", w.slot_mapping))}
+    host_src = [("q", w.q), ("bt", w.block_tables), ("cl", w.context_lens), ("kn", w.k_new), ("vn", w.v_new),
+                ("sm", w.slot_mapping)]
+    if grouped:
+        host_src += [("go", w.group_offsets), ("gp", w.group_prefix_pages)]
+    host = {n: t.pin_memory() for n, t in host_src}
     out_h = torch.empty(w.q.shape, dtype=torch.bfloat16).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_h.numel() * out_h.element_size()
     dev_in = {"q": q, "bt": bt, "cl": cl, "kn": kn, "vn": vn, "sm": sm}
+    if grouped:
+        dev_in.update(go=go, gp=gp)
 
     def e2e_step(c):
         for n, t in host.items():
@@ -349,7 +389,7 @@ def run_pa(args, ws, rank, local):
         return
     peak, peak_kind = _peaks()
     step_avg = total_ms / K
-    achieved = step_bytes / (step_avg * 1e-3) / 1e9   # the fused kernel is the step
+    achieved = step_bytes / (step_avg * 1e-3) / 1e9   # the fused kernel is the step (+ the prefix launch)
     value = ws * K * step_bytes / (total_ms * 1e-3) / 1e9
     l2 = (f"inputs larger than L2: {ncopies} copies of the {pool_bytes / 1e6:.0f} MB paged cache rotated, "
           f"no flush" if rotate else "flushed between steps (256 MB write, outside the timed events)")
@@ -381,15 +421,19 @@ def run_pa(args, ws, rank, local):
         "step_pct_of_8tbs_nominal": round(100 * achieved / 8000.0, 1),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                     "kernel": "pa::decode_kernel<..., APPEND> (pa_append_decode)",
+                     "kernel": ("pa::prefix_kernel + pa::decode_kernel<..., APPEND> (pa_decode_shared_prefix)"
+                                if grouped else "pa::decode_kernel<..., APPEND> (pa_append_decode)"),
                      "traffic": _traffic(args.workload),
                      "algorithmic_bytes_per_launch": step_bytes},
         "e2e": {"value": round(ws * K * step_bytes / (e2e_total * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_total / K, 5)},
-        "gpu_launches": K,
+        "gpu_launches": launches * K,
         "clocks": clk,
     }
+    if grouped:
+        line["config"]["shared_prefix_groups"] = w.num_groups
+        line["plain_path_step_us"] = round(plain_avg * 1e3, 2)
     if ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, dec_bytes, app_bytes)
     print(json.dumps(line), flush=True)

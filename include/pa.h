@@ -229,10 +229,13 @@ PA_API pa_status pa_decode_static_ws(const void* q, const void* k_cache, const v
  *     for offsets out of order or range, P_i > M, and a member whose table
  *     does not begin with the group's first member's P_i block ids (the
  *     output of such members is unspecified).
- *   - num_tokens > 0 also appends k_new/v_new at slot_mapping first, fused
- *     into the decode launch as in pa_append_decode; slots must not fall in
- *     the shared blocks (the prefix pass runs before the append).
+ *   - num_tokens > 0 also appends k_new/v_new at slot_mapping first (as
+ *     pa_cache_append), inside the prefix pass's launch (or, with no groups,
+ *     fused into the decode as in pa_append_decode); slots must not fall in
+ *     the shared blocks, which the prefix pass reads meanwhile.
  *     num_tokens = 0 skips the append (k_new, v_new, slot_mapping unused).
+ *   - Two launches: the prefix pass, then the decode as its programmatic
+ *     dependent, so that the decode's set-up overlaps the pass's end.
  *   - Supported shapes and alignment as for pa_decode.  The workspace must
  *     be at least pa_decode_shared_prefix_workspace_bytes(dims, num_groups,
  *     max_group_size) bytes, zero-filled before its first use, and is left

@@ -187,8 +187,10 @@ bool make_cache_map(CUtensorMap* map, const void* base, int64_t rows, int D, int
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// pdl: launched as a programmatic dependent of the kernel before it in the
+// stream (prefix_kernel), so that its set-up overlaps that kernel's end.
 template <MathKind MK, int D, int G, bool DUMP, bool APPEND>
-pa_status launch_decode(const pa::DecodeParams& p, int grid, cudaStream_t stream) {
+pa_status launch_decode(const pa::DecodeParams& p, int grid, cudaStream_t stream, bool pdl) {
     constexpr int NW = Tune<MK, D, G>::NW, R = Tune<MK, D, G>::R, PPS = Tune<MK, D, G>::PPS;
     using Cfg = pa::DecodeCfg<D, G, kBlockSize, NW, R, PPS>;
     auto kern = [] {
@@ -212,6 +214,18 @@ pa_status launch_decode(const pa::DecodeParams& p, int grid, cudaStream_t stream
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return PA_ERR_CUDA;
+    } else if (pdl) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(Cfg::kThreads);
+        cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return PA_ERR_CUDA;
     } else {
         kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(p);
     }
@@ -219,21 +233,21 @@ pa_status launch_decode(const pa::DecodeParams& p, int grid, cudaStream_t stream
 }
 
 template <MathKind MK, bool DUMP, bool APPEND>
-pa_status dispatch_d_g(int D, int G, const pa::DecodeParams& p, int grid, cudaStream_t s) {
+pa_status dispatch_d_g(int D, int G, const pa::DecodeParams& p, int grid, cudaStream_t s, bool pdl) {
     if (D == 64) {
         switch (G) {
-            case 1: return launch_decode<MK, 64, 1, DUMP, APPEND>(p, grid, s);
-            case 2: return launch_decode<MK, 64, 2, DUMP, APPEND>(p, grid, s);
-            case 4: return launch_decode<MK, 64, 4, DUMP, APPEND>(p, grid, s);
-            case 8: return launch_decode<MK, 64, 8, DUMP, APPEND>(p, grid, s);
+            case 1: return launch_decode<MK, 64, 1, DUMP, APPEND>(p, grid, s, pdl);
+            case 2: return launch_decode<MK, 64, 2, DUMP, APPEND>(p, grid, s, pdl);
+            case 4: return launch_decode<MK, 64, 4, DUMP, APPEND>(p, grid, s, pdl);
+            case 8: return launch_decode<MK, 64, 8, DUMP, APPEND>(p, grid, s, pdl);
         }
     } else if (D == 128) {
         switch (G) {
-            case 1: return launch_decode<MK, 128, 1, DUMP, APPEND>(p, grid, s);
-            case 2: return launch_decode<MK, 128, 2, DUMP, APPEND>(p, grid, s);
-            case 4: return launch_decode<MK, 128, 4, DUMP, APPEND>(p, grid, s);
+            case 1: return launch_decode<MK, 128, 1, DUMP, APPEND>(p, grid, s, pdl);
+            case 2: return launch_decode<MK, 128, 2, DUMP, APPEND>(p, grid, s, pdl);
+            case 4: return launch_decode<MK, 128, 4, DUMP, APPEND>(p, grid, s, pdl);
             case 8:
-                if constexpr (MK == MathKind::kMma) return launch_decode<MK, 128, 8, DUMP, APPEND>(p, grid, s);
+                if constexpr (MK == MathKind::kMma) return launch_decode<MK, 128, 8, DUMP, APPEND>(p, grid, s, pdl);
                 break;
         }
     }
@@ -241,9 +255,9 @@ pa_status dispatch_d_g(int D, int G, const pa::DecodeParams& p, int grid, cudaSt
 }
 
 template <bool DUMP, bool APPEND = false>
-pa_status dispatch_decode(int D, int G, const pa::DecodeParams& p, int grid, cudaStream_t s) {
-    return math_kind() == MathKind::kMma ? dispatch_d_g<MathKind::kMma, DUMP, APPEND>(D, G, p, grid, s)
-                                         : dispatch_d_g<MathKind::kSimt, DUMP, APPEND>(D, G, p, grid, s);
+pa_status dispatch_decode(int D, int G, const pa::DecodeParams& p, int grid, cudaStream_t s, bool pdl = false) {
+    return math_kind() == MathKind::kMma ? dispatch_d_g<MathKind::kMma, DUMP, APPEND>(D, G, p, grid, s, pdl)
+                                         : dispatch_d_g<MathKind::kSimt, DUMP, APPEND>(D, G, p, grid, s, pdl);
 }
 
 // ---- shared-prefix pass ----------------------------------------------------
@@ -558,6 +572,13 @@ pa_status pa_decode_shared_prefix(const void* k_new, const void* v_new, const in
         pp.qscale = p.qscale;
         pp.prefix_o = reinterpret_cast<float*>(ws + w.o);
         pp.prefix_ml = reinterpret_cast<float2*>(ws + w.ml);
+        // the append rides on the prefix launch; the decode follows it
+        pp.k_new = static_cast<const uint4*>(k_new);
+        pp.v_new = static_cast<const uint4*>(v_new);
+        pp.slot_mapping = slot_mapping;
+        pp.app_chunks = int64_t(num_tokens) * d.num_kv_heads * (d.head_dim / 8);
+        pp.k_cache_w = static_cast<uint4*>(k_cache);
+        pp.v_cache_w = static_cast<uint4*>(v_cache);
         const pa_status ps = dispatch_prefix(d.head_dim, G, pp, dim3(unsigned(num_groups * tiles),
                                                                      unsigned(d.num_kv_heads), unsigned(splits)), s);
         if (ps != PA_OK) return ps;
@@ -568,6 +589,7 @@ pa_status pa_decode_shared_prefix(const void* k_new, const void* v_new, const in
         p.prefix_splits = splits;
         p.prefix_o = pp.prefix_o;
         p.prefix_ml = pp.prefix_ml;
+        return dispatch_decode<false>(d.head_dim, G, p, grid, s, /*pdl=*/true);
     }
     if (num_tokens == 0) return dispatch_decode<false>(d.head_dim, G, p, grid, s);
     p.k_new = static_cast<const uint4*>(k_new);

@@ -276,6 +276,17 @@ struct SimtMath {
         }
     }
 
+    // A finished partial to fold into the state (SIMT: read when folded).
+    struct Piece {
+        const float* o;
+        const float2* ml;
+    };
+    __device__ __forceinline__ void piece_load(Piece& pc, const float* o, const float2* ml, int) const {
+        pc.o = o;
+        pc.ml = ml;
+    }
+    __device__ __forceinline__ void piece_absorb(const Piece& pc, int lane) { absorb(pc.o, pc.ml, lane); }
+
     // Folds a finished partial (normalised output o[G][D], (max logit base
     // 2, exp-sum) per head) into the state, as if its tokens had been paged
     // here.  The sums live in token group 0; every lane keeps the same m.
@@ -284,7 +295,6 @@ struct SimtMath {
 #pragma unroll
         for (int h = 0; h < G; ++h) {
             const float2 pml = __ldcg(ml + h);
-            if (!(pml.y > 0.f)) continue;
             const float M = fmaxf(m[h], pml.x);
             const float a_old = exp2f(m[h] - M), a_new = pml.y * exp2f(pml.x - M);
             m[h] = M;
@@ -462,27 +472,48 @@ struct MmaMath {
         }
     }
 
-    // Folds a finished partial (normalised output o[G][D], (max logit base
-    // 2, exp-sum) per head) into the state, as if its tokens had been paged
-    // here.  l lives in row group 0 (finish() sums the row groups).
-    __device__ __forceinline__ void absorb(const float* o, const float2* ml, int lane) {
+    // A finished partial (normalised output o[G][D], (max logit base 2,
+    // exp-sum) per head) held in this lane's accumulator layout, so that it
+    // can be loaded when a segment starts and folded in after its pages.
+    struct Piece {
+        float o[KS][4];
+        float2 ml[2];
+    };
+    __device__ __forceinline__ void piece_load(Piece& pc, const float* o, const float2* ml, int lane) const {
         const int h0 = (lane & 3) * 2, d0 = lane >> 2;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            const int h = h0 + e;
-            if (h >= G) continue;
-            const float2 pml = __ldcg(ml + h);
-            if (!(pml.y > 0.f)) continue;
-            const float M = fmaxf(m[e], pml.x);
-            const float a_old = exp2f(m[e] - M), a_new = pml.y * exp2f(pml.x - M);
+            const int h = h0 + e < G ? h0 + e : 0;  // heads past G: loaded, never folded
+            pc.ml[e] = __ldcg(ml + h);
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+                pc.o[mt][e] = __ldcg(o + h * D + 16 * mt + d0);
+                pc.o[mt][2 + e] = __ldcg(o + h * D + 16 * mt + d0 + 8);
+            }
+        }
+    }
+    // Folds the piece into the state, as if its tokens had been paged here;
+    // l lives in row group 0 (finish() sums the row groups).
+    __device__ __forceinline__ void piece_absorb(const Piece& pc, int lane) {
+        const int h0 = (lane & 3) * 2, d0 = lane >> 2;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            if (h0 + e >= G) continue;
+            const float M = fmaxf(m[e], pc.ml[e].x);
+            const float a_old = exp2f(m[e] - M), a_new = pc.ml[e].y * exp2f(pc.ml[e].x - M);
             m[e] = M;
             l[e] = l[e] * a_old + (d0 == 0 ? a_new : 0.f);
 #pragma unroll
             for (int mt = 0; mt < KS; ++mt) {
-                acc[mt][e] = acc[mt][e] * a_old + a_new * __ldcg(o + h * D + 16 * mt + d0);
-                acc[mt][2 + e] = acc[mt][2 + e] * a_old + a_new * __ldcg(o + h * D + 16 * mt + d0 + 8);
+                acc[mt][e] = acc[mt][e] * a_old + a_new * pc.o[mt][e];
+                acc[mt][2 + e] = acc[mt][2 + e] * a_old + a_new * pc.o[mt][2 + e];
             }
         }
+    }
+    __device__ __forceinline__ void absorb(const float* o, const float2* ml, int lane) {
+        Piece pc;
+        piece_load(pc, o, ml, lane);
+        piece_absorb(pc, lane);
     }
 
     // Sum l over the 8 row groups (lanes with equal lane % 4).
@@ -728,6 +759,11 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
         fence_proxy_async_global();
         if (misc->abort) return;
     }
+    // A decode launched right after prefix_kernel (programmatic dependent
+    // launch) has done the set-up above meanwhile; the prefix partials and
+    // the rows that kernel appended are read only after this wait (a no-op
+    // for an ordinary launch).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (p.num_groups > 0) {
         // Sequences whose whole context is their group's shared prefix take no
         // units: their output is the merge of the prefix partials alone.
@@ -945,15 +981,17 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
         __syncwarp();
         if (lane == 0) mbar_arrive(&segempty[s]);
         st.reset();
-        if (d.P > 0 && d.j0 == d.P) {
-            // the piece that starts at b's first own page carries the shared
-            // prefix: its partials are folded in, one key range per warp
-            const int per = prefix_split_pages(d.P, p.prefix_splits);
-            const int nz = (d.P + per - 1) / per;
-            for (int z = warp; z < nz; z += NW) {
-                const int64_t idx = (int64_t(z) * p.B + d.b) * p.Hq + int64_t(d.g) * G;
-                st.absorb(p.prefix_o + idx * D, p.prefix_ml + idx, lane);
-            }
+        // The piece that starts at b's first own page carries the shared
+        // prefix: warp z loads the partial of prefix key range z now and
+        // folds it in after its pages (the loads overlap the pages).
+        const int nz = (d.P > 0 && d.j0 == d.P)
+                           ? (d.P + prefix_split_pages(d.P, p.prefix_splits) - 1) /
+                                 prefix_split_pages(d.P, p.prefix_splits)
+                           : 0;
+        typename Math<D, G, BS>::Piece piece;
+        if (warp < nz) {
+            const int64_t idx = (int64_t(warp) * p.B + d.b) * p.Hq + int64_t(d.g) * G;
+            st.piece_load(piece, p.prefix_o + idx * D, p.prefix_ml + idx, lane);
         }
 
         const int nst = (d.npg + PPS - 1) / PPS;
@@ -988,6 +1026,13 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
             if (lane == 0) mbar_arrive(&empty[slot]);
         }
         stage_base += nst;
+        if (warp < nz) {
+            st.piece_absorb(piece, lane);
+            for (int z = warp + NW; z < nz; z += NW) {  // more key ranges than warps
+                const int64_t idx = (int64_t(z) * p.B + d.b) * p.Hq + int64_t(d.g) * G;
+                st.absorb(p.prefix_o + idx * D, p.prefix_ml + idx, lane);
+            }
+        }
 
         // ---- segment end: combine the NW warp states ----
         st.finish();

@@ -44,6 +44,14 @@ struct PrefixParams {
     float qscale;                       // scale * log2(e)
     float* prefix_o;                    // [splits][B][Hq][D] partial outputs
     float2* prefix_ml;                  // [splits][B][Hq] (max logit base 2, exp-sum)
+    // the step's slot-mapped append, done here (app_chunks = 0: none); the
+    // decode that follows reads the new rows
+    const uint4* k_new;                 // [T][Hkv][D] bf16 as 16-byte chunks
+    const uint4* v_new;
+    const int32_t* slot_mapping;        // [T]
+    int64_t app_chunks;                 // T * Hkv * D / 8
+    uint4* k_cache_w;
+    uint4* v_cache_w;
 };
 
 template <int D, int NW, int RS>
@@ -78,6 +86,36 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) prefix_kernel(const __grid_c
     volatile int* abort = &s_abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = blockIdx.y;
+
+    // The decode launched after this kernel may start its set-up now; it
+    // waits for this grid to complete before it reads anything written here.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    if (p.app_chunks > 0) {
+        // this CTA's slice of the append (a bit copy of 16-byte chunks; the
+        // rows land in the members' own blocks, never in the shared ones)
+        const int64_t ncta = int64_t(gridDim.x) * gridDim.y * gridDim.z;
+        const int64_t lin = (int64_t(blockIdx.z) * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+        const int64_t per = (p.app_chunks + ncta - 1) / ncta;
+        const int64_t c0 = lin * per;
+        const int64_t c1 = c0 + per < p.app_chunks ? c0 + per : p.app_chunks;
+        constexpr int CPR = D / 8;  // 16-byte chunks per row
+        for (int64_t idx = c0 + threadIdx.x; idx < c1; idx += Cfg::kThreads) {
+            const int64_t t = idx / (int64_t(p.Hkv) * CPR);
+            const int64_t rem = idx - t * p.Hkv * CPR;
+            const int32_t slot = __ldg(p.slot_mapping + t);
+            if (slot < 0) continue;
+            const int64_t block = slot / 16, offset = slot - (slot / 16) * 16;
+            if (block >= p.NB) {
+                if (rem == 0) raise_error(PA_DEVERR_SLOT);
+                continue;
+            }
+            const int64_t gg = rem / CPR, c = rem - gg * CPR;
+            const int64_t dst = ((block * p.Hkv + gg) * 16 + offset) * CPR + c;
+            p.k_cache_w[dst] = __ldg(p.k_new + idx);
+            p.v_cache_w[dst] = __ldg(p.v_new + idx);
+        }
+    }
 
     // ---- the group, its members and this CTA's rows and pages ----
     const int gi = int(blockIdx.x) / p.tiles_per_group;
