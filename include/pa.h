@@ -105,11 +105,12 @@ PA_API pa_status pa_cache_append(const void* k_new, const void* v_new, const int
 /*
  * Device workspace pa_decode needs, in bytes, when it runs on `num_ctas`
  * CTAs (0 = the default grid pa_decode picks on the current device).  The
- * workspace holds split-KV partial outputs and one merge counter per
- * (sequence, kv head).  It must be zero-filled once before its first use;
- * every completed call leaves it ready for the next (the counters return
- * to zero).  Calls that share one workspace must not overlap on the GPU.
- * Returns 0 for invalid dims.
+ * workspace holds split-KV partial outputs (two slots per CTA), one merge
+ * counter per (sequence, kv head) and the counters of the merge's first
+ * level.  It must be zero-filled once before its first use; every completed
+ * call leaves it ready for the next (the counters return to zero).  Calls
+ * that share one workspace must not overlap on the GPU.  Returns 0 for
+ * invalid dims.
  */
 PA_API size_t pa_decode_workspace_bytes(const pa_dims* dims, int32_t num_ctas);
 
@@ -118,16 +119,18 @@ PA_API int32_t pa_decode_default_ctas(void);
 
 /*
  * Paged decode attention (formula at the top of this file).  One persistent
- * CTA per SM walks an equal share of all (sequence, kv head, page) work;
- * all GQA query heads of a kv head share each staged K/V page.  A sequence
- * whose pages are shared between CTAs is finished by split-KV partials
- * (flash-decoding) and a log-sum-exp merge done by the last CTA to finish
- * its part.  Supported: block_size 16, head_dim 64 or 128, Hq/Hkv in
- * {1, 2, 4, 8}; fewer than 2^31 cache rows (NB*Hkv*bs).  q, k_cache,
- * v_cache and out must be 16-byte aligned.  The per-page math runs on the
- * tensor cores (mma.sync, fp32 accumulation); setting the environment
- * variable PA_DECODE_MATH=simt before the first call selects the fp32 CUDA
- * core variant instead (head_dim*Hq/Hkv <= 512 only).
+ * CTA per SM walks an equal share of all (sequence, kv-head group, page)
+ * work; a staged page holds one block's K and V tiles of up to 8 kv heads,
+ * one warp per kv head, and all GQA query heads of a kv head share its
+ * tiles.  A sequence whose pages are shared between CTAs is finished by
+ * split-KV partials (flash-decoding) and a log-sum-exp merge done by the
+ * last CTA to finish its part (in two levels beyond 16 parts).  Supported:
+ * block_size 16, head_dim 64 or 128, Hq/Hkv in {1, 2, 4, 8}; fewer than
+ * 2^31 cache rows (NB*Hkv*bs).  q, k_cache, v_cache and out must be 16-byte
+ * aligned.  The per-page math runs on the tensor cores (mma.sync, fp32
+ * accumulation); setting the environment variable PA_DECODE_MATH=simt
+ * before the first call selects the fp32 CUDA core variant instead
+ * (head_dim*Hq/Hkv <= 256 only).
  */
 PA_API pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
                     const int32_t* block_tables, const int32_t* context_lens, float scale,
@@ -154,8 +157,8 @@ PA_API pa_status pa_append_decode(const void* k_new, const void* v_new, const in
                                   void* stream);
 
 /*
- * Test hook: pa_decode on exactly `num_ctas` CTAs (which decides where
- * contexts are split), that also records every per-CTA segment it computes:
+ * Test hook: pa_decode on exactly `num_ctas` CTAs (1 .. 1024; it decides
+ * where contexts are split), that also records every per-CTA segment it computes:
  * segment i covers tokens [t0, t1) of kv head g of sequence b and stores
  *     seg_meta[i] = {b, g, t0, t1}                       int32[capacity][4]
  *     seg_o[i][j][:]  normalised partial output          f32[capacity][G][D]

@@ -17,70 +17,58 @@
 namespace {
 
 constexpr int kBlockSize = 16;  // tokens per physical block the decode kernels are built for
-constexpr int kMinPagesPerCta = 8;
+constexpr int kMinPagesPerCta = 2;  // pages of a head group: fewest worth a CTA
 constexpr int kMaxDevices = 64;
+constexpr int kMaxCtas = 1024;  // the two-level split merge handles up to 16 x 64 pieces
 constexpr float kLog2e = 1.4426950408889634f;
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
-// Per-shape tuning of the two math policies.
-//  SIMT: registers are split between the SM's four sub-partitions, so a CTA
-//    of 12 warps (11 consumers + the producer) caps a thread at 168
-//    registers and one of 8 warps at 255; G*D = 512 needs the latter.
-//  MMA: the per-lane state is small (2*D/16 fragment registers), 8
-//    consumer warps.
-// The ring depth R is a multiple of the consumer warps (each stage always
-// feeds the same warp) and holds 110-170 KB of K+V pages.
+// The math policies: tensor-core (default) or fp32 CUDA-core.
 enum class MathKind { kMma, kSimt };
 
-template <MathKind MK, int D, int G>
-struct Tune;
-
-#ifndef PA_MMA_NW
-#define PA_MMA_NW 8
-#endif
 #ifndef PA_MAX_RING
 #define PA_MAX_RING 64
 #endif
-#ifndef PA_MMA_STAGE_BYTES
-#define PA_MMA_STAGE_BYTES 8192  // pages per ring stage = this / (K+V bytes of a page)
-#endif
-// Deepest ring (a multiple of NW, at most PA_MAX_RING) whose CTA fits in shared memory.
-template <int D, int G, int NW, int PPS>
+// Deepest ring of stages whose CTA fits in shared memory, a multiple of
+// the most stages a page can take (with 32 KB stages: 7 at head_dim 64,
+// 6 at 128).
+template <int D>
 constexpr int ring_fit() {
-    int r = (PA_MAX_RING / NW) * NW;
-    while (r > NW && pa::DecodeCfg<D, G, kBlockSize, NW, 1, PPS>::kSmemBytes +
-                             (r - 1) * (PPS * 2 * kBlockSize * D * 2 + 16) > 232448)
-        r -= NW;
+    using C1 = pa::DecodeCfg<D, kBlockSize, 1>;
+    int r = PA_MAX_RING;
+    while (r > 1 && C1::kSmemBytes + (r - 1) * (C1::kStage + 16) > 232448) --r;
+    r -= r % C1::kMaxSpl;
     return r;
 }
-template <int D, int G>
-struct Tune<MathKind::kMma, D, G> {
-    static constexpr int NW = PA_MMA_NW;
-    static constexpr int PPS = (PA_MMA_STAGE_BYTES / (2 * kBlockSize * D * 2)) > 0
-                                   ? PA_MMA_STAGE_BYTES / (2 * kBlockSize * D * 2) : 1;
-    static constexpr int R = ring_fit<D, G, NW, PPS>();
-};
-
-template <int D, int G>
-struct Tune<MathKind::kSimt, D, G> {
-    static constexpr int NW = (G * D >= 512) ? 7 : 11;  // 8 warps: 255 registers each; 12: 168
-    static constexpr int PPS = 1;
-    static constexpr int R = ring_fit<D, G, NW, PPS>();
-};
 
 // Fixed cost of finishing a segment, expressed as K+V bytes that could be
-// streamed meanwhile (measured: ~1.5 us of a CTA's time per segment end);
+// streamed meanwhile, in pages of `heads` kv heads (rounded down);
 // PA_SEG_WEIGHT_BYTES overrides it.
-int32_t seg_weight_pages(int head_dim) {
+int32_t seg_weight_pages(int head_dim, int heads) {
     static const long long bytes = [] {
         const char* e = std::getenv("PA_SEG_WEIGHT_BYTES");
-        return e ? std::atoll(e) : 65536LL;
+        return e ? std::atoll(e) : 32768LL;
     }();
-    const long long page = 2LL * kBlockSize * head_dim * 2;
+    const long long page = 2LL * kBlockSize * head_dim * 2 * heads;
     return int32_t(bytes / page);
+}
+
+// kv heads per ring stage: as many whole K+V tiles as a stage holds.
+int heads_per_stage_max(int D) { return PA_STAGE_K_BYTES / (kBlockSize * D * 2); }
+
+// kv heads per head group: the largest divisor of Hkv that is at most 8
+// (one consumer warp per head) and splits into 1, 2, 4 or 8 equal stages.
+int heads_per_group(int Hkv, int D) {
+    const int hs = heads_per_stage_max(D);
+    for (int h = pa::kDecodeWarps; h > 1; --h) {
+        if (Hkv % h) continue;
+        for (int spl = 1; spl <= pa::kDecodeWarps; spl *= 2)
+            if (h % spl == 0 && h / spl <= hs) return h;
+    }
+    return 1;
 }
 
 MathKind math_kind() {
@@ -94,7 +82,7 @@ MathKind math_kind() {
 bool supported(int D, int G, MathKind mk) {
     if (D != 64 && D != 128) return false;
     if (G != 1 && G != 2 && G != 4 && G != 8) return false;
-    return mk == MathKind::kMma || G * D <= 512;
+    return mk == MathKind::kMma || G * D <= 256;
 }
 
 std::mutex g_mu;
@@ -118,19 +106,22 @@ int sm_count() {
     return g_sms[dev];
 }
 
-// Workspace layout: [counters: B*Hkv int32][part_o: grid*2*G*D f32][part_ml: grid*2*G float2]
+// Workspace layout: [counters: B*Hkv int32][part_o: grid*2*HG*G*D f32]
+// [part_ml: grid*2*HG*G float2][group counters: grid*2*HG int32]
 // [grid barrier of the fused append + decode: 2 uint32]
 struct WsLayout {
-    size_t counters, part_o, part_ml, grid_bar, total;
+    size_t counters, part_o, part_ml, slot_sync, grid_bar, total;
 };
 
 WsLayout ws_layout(const pa_dims& d, int grid) {
-    const size_t G = size_t(d.num_q_heads / d.num_kv_heads);
+    const size_t hG = size_t(heads_per_group(d.num_kv_heads, d.head_dim)) * (d.num_q_heads / d.num_kv_heads);
     WsLayout w;
     w.counters = 0;
     w.part_o = align_up(size_t(d.num_seqs) * d.num_kv_heads * 4, 256);
-    w.part_ml = align_up(w.part_o + size_t(grid) * 2 * G * d.head_dim * 4, 256);
-    w.grid_bar = align_up(w.part_ml + size_t(grid) * 2 * G * 8, 256);
+    w.part_ml = align_up(w.part_o + size_t(grid) * 2 * hG * d.head_dim * 4, 256);
+    w.slot_sync = align_up(w.part_ml + size_t(grid) * 2 * hG * 8, 256);
+    w.grid_bar = align_up(w.slot_sync + size_t(grid) * 2 * heads_per_group(d.num_kv_heads, d.head_dim) * 4,
+                          256);
     w.total = w.grid_bar + 256;
     return w;
 }
@@ -172,17 +163,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
     return fn;
 }
 
-// A cache [NB][Hkv][bs][D] bf16 seen as a 3-D tensor {64 columns, D/64
-// panels, NB*Hkv*bs rows} (strides 128 B and D*2 B); one box is one
-// 64-column panel of one (block, kv head) tile: {64, 1, bs}, 128-byte swizzle.
-bool make_cache_map(CUtensorMap* map, const void* base, int64_t rows, int D, int bs) {
+// A cache [NB][Hkv][bs][D] bf16 seen as a 4-D tensor {64 columns, bs rows,
+// D/64 panels, NB*Hkv tiles} (strides D*2 B, 128 B, bs*D*2 B).  One box is
+// `heads` consecutive (block, kv head) tiles whole: {64, bs, D/64, heads},
+// landing in shared memory as [tile][panel][row][128 B] with the 128-byte
+// swizzle.
+bool make_cache_map(CUtensorMap* map, const void* base, int64_t tiles, int D, int bs, int heads) {
     auto fn = encode_tiled();
     if (!fn) return false;
-    cuuint64_t dims[3] = {64, cuuint64_t(D / 64), cuuint64_t(rows)};
-    cuuint64_t strides[2] = {128, cuuint64_t(D) * 2};
-    cuuint32_t box[3] = {64, 1, cuuint32_t(bs)};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+    cuuint64_t dims[4] = {64, cuuint64_t(bs), cuuint64_t(D / 64), cuuint64_t(tiles)};
+    cuuint64_t strides[3] = {cuuint64_t(D) * 2, 128, cuuint64_t(bs) * D * 2};
+    cuuint32_t box[4] = {64, cuuint32_t(bs), cuuint32_t(D / 64), cuuint32_t(heads)};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, PA_L2_PROMOTION,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -191,13 +184,13 @@ bool make_cache_map(CUtensorMap* map, const void* base, int64_t rows, int D, int
 // stream (prefix_kernel), so that its set-up overlaps that kernel's end.
 template <MathKind MK, int D, int G, bool DUMP, bool APPEND>
 pa_status launch_decode(const pa::DecodeParams& p, int grid, cudaStream_t stream, bool pdl) {
-    constexpr int NW = Tune<MK, D, G>::NW, R = Tune<MK, D, G>::R, PPS = Tune<MK, D, G>::PPS;
-    using Cfg = pa::DecodeCfg<D, G, kBlockSize, NW, R, PPS>;
+    constexpr int R = ring_fit<D>();
+    using Cfg = pa::DecodeCfg<D, kBlockSize, R>;
     auto kern = [] {
         if constexpr (MK == MathKind::kMma)
-            return pa::decode_kernel<D, G, kBlockSize, NW, R, PPS, DUMP, APPEND, pa::MmaMath>;
+            return pa::decode_kernel<D, G, kBlockSize, R, DUMP, APPEND, pa::MmaMath>;
         else
-            return pa::decode_kernel<D, G, kBlockSize, NW, R, PPS, DUMP, APPEND, pa::SimtMath>;
+            return pa::decode_kernel<D, G, kBlockSize, R, DUMP, APPEND, pa::SimtMath>;
     }();
     static unsigned attr_done[kMaxDevices];
     if (!set_smem_once(kern, Cfg::kSmemBytes, attr_done)) return PA_ERR_CUDA;
@@ -232,23 +225,30 @@ pa_status launch_decode(const pa::DecodeParams& p, int grid, cudaStream_t stream
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+// The SIMT policy is built only for G*D <= 256 (its per-lane state grows with G*D).
+template <MathKind MK, int D, int G, bool DUMP, bool APPEND>
+pa_status launch_built(const pa::DecodeParams& p, int grid, cudaStream_t s, bool pdl) {
+    if constexpr (MK == MathKind::kMma || G * D <= 256)
+        return launch_decode<MK, D, G, DUMP, APPEND>(p, grid, s, pdl);
+    else
+        return PA_ERR_UNSUPPORTED;
+}
+
 template <MathKind MK, bool DUMP, bool APPEND>
 pa_status dispatch_d_g(int D, int G, const pa::DecodeParams& p, int grid, cudaStream_t s, bool pdl) {
     if (D == 64) {
         switch (G) {
-            case 1: return launch_decode<MK, 64, 1, DUMP, APPEND>(p, grid, s, pdl);
-            case 2: return launch_decode<MK, 64, 2, DUMP, APPEND>(p, grid, s, pdl);
-            case 4: return launch_decode<MK, 64, 4, DUMP, APPEND>(p, grid, s, pdl);
-            case 8: return launch_decode<MK, 64, 8, DUMP, APPEND>(p, grid, s, pdl);
+            case 1: return launch_built<MK, 64, 1, DUMP, APPEND>(p, grid, s, pdl);
+            case 2: return launch_built<MK, 64, 2, DUMP, APPEND>(p, grid, s, pdl);
+            case 4: return launch_built<MK, 64, 4, DUMP, APPEND>(p, grid, s, pdl);
+            case 8: return launch_built<MK, 64, 8, DUMP, APPEND>(p, grid, s, pdl);
         }
     } else if (D == 128) {
         switch (G) {
-            case 1: return launch_decode<MK, 128, 1, DUMP, APPEND>(p, grid, s, pdl);
-            case 2: return launch_decode<MK, 128, 2, DUMP, APPEND>(p, grid, s, pdl);
-            case 4: return launch_decode<MK, 128, 4, DUMP, APPEND>(p, grid, s, pdl);
-            case 8:
-                if constexpr (MK == MathKind::kMma) return launch_decode<MK, 128, 8, DUMP, APPEND>(p, grid, s, pdl);
-                break;
+            case 1: return launch_built<MK, 128, 1, DUMP, APPEND>(p, grid, s, pdl);
+            case 2: return launch_built<MK, 128, 2, DUMP, APPEND>(p, grid, s, pdl);
+            case 4: return launch_built<MK, 128, 4, DUMP, APPEND>(p, grid, s, pdl);
+            case 8: return launch_built<MK, 128, 8, DUMP, APPEND>(p, grid, s, pdl);
         }
     }
     return PA_ERR_UNSUPPORTED;
@@ -339,14 +339,20 @@ pa_status prepare_decode(const void* q, const void* k_cache, const void* v_cache
         !aligned16(workspace) || !aligned4(block_tables) || !aligned4(context_lens))
         return PA_ERR_ALIGN;
     if (grid <= 0) return PA_ERR_CUDA;
+    if (grid > kMaxCtas) return PA_ERR_SHAPE;
     const WsLayout w = ws_layout(d, grid);
     if (workspace_bytes < w.total) return PA_ERR_WORKSPACE;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     p = pa::DecodeParams{};
     const int64_t rows = int64_t(d.num_blocks) * d.num_kv_heads * d.block_size;
-    if (rows >= (int64_t(1) << 31)) return PA_ERR_SHAPE;  // TMA row coordinates are int32
-    if (!make_cache_map(&p.tmap_k, k_cache, rows, d.head_dim, d.block_size) ||
-        !make_cache_map(&p.tmap_v, v_cache, rows, d.head_dim, d.block_size))
+    if (rows >= (int64_t(1) << 31)) return PA_ERR_SHAPE;  // TMA coordinates are int32
+    const int HG = heads_per_group(d.num_kv_heads, d.head_dim);
+    int SPL = 1;
+    while (HG / SPL > heads_per_stage_max(d.head_dim) || HG % SPL) SPL *= 2;
+    const int HS = HG / SPL;
+    const int64_t tiles = int64_t(d.num_blocks) * d.num_kv_heads;
+    if (!make_cache_map(&p.tmap_k, k_cache, tiles, d.head_dim, d.block_size, HS) ||
+        !make_cache_map(&p.tmap_v, v_cache, tiles, d.head_dim, d.block_size, HS))
         return PA_ERR_CUDA;
     p.q = static_cast<const uint8_t*>(q);
     p.block_tables = block_tables;
@@ -358,11 +364,17 @@ pa_status prepare_decode(const void* q, const void* k_cache, const void* v_cache
     p.Hkv = d.num_kv_heads;
     p.NB = d.num_blocks;
     p.M = d.max_blocks_per_seq;
+    p.HG = HG;
+    p.NG = d.num_kv_heads / HG;
+    p.HS = HS;
+    p.SPL = SPL;
+    p.SPL_LOG = SPL == 1 ? 0 : SPL == 2 ? 1 : SPL == 4 ? 2 : 3;
     p.min_pages = kMinPagesPerCta;
-    p.seg_weight = seg_weight_pages(d.head_dim);
+    p.seg_weight = seg_weight_pages(d.head_dim, HG);
     p.counters = reinterpret_cast<int32_t*>(ws + w.counters);
     p.part_o = reinterpret_cast<float*>(ws + w.part_o);
     p.part_ml = reinterpret_cast<float2*>(ws + w.part_ml);
+    p.slot_sync = reinterpret_cast<int32_t*>(ws + w.slot_sync);
     p.grid_bar = reinterpret_cast<unsigned int*>(ws + w.grid_bar);
     return PA_OK;
 }
@@ -554,8 +566,10 @@ pa_status pa_decode_shared_prefix(const void* k_new, const void* v_new, const in
         if (int64_t(num_groups) * tiles > 0x7fffffffLL || d.num_kv_heads > 65535) return PA_ERR_SHAPE;
         uint8_t* ws = static_cast<uint8_t*>(workspace);
         pa::PrefixParams pp;
-        pp.tmap_k = p.tmap_k;
-        pp.tmap_v = p.tmap_v;
+        const int64_t cache_tiles = int64_t(d.num_blocks) * d.num_kv_heads;
+        if (!make_cache_map(&pp.tmap_k, k_cache, cache_tiles, d.head_dim, d.block_size, 1) ||
+            !make_cache_map(&pp.tmap_v, v_cache, cache_tiles, d.head_dim, d.block_size, 1))
+            return PA_ERR_CUDA;
         pp.q = p.q;
         pp.block_tables = block_tables;
         pp.context_lens = context_lens;
@@ -616,10 +630,13 @@ pa_status pa_decode_static_ws(const void* q, const void* k_cache, const void* v_
     st = prepare_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, dims, grid, scratch,
                         PA_STATIC_SCRATCH_BYTES, p);
     if (st != PA_OK || dims->num_seqs == 0) return st;
-    // the array keeps the last call's contents: the merge counters must start at zero
+    // the array keeps the last call's contents (another problem's partials may
+    // sit where this one's counters go): the merge counters must start at zero
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const WsLayout w = ws_layout(*dims, grid);
     if (cudaMemsetAsync(p.counters, 0, size_t(dims->num_seqs) * dims->num_kv_heads * sizeof(int32_t), s) !=
-        cudaSuccess)
+            cudaSuccess ||
+        cudaMemsetAsync(p.slot_sync, 0, w.grid_bar - w.slot_sync, s) != cudaSuccess)
         return PA_ERR_CUDA;
     return dispatch_decode<false>(dims->head_dim, dims->num_q_heads / dims->num_kv_heads, p, grid, s);
 }

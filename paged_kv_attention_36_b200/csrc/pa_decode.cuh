@@ -1,37 +1,46 @@
 // pa_decode.cuh -- paged decode attention for sm_100a.
 //
-// Work decomposition.  The decode reads, for every (sequence b, kv head g),
-// the np_b = ceil(L_b / bs) pages of that sequence.  Lay all (b, g) out in
-// order on one line, each taking np_b + X units: its pages, then X units
-// that stand for the fixed cost of finishing a segment (combining the warp
-// states and writing the output; X = seg_weight, measured in pages).  Each
-// persistent CTA (one per SM) takes an equal contiguous share of the line,
-// so a share made of many short segments gets fewer pages.  A share is a
-// run of "segments": whole (b, g) page lists, plus at most a partial one at
-// each end.  A whole segment is finished inside the CTA and writes bf16
-// output; a partial one writes an fp32 split-KV partial (normalised output,
-// max logit, exp-sum) and the last CTA to finish a piece of that (b, g)
-// merges the pieces by log-sum-exp (flash-decoding), so long or skewed
-// contexts are split exactly where the balance needs it and nowhere else.
+// Work decomposition.  The kv heads of a sequence are taken in head groups
+// of HG (HG = the largest divisor of Hkv that is <= 8).  The decode reads,
+// for every (sequence b, head group hg), np_b = ceil(L_b / bs) pages; a page
+// is one physical block's K and V tiles for the HG heads, which sit next to
+// each other in the cache.  Lay all (b, hg) out in order on one line, each
+// taking np_b + X units: its pages, then X units for the fixed cost of
+// finishing a segment (X = seg_weight, measured in pages).  Each persistent
+// CTA (one per SM) takes an equal contiguous share of the line, a run of
+// "segments": whole (b, hg) page lists, plus at most a partial one at each
+// end.  A whole segment writes bf16 output; a partial one writes fp32
+// split-KV partials (normalised output, max logit, exp-sum) and the last
+// CTA to finish a piece of that (b, kv head) merges the pieces by
+// log-sum-exp (flash-decoding), so long or skewed contexts are split exactly
+// where the balance needs it and nowhere else.  A (b, kv head) in two
+// pieces takes its merge ticket first: the first piece to finish publishes
+// its partial with a ready flag and the other folds it into its own
+// registers, so the merge adds two memory round trips to that CTA.  More
+// pieces publish first and the last merges from memory, in two levels
+// beyond 16 pieces: the last piece to finish in each run of 16 merges that
+// run, and the last run merges the runs, so no CTA reads more than 16.
 //
-// Inside a CTA.  Warp NW (the producer) walks the CTA's share, reads block
-// ids from the block table and streams each (block, kv head) K tile and V
-// tile into a ring of R shared-memory stages with tiled TMA copies
-// (128-byte swizzle), completing on a per-stage mbarrier.  Per segment it
-// also copies the G query rows of kv head g (contiguous in q) into a small
-// descriptor ring.  Warps 0..NW-1 (consumers) take stage i when i % NW
-// equals their index, so each page is read by exactly one warp and no
-// CTA-wide barrier is needed per page.  Each consumer warp keeps its own
-// online-softmax state (running max m, running sum l, fp32 accumulator) for
-// all G query heads; at a segment end the warps combine their states
-// through shared memory.  Every wait on an mbarrier is bounded in time.
+// Inside a CTA.  Warp 8 (the producer) walks the share, reads one block id
+// per page from the block table and copies the page into a ring of R
+// shared-memory stages of 32 KB: SPL stages per page (1 at head_dim 64, 2 at
+// head_dim 128 with 8 heads), each holding HS = HG / SPL heads' K tiles and
+// then their V tiles, moved by two tiled TMA copies (a 4-D box over
+// [tile][panel][row][column], 128-byte swizzle) that complete on the
+// stage's mbarrier.  Consumer warp w < HG owns kv head hg*HG + w: it reads
+// its head's tiles from stage w / HS of every page, keeps the
+// online-softmax state (running max m, running sum l, fp32 accumulator) of
+// its G query heads, and at a segment end writes that head's output or
+// partial by itself.  A stage is free again when its HS warps have read it;
+// no CTA-wide barrier is taken per page or per segment.  Every wait on an
+// mbarrier is bounded in time.
 //
-// Staged tile layout.  A (block, kv head) tile is bs = 16 rows of D bf16.
-// TMA writes it as D/64 panels of 16 lines x 128 bytes (panel p holds
-// columns 64p .. 64p+63), with the 128-byte swizzle: the 16-byte chunk c of
-// line t sits at chunk position c ^ (t % 8).  Any 8 consecutive rows read
-// at one logical chunk therefore hit 8 different bank groups, which makes
-// both the SIMT row reads and the tensor-core ldmatrix reads conflict-free.
+// Staged tile layout.  A (block, kv head) tile is bs = 16 rows of D bf16,
+// held as D/64 panels of 16 lines x 128 bytes (panel p holds columns
+// 64p .. 64p+63) with the 128-byte swizzle: the 16-byte chunk c of line t
+// sits at chunk position c ^ (t % 8).  Any 8 consecutive rows read at one
+// logical chunk therefore hit 8 different bank groups, which makes both the
+// SIMT row reads and the tensor-core ldmatrix reads conflict-free.
 //
 // Per-page math, two policies:
 //   SimtMath: lane = 8*tg + c; the 8 lanes of token group tg share one K
@@ -51,8 +60,9 @@
 #ifndef PA_EVICT_FIRST
 #define PA_EVICT_FIRST 1  // K/V pages are read once: first candidates for L2 eviction
 #endif
-#ifndef PA_L2_PREFETCH
-#define PA_L2_PREFETCH 0  // L2-prefetch a page before waiting for its stage
+
+#ifndef PA_STAGE_K_BYTES
+#define PA_STAGE_K_BYTES 16384  // K bytes of a ring stage (as many V bytes follow)
 #endif
 
 namespace pa {
@@ -66,11 +76,15 @@ struct DecodeParams {
     __nv_bfloat16* out;           // [B][Hq][D]
     float qscale;                 // scale * log2(e): logits in base-2 units
     int32_t B, Hq, Hkv, NB, M;
+    int32_t HG, NG;               // kv heads per head group (<= 8), head groups per sequence
+    int32_t HS, SPL, SPL_LOG;     // kv heads per ring stage, stages per page (HG = HS * SPL, SPL = 2^SPL_LOG)
     int32_t min_pages;            // fewest pages worth giving a CTA
     int32_t seg_weight;           // cost of finishing a segment, in pages (weights the split)
     int32_t* counters;            // [B*Hkv] merge tickets, zero between calls
-    float* part_o;                // [grid][2][G][D] split-KV partial outputs
-    float2* part_ml;              // [grid][2][G] (max logit base 2, exp-sum)
+    int32_t* slot_sync;           // [grid][2][HG], per partial slot: a ready flag (a (b, kv head) in two
+                                  // pieces) or a run ticket (> 16 pieces); zero between calls
+    float* part_o;                // [grid][2][HG*G][D] split-KV partial outputs
+    float2* part_ml;              // [grid][2][HG*G] (max logit base 2, exp-sum)
     // test hook (DUMP): every segment's partials
     int32_t dump_capacity;
     int32_t* seg_meta;
@@ -98,11 +112,11 @@ struct DecodeParams {
 
 // One segment of a CTA's share, handed from the producer to the consumers.
 struct SegDesc {
-    int32_t b, g;
+    int32_t b, hg;     // sequence, head group
     int32_t j0;        // first page of the segment within sequence b
     int32_t npg;       // pages in the segment; 0 marks the end of the share
     int32_t L;         // context length of b
-    int32_t k0, k1;    // CTAs holding pages of (b, g); whole iff k0 == k1
+    int32_t k0, k1;    // CTAs holding pages of (b, hg); whole iff k0 == k1
     int32_t P;         // shared-prefix pages of b (the line holds pages P .. ceil(L/bs)-1)
     int32_t pad[8];
 };
@@ -121,11 +135,7 @@ struct Split {
 // Shared scalars.
 struct Misc {
     int abort;
-    int is_last;
-    int dump_idx;
-    int found;
     int b0;              // sequence where the share starts
-    int pad1;
     long long pre0;      // weighted position of b0's first unit
     long long red[16];  // block reductions, one slot per warp (<= 16 warps)
 };
@@ -146,23 +156,8 @@ struct SimtMath {
     float m[G];
     float l[G];
 
-    __device__ __forceinline__ void load_q(const uint8_t* qs, int lane, float qscale) {
-        const int c = lane & 7;
-#pragma unroll
-        for (int h = 0; h < G; ++h)
-#pragma unroll
-            for (int i = 0; i < NCH; ++i) {
-                const uint4 v = lds128(qs + h * D * 2 + (c + 8 * i) * 16);
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float2 f = bf16x2_to_float2(w[j]);
-                    q2[h][i][j] = make_float2(f.x * qscale, f.y * qscale);
-                }
-            }
-    }
-
-    // Same, from global memory (the G rows of q of one kv head).
+    // q of the G query heads of one kv head (G rows of D bf16, global
+    // memory), pre-scaled by scale * log2(e).
     __device__ __forceinline__ void load_q_global(const uint8_t* gq, int lane, float qscale) {
         const int c = lane & 7;
 #pragma unroll
@@ -329,24 +324,48 @@ struct SimtMath {
         }
     }
 
-    // Warp state -> dep: acc[h][d] (G*D floats), then m[h], then l[h].
-    __device__ __forceinline__ void deposit(float* dep, int lane) const {
+    // After finish(): out[h][:] = acc / l in bf16, for the G heads.
+    __device__ __forceinline__ void store_out(__nv_bfloat16* out, int lane) const {
         const int tg = lane >> 3, c = lane & 7;
-        if (tg == 0) {
+        if (tg != 0) return;
 #pragma unroll
-            for (int h = 0; h < G; ++h)
+        for (int h = 0; h < G; ++h) {
+            const float inv = 1.f / l[h];
 #pragma unroll
-                for (int i = 0; i < NCH; ++i) {
-                    float4* dst = reinterpret_cast<float4*>(dep + h * D + (c + 8 * i) * 8);
-                    dst[0] = make_float4(acc[h][i][0].x, acc[h][i][0].y, acc[h][i][1].x, acc[h][i][1].y);
-                    dst[1] = make_float4(acc[h][i][2].x, acc[h][i][2].y, acc[h][i][3].x, acc[h][i][3].y);
-                }
+            for (int i = 0; i < NCH; ++i) {
+                uint4 v;
+                v.x = float2_to_bf16x2(acc[h][i][0].x * inv, acc[h][i][0].y * inv);
+                v.y = float2_to_bf16x2(acc[h][i][1].x * inv, acc[h][i][1].y * inv);
+                v.z = float2_to_bf16x2(acc[h][i][2].x * inv, acc[h][i][2].y * inv);
+                v.w = float2_to_bf16x2(acc[h][i][3].x * inv, acc[h][i][3].y * inv);
+                *reinterpret_cast<uint4*>(out + h * D + (c + 8 * i) * 8) = v;
+            }
         }
-        if (lane == 0) {
+    }
+    // After finish(): o[h][:] = acc / l (fp32) and the (max logit base 2,
+    // exp-sum) pair of each head: to ml[h] if ml, else m (natural log units)
+    // to mo[h] and l to lo[h].
+    __device__ __forceinline__ void store_partial(float* o, float2* ml, float* mo, float* lo, int lane) const {
+        const int tg = lane >> 3, c = lane & 7;
+        if (tg != 0) return;
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-                dep[G * D + h] = m[h];
-                dep[G * D + G + h] = l[h];
+        for (int h = 0; h < G; ++h) {
+            const float inv = 1.f / l[h];
+#pragma unroll
+            for (int i = 0; i < NCH; ++i) {
+                float4* dst = reinterpret_cast<float4*>(o + h * D + (c + 8 * i) * 8);
+                dst[0] = make_float4(acc[h][i][0].x * inv, acc[h][i][0].y * inv, acc[h][i][1].x * inv,
+                                     acc[h][i][1].y * inv);
+                dst[1] = make_float4(acc[h][i][2].x * inv, acc[h][i][2].y * inv, acc[h][i][3].x * inv,
+                                     acc[h][i][3].y * inv);
+            }
+            if (c == 0) {
+                if (ml) {
+                    ml[h] = make_float2(m[h], l[h]);
+                } else {
+                    mo[h] = m[h] * 0.69314718055994531f;
+                    lo[h] = l[h];
+                }
             }
         }
     }
@@ -370,22 +389,8 @@ struct MmaMath {
     float m[2], l[2];    // heads h0, h0 + 1 of this lane (l: this lane's rows only)
     float qscale;
 
-    __device__ __forceinline__ void load_q(const uint8_t* qs, int lane, float qs_scale) {
-        qscale = qs_scale;
-        const int h = lane >> 2, kk = (lane & 3) * 2;
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-            if (h < G) {
-                const uint8_t* row = qs + h * D * 2;
-                qb[ks][0] = *reinterpret_cast<const uint32_t*>(row + (16 * ks + kk) * 2);
-                qb[ks][1] = *reinterpret_cast<const uint32_t*>(row + (16 * ks + kk + 8) * 2);
-            } else {
-                qb[ks][0] = qb[ks][1] = 0u;
-            }
-        }
-    }
-
-    // Same, from global memory (the G rows of q of one kv head).
+    // q of the G query heads of one kv head (G rows of D bf16, global
+    // memory) as B fragments; the logits are scaled by scale * log2(e) later.
     __device__ __forceinline__ void load_q_global(const uint8_t* gq, int lane, float qs_scale) {
         qscale = qs_scale;
         const int h = lane >> 2, kk = (lane & 3) * 2;
@@ -525,56 +530,75 @@ struct MmaMath {
         }
     }
 
-    // Warp state -> dep: acc[h][d] (G*D floats), then m[h], then l[h].
-    __device__ __forceinline__ void deposit(float* dep, int lane) const {
+    // After finish(): out[h][:] = acc / l in bf16, for the G heads.
+    __device__ __forceinline__ void store_out(__nv_bfloat16* out, int lane) const {
         const int h0 = (lane & 3) * 2, d0 = lane >> 2;
 #pragma unroll
-        for (int mt = 0; mt < KS; ++mt) {
-            const int d = 16 * mt + d0;
-            if (h0 < G) {
-                dep[h0 * D + d] = acc[mt][0];
-                dep[h0 * D + d + 8] = acc[mt][2];
-            }
-            if (h0 + 1 < G) {
-                dep[(h0 + 1) * D + d] = acc[mt][1];
-                dep[(h0 + 1) * D + d + 8] = acc[mt][3];
+        for (int e = 0; e < 2; ++e) {
+            const int h = h0 + e;
+            if (h >= G) continue;
+            const float inv = 1.f / l[e];
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+                out[h * D + 16 * mt + d0] = __float2bfloat16_rn(acc[mt][e] * inv);
+                out[h * D + 16 * mt + d0 + 8] = __float2bfloat16_rn(acc[mt][2 + e] * inv);
             }
         }
-        if (d0 == 0) {
+    }
+    // After finish(): o[h][:] = acc / l (fp32) and the (max logit base 2,
+    // exp-sum) pair of each head: to ml[h] if ml, else m (natural log units)
+    // to mo[h] and l to lo[h].
+    __device__ __forceinline__ void store_partial(float* o, float2* ml, float* mo, float* lo, int lane) const {
+        const int h0 = (lane & 3) * 2, d0 = lane >> 2;
 #pragma unroll
-            for (int e = 0; e < 2; ++e)
-                if (h0 + e < G) {
-                    dep[G * D + h0 + e] = m[e];
-                    dep[G * D + G + h0 + e] = l[e];
+        for (int e = 0; e < 2; ++e) {
+            const int h = h0 + e;
+            if (h >= G) continue;
+            const float inv = 1.f / l[e];
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+                o[h * D + 16 * mt + d0] = acc[mt][e] * inv;
+                o[h * D + 16 * mt + d0 + 8] = acc[mt][2 + e] * inv;
+            }
+            if (d0 == 0) {
+                if (ml) {
+                    ml[h] = make_float2(m[e], l[e]);
+                } else {
+                    mo[h] = m[e] * 0.69314718055994531f;
+                    lo[h] = l[e];
                 }
+            }
         }
     }
 };
 
 // ===========================================================================
-template <int D, int G, int BS, int NW, int R, int PPS>
+// Consumer warps of a decode CTA: warp w < HG owns kv head hg*HG + w.
+constexpr int kDecodeWarps = 8;
+
+template <int D, int BS, int R>
 struct DecodeCfg {
+    static constexpr int NW = kDecodeWarps;
     static constexpr int kRow = D * 2;              // bytes of one K or V row
     static constexpr int kTile = BS * kRow;         // one (block, kv head) tile
     static constexpr int kPanel = BS * 128;         // one 64-column panel of a tile
-    static constexpr int kPage = 2 * kTile;         // K tile then V tile
-    static constexpr int kStage = PPS * kPage;      // PPS pages of one segment
+    static constexpr int kStageK = PA_STAGE_K_BYTES;  // K tiles of up to kHeadsPerStage heads of one block
+    static constexpr int kStage = 2 * kStageK;        // then their V tiles
+    static constexpr int kHeadsPerStage = kStageK / kTile;
+    static constexpr int kMaxSpl = NW / kHeadsPerStage > 1 ? NW / kHeadsPerStage : 1;  // stages per page, at most
+    static_assert(kHeadsPerStage >= 1, "a stage holds at least one head's tiles");
     static constexpr int kSegSlots = 4;
-    static constexpr int kQBytes = G * kRow;
-    static constexpr int kCombFloats = G * D + ((2 * G + 3) / 4) * 4;  // one warp's state, 16-byte padded
     static constexpr int kThreads = (NW + 1) * 32;
 
     // offsets from the 1024-byte aligned base
     static constexpr int kRingOff = 0;
-    static constexpr int kQOff = kRingOff + R * kStage;
-    static constexpr int kDescOff = kQOff + kSegSlots * kQBytes;
-    static constexpr int kCombOff = kDescOff + kSegSlots * int(sizeof(SegDesc));
-    static constexpr int kBarOff = kCombOff + NW * kCombFloats * 4;
-    static constexpr int kNumBars = 2 * R + 2 * kSegSlots + 1;
+    static constexpr int kDescOff = kRingOff + R * kStage;
+    static constexpr int kBarOff = kDescOff + kSegSlots * int(sizeof(SegDesc));
+    static constexpr int kNumBars = 2 * R + 2 * kSegSlots;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kMiscBytes = 256;
     static constexpr int kSmemBytes = kMiscOff + kMiscBytes + 1024;  // + alignment slack
-    static_assert(kQBytes % 16 == 0 && kTile % 1024 == 0, "TMA tile alignment");
+    static_assert(kTile % 1024 == 0 && kStage % 1024 == 0, "TMA tile alignment");
     static_assert(kBarOff % 8 == 0, "mbarrier alignment");
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
@@ -645,44 +669,163 @@ __device__ __forceinline__ SeqPages seq_pages(const DecodeParams& p, int b, bool
     return s;
 }
 
-template <int D, int G, int BS, int NW, int R, int PPS, bool DUMP, bool APPEND, template <int, int, int> class Math>
-__global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
-    // Stage i % R always feeds warp i % NW, so a warp waiting on a stage is at
-    // most one phase away from it and the parity waits are exact.
-    static_assert(R % NW == 0, "ring depth must be a multiple of the consumer warps");
-    static_assert(NW + 1 <= 16, "block reductions hold 16 warps");
-    using Cfg = DecodeCfg<D, G, BS, NW, R, PPS>;
+// Split-KV merge.  Pieces of a (b, kv head) are merged in registers by the
+// last one when there are at most kFastMergePieces, else from memory in
+// runs of at most kMergeFanIn; with at most 1024 CTAs there are at most 64 runs.
+constexpr int kFastMergePieces = 2;  // one other piece in registers: fits the 168-register budget
+constexpr int kMergeFanIn = 16;
+
+// Slot index of piece `leaf` of a (b, hg) whose first piece is in CTA k0:
+// leaf 0 sits in slot 1 of CTA k0, every other leaf in slot 0 of its CTA.
+__device__ __forceinline__ int64_t leaf_slot(int k0, int leaf) {
+    return int64_t(k0 + leaf) * 2 + (leaf == 0 ? 1 : 0);
+}
+
+// Adds this warp's arrival to a ticket counter; true in every lane of the
+// warp whose arrival completes `count` (the caller has fenced its writes).
+__device__ __forceinline__ bool ticket(int32_t* counter, int count, int lane) {
+    int last = 0;
+    if (lane == 0) last = atomicAdd(counter, 1) == count - 1;
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last) __threadfence();
+    return last != 0;
+}
+
+// Merges, by log-sum-exp, the split-KV partials of one warp's (b, kv head)
+// held by the pieces ("leaves") off, off + stride, ... (n <= 64 of them) of
+// the CTAs k0 + leaf: into out (bf16, [G][D]) if given, else into the
+// partial slot of leaf `off`.  Leaf 0 sits in slot 1 of CTA k0, every other
+// leaf in slot 0 of its CTA.  Lane l loads the (max, sum) of pieces l and
+// l + 32 for each head; the weighted sums keep a pass's loads in flight.
+constexpr int kMergeMaxPieces = 64;
+
+template <int D, int G>
+__device__ __noinline__ void merge_pieces(const DecodeParams& p, int k0, int off, int stride, int n, int HG,
+                                          int warp, int lane, __nv_bfloat16* out) {
+    auto base = [&](int i) -> int64_t {
+        const int leaf = off + i * stride;
+        return ((int64_t(k0 + leaf) * 2 + (leaf == 0 ? 1 : 0)) * HG + warp) * G;
+    };
+    float M[G], lsum[G], w[G][2];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        float2 ml[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int i = lane + 32 * r;
+            ml[r] = i < n ? __ldcg(&p.part_ml[base(i) + h]) : make_float2(-INFINITY, 0.f);
+        }
+        float mx = fmaxf(ml[0].x, ml[1].x);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float sm = 0.f;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            w[h][r] = lane + 32 * r < n ? ml[r].y * exp2f(ml[r].x - mx) : 0.f;
+            sm += w[h][r];
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
+        M[h] = mx;
+        lsum[h] = sm;
+    }
+    // pass t covers elements 128t .. 128t+127 of [G][D]: heads hl and hl + 1
+    // (head_dim 64) or hl alone (head_dim 128); this lane's 4 are e .. e+3.
+    // The piece loop is outermost so that every pass's load of 4 pieces is
+    // in flight at once.
+    constexpr int T = (G * D + 127) / 128;
+    constexpr int hstep = 128 / D;
+    float4 a[T];
+#pragma unroll
+    for (int t = 0; t < T; ++t) a[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int i = 0; i < n; ++i) {
+        const int r = i >> 5, src = i & 31;
+        const int64_t bi = base(i);
+#pragma unroll
+        for (int t = 0; t < T; ++t) {
+            const int e = 128 * t + 4 * lane;
+            const int hl = (128 * t) / D;
+            const bool valid = e < G * D;
+            const int h = valid ? e / D : 0, dd = e - h * D;
+            // every lane takes part in the shuffles; only valid lanes load
+            float wi = __shfl_sync(0xffffffffu, r ? w[hl < G ? hl : 0][1] : w[hl < G ? hl : 0][0], src);
+            if (hstep > 1 && hl + 1 < G) {
+                const int h1 = hl + 1 < G ? hl + 1 : 0;
+                const float wj = __shfl_sync(0xffffffffu, r ? w[h1][1] : w[h1][0], src);
+                if (h != hl) wi = wj;
+            }
+            if (valid) {
+                const float4 v = __ldcg(reinterpret_cast<const float4*>(&p.part_o[(bi + h) * D + dd]));
+                a[t].x += wi * v.x;
+                a[t].y += wi * v.y;
+                a[t].z += wi * v.z;
+                a[t].w += wi * v.w;
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+        const int e = 128 * t + 4 * lane;
+        if (e >= G * D) continue;
+        const int h = e / D, dd = e - h * D;
+        float ls = lsum[0];
+#pragma unroll
+        for (int hh = 1; hh < G; ++hh)
+            if (hh == h) ls = lsum[hh];
+        const float inv = 1.f / ls;
+        if (out) {
+            *reinterpret_cast<uint2*>(out + h * D + dd) = make_uint2(float2_to_bf16x2(a[t].x * inv, a[t].y * inv),
+                                                                     float2_to_bf16x2(a[t].z * inv, a[t].w * inv));
+        } else {
+            *reinterpret_cast<float4*>(&p.part_o[(base(0) + h) * D + dd]) =
+                make_float4(a[t].x * inv, a[t].y * inv, a[t].z * inv, a[t].w * inv);
+        }
+    }
+    if (!out && lane < G) {
+        float mh = M[0], lh = lsum[0];
+#pragma unroll
+        for (int hh = 1; hh < G; ++hh)
+            if (hh == lane) {
+                mh = M[hh];
+                lh = lsum[hh];
+            }
+        p.part_ml[base(0) + lane] = make_float2(mh, lh);
+    }
+}
+
+template <int D, int G, int BS, int R, bool DUMP, bool APPEND, template <int, int, int> class Math>
+__global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
+    using Cfg = DecodeCfg<D, BS, R>;
+    constexpr int NW = Cfg::NW;
     constexpr int S = Cfg::kSegSlots;
     constexpr int NT = Cfg::kThreads;
-    constexpr int NPANEL = D / 64;
+    static_assert(NW + 1 <= 16, "block reductions hold 16 warps");
+    static_assert(R % Cfg::kMaxSpl == 0, "the stages of a page recur in the same slots");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* ring = smem + Cfg::kRingOff;
-    uint8_t* qring = smem + Cfg::kQOff;
     SegDesc* descs = reinterpret_cast<SegDesc*>(smem + Cfg::kDescOff);
-    float* combbuf = reinterpret_cast<float*>(smem + Cfg::kCombOff);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
     uint64_t* empty = full + R;
     uint64_t* segfull = empty + R;
     uint64_t* segempty = segfull + S;
-    uint64_t* consbar = segempty + S;
     Misc* misc = reinterpret_cast<Misc*>(smem + Cfg::kMiscOff);
     volatile int* abort = &misc->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int HG = p.HG, HS = p.HS, SPL = p.SPL;
 
     if (threadIdx.x == 0) {
         for (int r = 0; r < R; ++r) {
             mbar_init(&full[r], 1);
-            mbar_init(&empty[r], 1);
+            mbar_init(&empty[r], uint32_t(HS));
         }
         for (int s = 0; s < S; ++s) {
             mbar_init(&segfull[s], 1);
-            mbar_init(&segempty[s], NW);
+            mbar_init(&segempty[s], uint32_t(HG));
         }
-        mbar_init(consbar, NW);
         misc->abort = 0;
-        misc->found = 0;
         fence_mbar_init();
     }
 
@@ -715,9 +858,9 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
         if (threadIdx.x == 0) atomicAdd(&p.grid_bar[0], 1u);
     }
 
-    // ---- the CTA's share: a scan of v_b = Hkv * pages(b) over the sequences;
-    // sequences with no context get zero output here.  When B fits in one
-    // chunk the same scan also locates the share's ends (no second read). ----
+    // ---- the CTA's share: a scan of v_b = NG * (pages(b) + seg_weight) over
+    // the sequences; sequences with no context get zero output here.  When B
+    // fits in one chunk the same scan also locates the share's start. ----
     const bool one_chunk = p.B <= NT;
     long long v_mine = 0, incl_mine = 0, Wt = 0;
     for (int base = 0; base < p.B; base += NT) {
@@ -725,7 +868,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
         long long v = 0;
         if (b < p.B) {
             const SeqPages sp = seq_pages<BS>(p, b, blockIdx.x == 0);
-            v = (long long)(sp.np > 0 ? sp.np + p.seg_weight : 0) * p.Hkv;
+            v = (long long)(sp.np > 0 ? sp.np + p.seg_weight : 0) * p.NG;
             if (sp.L == 0 && (b % int(gridDim.x)) == int(blockIdx.x)) {
                 uint4* o = reinterpret_cast<uint4*>(p.out + int64_t(b) * p.Hq * D);
                 for (int i = 0; i < p.Hq * D / 8; ++i) o[i] = make_uint4(0, 0, 0, 0);
@@ -813,7 +956,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
             long long v = 0;
             if (b < p.B) {
                 const int32_t npb = seq_pages<BS>(p, b, false).np;
-                v = (long long)(npb > 0 ? npb + p.seg_weight : 0) * p.Hkv;
+                v = (long long)(npb > 0 ? npb + p.seg_weight : 0) * p.NG;
             }
             long long chunk_total;
             const long long incl = carry + block_incl_scan<NT>(v, misc->red, chunk_total);
@@ -833,14 +976,15 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
         constexpr int C = R < 32 ? R : 32;
         bool ok = true;
         const uint64_t pol = PA_EVICT_FIRST ? policy_evict_first() : policy_evict_normal();
+        const uint32_t stage_tx = uint32_t(2 * HS * Cfg::kTile);
 
-        // walk the (b, g) whose units meet the share [p_start, p_end)
+        // walk the (b, hg) whose units meet the share [p_start, p_end)
         int b = misc->b0;
         SeqPages sp = seq_pages<BS>(p, b, false);
         int32_t Lb = sp.L, Pb = sp.P, np = sp.np;  // the line holds b's pages Pb .. Pb+np-1
         int64_t unit = np + p.seg_weight;
-        int g = int((p_start - misc->pre0) / unit);
-        int64_t u0 = misc->pre0 + int64_t(g) * unit;  // line position of (b, g)'s first page
+        int hg = int((p_start - misc->pre0) / unit);
+        int64_t u0 = misc->pre0 + int64_t(hg) * unit;  // line position of (b, hg)'s first page
         while (ok && u0 < p_end) {
             const int64_t lo = p_start > u0 ? p_start : u0;
             const int64_t hi = p_end < u0 + np ? p_end : u0 + np;
@@ -853,72 +997,42 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
                     if (ok) {
                         SegDesc& d = descs[s];
                         d.b = b;
-                        d.g = g;
+                        d.hg = hg;
                         d.j0 = j;
                         d.npg = npg;
                         d.L = Lb;
                         d.k0 = split.owner(u0);
                         d.k1 = split.owner(u0 + np - 1);
                         d.P = Pb;
-                        mbar_arrive_expect_tx(&segfull[s], Cfg::kQBytes);
-                        bulk_g2s(qring + s * Cfg::kQBytes,
-                                 p.q + (int64_t(b) * p.Hq + int64_t(g) * G) * Cfg::kRow, Cfg::kQBytes,
-                                 &segfull[s]);
+                        mbar_arrive(&segfull[s]);
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
-                // one lane per stage of PPS consecutive pages of the segment
+                // one lane per stage: HS heads' K tiles, then their V tiles
                 const int32_t* bt = p.block_tables + int64_t(b) * p.M + j;
-                const int nst = (npg + PPS - 1) / PPS;
+                const int tile0 = hg * HG;
+                const int nst = npg * SPL;
                 for (int c0 = 0; ok && c0 < nst; c0 += C) {
                     const int n = (nst - c0) < C ? (nst - c0) : C;
                     bool lane_ok = true;
                     if (lane < n) {
-                        const int sj = (c0 + lane) * PPS;  // first page of the stage in the segment
-                        const int npst = (npg - sj) < PPS ? (npg - sj) : PPS;
-                        int32_t blk[PPS];
-#pragma unroll
-                        for (int q = 0; q < PPS; ++q) {
-                            blk[q] = 0;
-                            if (q < npst) {
-                                blk[q] = __ldg(bt + sj + q);
-                                if (blk[q] < 0 || blk[q] >= p.NB) {
-                                    raise_error(PA_DEVERR_BLOCK_ID);
-                                    blk[q] = 0;
-                                }
-                            }
+                        const int x = c0 + lane;
+                        const int pg = x >> p.SPL_LOG, sub = x & (SPL - 1);
+                        int32_t blk = __ldg(bt + pg);
+                        if (blk < 0 || blk >= p.NB) {
+                            raise_error(PA_DEVERR_BLOCK_ID);
+                            blk = 0;
                         }
-                        const uint32_t i = stage_i + c0 + lane;
+                        const uint32_t i = stage_i + x;
                         const int slot = int(i % R);
                         const uint32_t use = i / R;
-                        if (PA_L2_PREFETCH && use > 0) {
-                            // start the DRAM read now; the load below waits for a free stage
-#pragma unroll
-                            for (int q = 0; q < PPS; ++q)
-                                if (q < npst)
-#pragma unroll
-                                    for (int pn = 0; pn < NPANEL; ++pn) {
-                                        tma_prefetch_3d(&p.tmap_k, 0, pn, (blk[q] * p.Hkv + g) * BS, pol);
-                                        tma_prefetch_3d(&p.tmap_v, 0, pn, (blk[q] * p.Hkv + g) * BS, pol);
-                                    }
-                        }
                         if (use > 0) lane_ok = mbar_wait(&empty[slot], (use - 1) & 1, abort);
                         if (lane_ok) {
                             uint8_t* st = ring + slot * Cfg::kStage;
-                            mbar_arrive_expect_tx(&full[slot], uint32_t(npst) * Cfg::kPage);
-#pragma unroll
-                            for (int q = 0; q < PPS; ++q) {
-                                if (q < npst) {
-                                    const int row = (blk[q] * p.Hkv + g) * BS;
-                                    uint8_t* pg = st + q * Cfg::kPage;
-#pragma unroll
-                                    for (int pn = 0; pn < NPANEL; ++pn) {
-                                        tma_load_3d(pg + pn * Cfg::kPanel, &p.tmap_k, 0, pn, row, &full[slot], pol);
-                                        tma_load_3d(pg + Cfg::kTile + pn * Cfg::kPanel, &p.tmap_v, 0, pn, row,
-                                                    &full[slot], pol);
-                                    }
-                                }
-                            }
+                            mbar_arrive_expect_tx(&full[slot], stage_tx);
+                            const int tile = blk * p.Hkv + tile0 + sub * HS;
+                            tma_load_4d(st, &p.tmap_k, 0, 0, 0, tile, &full[slot], pol);
+                            tma_load_4d(st + Cfg::kStageK, &p.tmap_v, 0, 0, 0, tile, &full[slot], pol);
                         }
                     }
                     ok = __all_sync(0xffffffffu, lane_ok);
@@ -926,10 +1040,10 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
                 stage_i += nst;
                 ++seg_i;
             }
-            // next (b, g) on the line (sequences without context take no units)
+            // next (b, hg) on the line (sequences without own pages take no units)
             u0 += unit;
-            if (u0 < p_end && ++g == p.Hkv) {
-                g = 0;
+            if (u0 < p_end && ++hg == p.NG) {
+                hg = 0;
                 do {
                     ++b;
                     sp = seq_pages<BS>(p, b, false);
@@ -958,197 +1072,164 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) decode_kernel(const __grid_c
         }
         return;
     }
+    if (warp >= HG) return;
 
     // ========================= consumer warps =========================
-    Math<D, G, BS> st;
-    const int ct = threadIdx.x;  // 0 .. NW*32-1
-    uint32_t stage_base = 0, seg_i = 0, cons_phase = 0;
-
-    auto rendezvous = [&]() -> bool {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(consbar);
-        const bool ok = mbar_wait(consbar, cons_phase & 1, abort);
-        ++cons_phase;
-        return ok;
-    };
+    using MathT = Math<D, G, BS>;
+    MathT st;
+    uint32_t stage_base = 0, seg_i = 0;
+    const int64_t hgG = int64_t(HG) * G;  // query heads of one partial slot
+    const int sub = warp / HS;              // this warp's stage within a page
+    const int pos = warp - sub * HS;        // and its tile within that stage
 
     while (true) {
         const int s = seg_i % S;
         if (!mbar_wait(&segfull[s], (seg_i / S) & 1, abort)) return;
         const SegDesc d = descs[s];
-        if (d.npg == 0) break;
-        st.load_q(qring + s * Cfg::kQBytes, lane, p.qscale);
         __syncwarp();
         if (lane == 0) mbar_arrive(&segempty[s]);
+        if (d.npg == 0) break;
+        const int g = d.hg * HG + warp;  // this warp's kv head
+        const int64_t row = int64_t(d.b) * p.Hq + int64_t(g) * G;  // its first query head
+        st.load_q_global(p.q + row * (D * 2), lane, p.qscale);
         st.reset();
         // The piece that starts at b's first own page carries the shared
-        // prefix: warp z loads the partial of prefix key range z now and
-        // folds it in after its pages (the loads overlap the pages).
+        // prefix: the partial of prefix key range 0 is loaded now and folded
+        // in after the pages (the loads overlap them), the others after it.
         const int nz = (d.P > 0 && d.j0 == d.P)
                            ? (d.P + prefix_split_pages(d.P, p.prefix_splits) - 1) /
                                  prefix_split_pages(d.P, p.prefix_splits)
                            : 0;
-        typename Math<D, G, BS>::Piece piece;
-        if (warp < nz) {
-            const int64_t idx = (int64_t(warp) * p.B + d.b) * p.Hq + int64_t(d.g) * G;
-            st.piece_load(piece, p.prefix_o + idx * D, p.prefix_ml + idx, lane);
-        }
+        typename MathT::Piece piece;
+        if (nz > 0) st.piece_load(piece, p.prefix_o + row * D, p.prefix_ml + row, lane);
 
-        const int nst = (d.npg + PPS - 1) / PPS;
-        for (int k = int((uint32_t(warp) + NW - stage_base % NW) % NW); k < nst; k += NW) {
-            const uint32_t i = stage_base + k;
+        // (R is a multiple of SPL, so the stages of each warp recur in the
+        // same slots and every parity wait is exact)
+        for (int k = 0; k < d.npg; ++k) {
+            const uint32_t i = stage_base + uint32_t(k * SPL + sub);
             const int slot = int(i % R);
             if (!mbar_wait(&full[slot], (i / R) & 1, abort)) return;
-            uint8_t* stg = ring + slot * Cfg::kStage;
-#pragma unroll
-            for (int q = 0; q < PPS; ++q) {
-                const int pgi = k * PPS + q;  // page of the segment
-                if (pgi >= d.npg) break;
-                uint8_t* pg = stg + q * Cfg::kPage;
-                const int nv_raw = d.L - (d.j0 + pgi) * BS;
-                const int nv = nv_raw < BS ? nv_raw : BS;
-                if (Math<D, G, BS>::kZeroMaskedV && nv < BS) {
-                    // rows past the context may hold anything (NaN included): clear
-                    // them in the V tile so that 0 * row stays 0 in the tensor core
-                    const int per_panel = (BS - nv) * 8;  // 16-byte chunks
-                    for (int x = lane; x < NPANEL * per_panel; x += 32) {
-                        const int pn = x / per_panel, rem = x - pn * per_panel;
-                        const int t = nv + (rem >> 3), cch = rem & 7;
-                        *reinterpret_cast<uint4*>(pg + Cfg::kTile + pn * Cfg::kPanel + t * 128 + cch * 16) =
-                            make_uint4(0, 0, 0, 0);
-                    }
-                    __syncwarp();
-                    fence_proxy_async_smem();
+            uint8_t* kt = ring + slot * Cfg::kStage + pos * Cfg::kTile;
+            uint8_t* vt = kt + Cfg::kStageK;
+            const int nv_raw = d.L - (d.j0 + k) * BS;
+            const int nv = nv_raw < BS ? nv_raw : BS;
+            if (MathT::kZeroMaskedV && nv < BS) {
+                // rows past the context may hold anything (NaN included): clear
+                // them in this head's V tile so that 0 * row stays 0 in the tensor core
+                constexpr int NPANEL = D / 64;
+                const int per_panel = (BS - nv) * 8;  // 16-byte chunks
+                for (int x = lane; x < NPANEL * per_panel; x += 32) {
+                    const int pn = x / per_panel, rem = x - pn * per_panel;
+                    const int t = nv + (rem >> 3), cch = rem & 7;
+                    *reinterpret_cast<uint4*>(vt + pn * Cfg::kPanel + t * 128 + cch * 16) = make_uint4(0, 0, 0, 0);
                 }
-                st.page(pg, pg + Cfg::kTile, nv, lane);
+                __syncwarp();
+                fence_proxy_async_smem();
             }
+            st.page(kt, vt, nv, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[slot]);
         }
-        stage_base += nst;
-        if (warp < nz) {
+        stage_base += uint32_t(d.npg * SPL);
+        if (nz > 0) {
             st.piece_absorb(piece, lane);
-            for (int z = warp + NW; z < nz; z += NW) {  // more key ranges than warps
-                const int64_t idx = (int64_t(z) * p.B + d.b) * p.Hq + int64_t(d.g) * G;
+            for (int z = 1; z < nz; ++z) {
+                const int64_t idx = int64_t(z) * p.B * p.Hq + row;
                 st.absorb(p.prefix_o + idx * D, p.prefix_ml + idx, lane);
             }
         }
 
-        // ---- segment end: combine the NW warp states ----
-        st.finish();
-        float* comb = combbuf;
-        st.deposit(comb + warp * Cfg::kCombFloats, lane);
-        if (!rendezvous()) return;
-
+        // ---- segment end: this warp's (b, g) result ----
         const bool whole = d.k0 == d.k1;
-        // partial slot: the piece of the CTA that owns the segment's first page
-        // goes to slot 1 (it ends that CTA's share), any other piece to slot 0
-        // (it starts its CTA's share): at most one of each per CTA
-        const int my_slot = int(blockIdx.x) == d.k0 ? 1 : 0;
-        if (DUMP) {
-            if (ct == 0) misc->dump_idx = atomicAdd(p.seg_count, 1);
-            if (!rendezvous()) return;
-        }
-        const int dump_idx = DUMP ? misc->dump_idx : 0;
-        for (int o = ct; o < G * D; o += NW * 32) {
-            const int h = o / D, dd = o - h * D;
-            float M = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < NW; ++w) M = fmaxf(M, comb[w * Cfg::kCombFloats + G * D + h]);
-            float lsum = 0.f, a = 0.f;
-#pragma unroll
-            for (int w = 0; w < NW; ++w) {
-                const float* cw = comb + w * Cfg::kCombFloats;
-                const float sc = exp2f(cw[G * D + h] - M);
-                lsum += cw[G * D + G + h] * sc;
-                a += cw[h * D + dd] * sc;
-            }
-            const float val = a / lsum;
-            if (whole) {
-                p.out[(int64_t(d.b) * p.Hq + int64_t(d.g) * G + h) * D + dd] = __float2bfloat16_rn(val);
-            } else {
-                const int64_t ps = int64_t(blockIdx.x) * 2 + my_slot;
-                p.part_o[(ps * G + h) * D + dd] = val;
-                if (dd == 0) p.part_ml[ps * G + h] = make_float2(M, lsum);
-            }
-            if (DUMP && dump_idx < p.dump_capacity) {
-                p.seg_o[(int64_t(dump_idx) * G + h) * D + dd] = val;
-                if (dd == 0) {
-                    p.seg_m[int64_t(dump_idx) * G + h] = M * 0.69314718055994531f;  // base 2 -> natural
-                    p.seg_l[int64_t(dump_idx) * G + h] = lsum;
+        const int nk = d.k1 - d.k0 + 1;
+        const int leaf = int(blockIdx.x) - d.k0;
+        int32_t* top = p.counters + int64_t(d.b) * p.Hkv + g;
+        if (!DUMP && !whole && nk <= kFastMergePieces) {
+            // ticket first; the second piece to finish folds the first one's
+            // published partial into its registers
+            if (ticket(top, nk, lane)) {
+                const int64_t sl = leaf_slot(d.k0, 1 - leaf);
+                const int* flag = p.slot_sync + sl * HG + warp;
+                const uint64_t t0 = globaltimer_ns();
+                for (uint32_t it = 0; ld_acquire_gpu(flag) == 0; ++it) {  // set right after its ticket
+                    __nanosleep(32);
+                    if ((it & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) {
+                        raise_error(PA_DEVERR_TIMEOUT);
+                        break;
+                    }
                 }
-                if (o == 0) {
-                    int32_t* mt = p.seg_meta + int64_t(dump_idx) * 4;
+                __syncwarp();
+                const int64_t ps = sl * hgG + int64_t(warp) * G;
+                st.absorb(p.part_o + ps * D, p.part_ml + ps, lane);
+                st.finish();
+                st.store_out(p.out + row * D, lane);
+                __syncwarp();
+                if (lane == 0) {
+                    p.slot_sync[sl * HG + warp] = 0;
+                    *top = 0;
+                }
+            } else {
+                const int64_t ps = leaf_slot(d.k0, leaf) * hgG + int64_t(warp) * G;
+                st.finish();
+                st.store_partial(p.part_o + ps * D, p.part_ml + ps, nullptr, nullptr, lane);
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) st_release_gpu(p.slot_sync + leaf_slot(d.k0, leaf) * HG + warp, 1);
+            }
+            ++seg_i;
+            continue;
+        }
+        st.finish();
+        if (DUMP) {
+            int di = 0;
+            if (lane == 0) di = atomicAdd(p.seg_count, 1);
+            di = __shfl_sync(0xffffffffu, di, 0);
+            if (di < p.dump_capacity) {
+                st.store_partial(p.seg_o + int64_t(di) * G * D, nullptr, p.seg_m + int64_t(di) * G,
+                                 p.seg_l + int64_t(di) * G, lane);
+                if (lane == 0) {
+                    int32_t* mt = p.seg_meta + int64_t(di) * 4;
                     mt[0] = d.b;
-                    mt[1] = d.g;
+                    mt[1] = g;
                     mt[2] = d.j0 * BS;
                     const int t1 = (d.j0 + d.npg) * BS;
                     mt[3] = t1 < d.L ? t1 : d.L;
                 }
             }
         }
-
         if (whole) {
-            // every warp has read comb before any warp deposits the next segment
-            if (!rendezvous()) return;
+            st.store_out(p.out + row * D, lane);
         } else {
-            // ---- split-KV: the last CTA to finish a piece of (b, g) merges ----
+            // ---- split-KV: the last CTA to finish a piece of (b, g) merges.
+            // Partial slot: the piece of the CTA that owns the segment's first
+            // page goes to slot 1 (it ends that CTA's share), any other piece
+            // to slot 0 (it starts its CTA's share): one of each per CTA. ----
+            const int my_slot = int(blockIdx.x) == d.k0 ? 1 : 0;
+            const int64_t ps = (int64_t(blockIdx.x) * 2 + my_slot) * hgG + int64_t(warp) * G;
+            st.store_partial(p.part_o + ps * D, p.part_ml + ps, nullptr, nullptr, lane);
             __threadfence();
-            if (!rendezvous()) return;
-            if (ct == 0) {
-                const int t = atomicAdd(p.counters + int64_t(d.b) * p.Hkv + d.g, 1);
-                misc->is_last = (t == d.k1 - d.k0);
-            }
-            if (!rendezvous()) return;
-            if (misc->is_last) {
-                __threadfence();
-                // Every piece's (max, sum) goes to shared memory (the combine area
-                // is free again), then each thread merges 4 outputs with float4
-                // loads kept in flight, so the merge costs a few L2 round trips.
-                const int nk = d.k1 - d.k0 + 1;
-                float2* stage = reinterpret_cast<float2*>(comb);
-                const bool staged = nk * G * 2 <= NW * Cfg::kCombFloats;
-                if (staged) {
-                    for (int x = ct; x < nk * G; x += NW * 32) {
-                        const int k = d.k0 + x / G, h = x % G;
-                        const int64_t pk = int64_t(k) * 2 + (k == d.k0 ? 1 : 0);
-                        stage[x] = __ldcg(&p.part_ml[pk * G + h]);
+            __syncwarp();
+            if (nk <= kMergeFanIn) {
+                if (ticket(top, nk, lane)) {
+                    merge_pieces<D, G>(p, d.k0, 0, 1, nk, HG, warp, lane, p.out + row * D);
+                    if (lane == 0) *top = 0;
+                }
+            } else {
+                const int first = leaf - leaf % kMergeFanIn;
+                const int runs = (nk + kMergeFanIn - 1) / kMergeFanIn;
+                const int in_run = nk - first < kMergeFanIn ? nk - first : kMergeFanIn;
+                int32_t* gc = p.slot_sync + (int64_t(d.k0 + first) * 2 + (first == 0 ? 1 : 0)) * HG + warp;
+                if (ticket(gc, in_run, lane)) {
+                    // this run's pieces -> the partial slot of its first piece
+                    merge_pieces<D, G>(p, d.k0, first, 1, in_run, HG, warp, lane, nullptr);
+                    if (lane == 0) *gc = 0;
+                    __threadfence();
+                    __syncwarp();
+                    if (ticket(top, runs, lane)) {
+                        merge_pieces<D, G>(p, d.k0, 0, kMergeFanIn, runs, HG, warp, lane, p.out + row * D);
+                        if (lane == 0) *top = 0;
                     }
                 }
-                if (!rendezvous()) return;
-                for (int o4 = ct; o4 < G * D / 4; o4 += NW * 32) {
-                    const int h = (o4 * 4) / D, dd = o4 * 4 - h * D;
-                    float M = -INFINITY;
-                    for (int kk = 0; kk < nk; ++kk) {
-                        const int k = d.k0 + kk;
-                        const float mk =
-                            staged ? stage[kk * G + h].x
-                                   : __ldcg(&p.part_ml[(int64_t(k) * 2 + (k == d.k0 ? 1 : 0)) * G + h].x);
-                        M = fmaxf(M, mk);
-                    }
-                    float lsum = 0.f;
-                    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-                    for (int kk = 0; kk < nk; ++kk) {
-                        const int k = d.k0 + kk;
-                        const int64_t pk = int64_t(k) * 2 + (k == d.k0 ? 1 : 0);
-                        const float2 ml = staged ? stage[kk * G + h] : __ldcg(&p.part_ml[pk * G + h]);
-                        const float sc = ml.y * exp2f(ml.x - M);
-                        const float4 v = __ldcg(reinterpret_cast<const float4*>(&p.part_o[(pk * G + h) * D + dd]));
-                        lsum += sc;
-                        a.x += sc * v.x;
-                        a.y += sc * v.y;
-                        a.z += sc * v.z;
-                        a.w += sc * v.w;
-                    }
-                    const float inv = 1.f / lsum;
-                    __nv_bfloat16* dst = p.out + (int64_t(d.b) * p.Hq + int64_t(d.g) * G + h) * D + dd;
-                    *reinterpret_cast<uint2*>(dst) =
-                        make_uint2(float2_to_bf16x2(a.x * inv, a.y * inv), float2_to_bf16x2(a.z * inv, a.w * inv));
-                }
-                if (ct == 0) p.counters[int64_t(d.b) * p.Hkv + d.g] = 0;
-                // the staged values are read before the next segment's deposit
-                if (!rendezvous()) return;
             }
         }
         ++seg_i;

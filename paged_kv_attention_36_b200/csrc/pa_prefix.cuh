@@ -15,9 +15,10 @@
 //
 // CTA = (group, row tile, kv head, key range).  Consumer warp w owns rows
 // 16w .. 16w+15 of the tile; warp NW streams the range's pages (K and V
-// tiles of the group's first member's blocks) with tiled TMA, in the
-// 128-byte-swizzled panel layout of the decode, into a ring of RS stages
-// that every consumer warp reads (a stage is free when all have arrived).
+// tiles of the group's first member's blocks, one tiled TMA copy each, in
+// the 128-byte-swizzled panel layout of the decode) into a ring of RS
+// stages that every consumer warp reads (a stage is free when all have
+// arrived).
 //
 // Per page and warp (FlashAttention-2 fragment flow): S[16 x 16] = Q . K^T
 // with K rows from ldmatrix; each row's max over the 4 lanes that hold it;
@@ -76,7 +77,6 @@ template <int D, int G, int NW, int RS>
 __global__ void __launch_bounds__((NW + 1) * 32, 1) prefix_kernel(const __grid_constant__ PrefixParams p) {
     using Cfg = PrefixCfg<D, NW, RS>;
     constexpr int KS = D / 16;
-    constexpr int NPANEL = D / 64;
     static_assert(Cfg::kRows % G == 0, "a tile holds whole members");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -178,13 +178,9 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) prefix_kernel(const __grid_c
                 if (use > 0) lane_ok = mbar_wait(&empty[slot], (use - 1) & 1, abort);
                 if (lane_ok) {
                     uint8_t* st = smem + slot * Cfg::kPage;
-                    const int row = (blk * p.Hkv + g) * 16;
                     mbar_arrive_expect_tx(&full[slot], Cfg::kPage);
-#pragma unroll
-                    for (int pn = 0; pn < NPANEL; ++pn) {
-                        tma_load_3d(st + pn * Cfg::kPanel, &p.tmap_k, 0, pn, row, &full[slot], pol);
-                        tma_load_3d(st + Cfg::kTile + pn * Cfg::kPanel, &p.tmap_v, 0, pn, row, &full[slot], pol);
-                    }
+                    tma_load_4d(st, &p.tmap_k, 0, 0, 0, blk * p.Hkv + g, &full[slot], pol);
+                    tma_load_4d(st + Cfg::kTile, &p.tmap_v, 0, 0, 0, blk * p.Hkv + g, &full[slot], pol);
                 }
             }
             ok = __all_sync(0xffffffffu, lane_ok);

@@ -85,11 +85,13 @@ def test_append_host_validation(binding):
 
 
 def test_workspace_size_formula(binding):
-    # counters (B*Hkv int32) + per-CTA two partial slots (G*D floats + G (m, l) pairs)
+    # counters (B*Hkv int32) + per-CTA two partial slots, each holding the query
+    # heads of one head group (HG = 8 kv heads x G: HG*G*D floats + HG*G (m, l)
+    # pairs) + per-CTA two first-level merge counters per head of the group
     d = _dims(binding, num_seqs=64, num_q_heads=32, num_kv_heads=8, head_dim=128)
     n = binding.pa_decode_workspace_bytes(d, 148)
-    G = 4
-    need = 64 * 8 * 4 + 148 * 2 * G * 128 * 4 + 148 * 2 * G * 8
+    hG = 8 * 4
+    need = 64 * 8 * 4 + 148 * 2 * hG * 128 * 4 + 148 * 2 * hG * 8 + 148 * 2 * 8 * 4
     assert need <= n <= need + 4 * 256  # + alignment and the fused path's grid barrier
     with pytest.raises(ValueError):
         binding.pa_decode_workspace_bytes(_dims(binding, num_kv_heads=3), 148)

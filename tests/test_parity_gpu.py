@@ -125,7 +125,7 @@ def _case(oracle_lib, pa, lens, Hq, Hkv, D, seed, poison=True, num_ctas=None):
     else:
         dims = pa.make_dims(tq, tk, tbt)
         ws = pa.alloc_workspace(dims, num_ctas)
-        cap = 4096
+        cap = 16384
         G = Hq // Hkv
         meta = torch.zeros((cap, 4), dtype=torch.int32, device=d)
         so = torch.zeros((cap, G, D), dtype=torch.float32, device=d)
@@ -216,6 +216,15 @@ def test_forced_splits_partials_and_merge(pa, oracle_lib, num_ctas):
 def test_forced_splits_head_dim_128(pa, oracle_lib, num_ctas):
     lens = [1500, 1, 333, 64]
     _case(oracle_lib, pa, lens, 32, 8, 128, seed=200 + num_ctas, num_ctas=num_ctas)
+
+
+@pytest.mark.parametrize("num_ctas", [17, 600, 1024])
+def test_split_merge_levels(pa, oracle_lib, num_ctas):
+    # one sequence cut into num_ctas pieces: 17 needs the second merge level
+    # by one piece, 600 and 1024 give 38 and 64 runs of 16 (the most the
+    # second level takes)
+    lens = [16 * 1100, 5]
+    _case(oracle_lib, pa, lens, 16, 8, 64, seed=300 + num_ctas, num_ctas=num_ctas)
 
 
 def test_long_single_sequence(pa, oracle_lib):
