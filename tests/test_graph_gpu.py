@@ -1,0 +1,118 @@
+"""CUDA-graph capture of the decode step (the pages' engines replay a
+captured decode to cut launch latency: miniVLLM docs index, "What is
+miniVLLM?": CUDA graph optimization for low-latency decode).
+
+Every C-ABI call is asynchronous, allocates nothing and never synchronises,
+so a whole step can be captured on a torch stream and replayed.  These
+tests capture (1) the fused append + decode (a cooperative launch with a
+grid barrier in the workspace), (2) the shared-prefix step (the prefix pass
+and the decode launched as its programmatic dependent) and (3) the two-call
+step (append, then decode), replay each several times with new inputs
+written into the captured buffers, and compare every replay with the fp64
+oracle.  Replays reuse the workspace, so they also prove that every call
+leaves its counters and barrier at zero.
+"""
+import numpy as np
+import pytest
+import torch
+
+from tests import paging
+
+pytestmark = pytest.mark.gpu
+
+ATOL, RTOL = 1e-2, 1e-2
+
+
+@pytest.fixture(scope="module")
+def pa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from paged_kv_attention_36_b200 import binding
+    binding.pa_device_errors(clear=True)
+    return binding
+
+
+def _close(out, ref):
+    got = out.to(torch.float64).cpu().numpy()
+    assert not np.isnan(got).any()
+    assert (np.abs(got - ref) <= ATOL + RTOL * np.abs(ref)).all(), float(np.abs(got - ref).max())
+
+
+def _oracle(oracle, w, q, k_new, v_new):
+    kb, vb = paging.bits(w.k_cache).copy(), paging.bits(w.v_cache).copy()
+    oracle.append(paging.bits(k_new), paging.bits(v_new), w.slot_mapping.numpy(), kb, vb)
+    return oracle.decode(paging.bits(q), kb, vb, w.block_tables.numpy(), w.context_lens.numpy(), w.scale)
+
+
+def _run(pa, oracle_lib, w, step, replays=3):
+    """Capture `step(t, out)` once, then replay it with fresh q / new rows."""
+    d = torch.device("cuda")
+    t = {k: getattr(w, k).to(d) for k in ("q", "k_cache", "v_cache", "block_tables", "context_lens", "k_new",
+                                          "v_new", "slot_mapping")}
+    if w.num_groups:
+        t["group_offsets"], t["group_prefix_pages"] = w.group_offsets.to(d), w.group_prefix_pages.to(d)
+    out = torch.empty_like(t["q"])
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        step(t, out)  # warm-up outside capture (first-call attribute set-up)
+    torch.cuda.current_stream().wait_stream(stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        step(t, out)
+    gen = torch.Generator().manual_seed(77)
+    for _ in range(replays):
+        q = torch.randn(w.q.shape, generator=gen).to(torch.bfloat16)
+        kn = torch.randn(w.k_new.shape, generator=gen).to(torch.bfloat16)
+        vn = torch.randn(w.v_new.shape, generator=gen).to(torch.bfloat16)
+        t["q"].copy_(q)
+        t["k_new"].copy_(kn)
+        t["v_new"].copy_(vn)
+        g.replay()
+        torch.cuda.synchronize()
+        _close(out, _oracle(oracle_lib, w, q, kn, vn))
+    assert pa.pa_device_errors(clear=True) == 0
+
+
+def test_graph_fused_append_decode(pa, oracle_lib):
+    from paged_kv_attention_36_b200 import workloads
+    w = workloads.make("qwen3", poison=True)
+
+    def step(t, out):
+        dims = pa.make_dims(t["q"], t["k_cache"], t["block_tables"])
+        if not hasattr(step, "ws"):
+            step.ws = pa.alloc_workspace(dims)
+        pa.pa_append_decode(t["k_new"], t["v_new"], t["slot_mapping"], t["q"], t["k_cache"], t["v_cache"],
+                            t["block_tables"], t["context_lens"], w.scale, out, workspace=step.ws)
+    _run(pa, oracle_lib, w, step)
+
+
+def test_graph_two_call_step(pa, oracle_lib):
+    from paged_kv_attention_36_b200 import workloads
+    w = workloads.make("longskew")
+
+    def step(t, out):
+        dims = pa.make_dims(t["q"], t["k_cache"], t["block_tables"])
+        if not hasattr(step, "ws"):
+            step.ws = pa.alloc_workspace(dims)
+        pa.pa_cache_append(t["k_new"], t["v_new"], t["slot_mapping"], t["k_cache"], t["v_cache"])
+        pa.pa_decode(t["q"], t["k_cache"], t["v_cache"], t["block_tables"], t["context_lens"], w.scale, out,
+                     workspace=step.ws)
+    _run(pa, oracle_lib, w, step, replays=2)
+
+
+def test_graph_shared_prefix_step(pa, oracle_lib):
+    from paged_kv_attention_36_b200 import workloads
+    w = workloads.make("prefix", poison=True)
+
+    def step(t, out):
+        dims = pa.make_dims(t["q"], t["k_cache"], t["block_tables"])
+        if not hasattr(step, "ws"):
+            step.ws = torch.zeros(pa.pa_decode_shared_prefix_workspace_bytes(dims, w.num_groups, w.max_group_size),
+                                  dtype=torch.uint8, device="cuda")
+        pa.pa_decode_shared_prefix(t["q"], t["k_cache"], t["v_cache"], t["block_tables"], t["context_lens"],
+                                   w.scale, t["group_offsets"], t["group_prefix_pages"], w.max_group_size, out,
+                                   k_new=t["k_new"], v_new=t["v_new"], slot_mapping=t["slot_mapping"],
+                                   workspace=step.ws)
+    _run(pa, oracle_lib, w, step)
