@@ -58,6 +58,14 @@ def _load():
         lib.pa_oracle_lse_merge.restype = i32
         lib.pa_oracle_append.argtypes = [vp, vp, vp, i64, vp, vp, i64, i64, i64, i64]
         lib.pa_oracle_append.restype = i32
+        lib.pa_oracle_e4m3_encode_array.argtypes = [vp, i64, vp]
+        lib.pa_oracle_e4m3_encode_array.restype = None
+        lib.pa_oracle_e4m3_decode_array.argtypes = [vp, i64, vp]
+        lib.pa_oracle_e4m3_decode_array.restype = None
+        lib.pa_oracle_append_fp8.argtypes = [vp, vp, vp, i64, vp, vp, vp, vp, i64, i64, i64]
+        lib.pa_oracle_append_fp8.restype = i32
+        lib.pa_oracle_decode_fp8.argtypes = [vp] * 7 + [i64] * 6 + [dbl, vp]
+        lib.pa_oracle_decode_fp8.restype = i32
         _lib = lib
     return _lib
 
@@ -157,3 +165,60 @@ def append(k_new, v_new, slot_mapping, k_cache, v_cache) -> None:
     rc = _load().pa_oracle_append(_ptr(k_new), _ptr(v_new), _ptr(slot_mapping), T,
                                   _ptr(k_cache), _ptr(v_cache), Hkv, D, bs, NB)
     _check(rc)
+
+
+# ---------------------------------------------------------------------------
+# fp8 (OCP E4M3) KV cache with per-kv-head scales; layouts in pa_oracle.c.
+
+def e4m3_encode(x) -> np.ndarray:
+    """Nearest E4M3 codes (ties to even, |x| > 448 saturating, NaN -> 0x7F)
+    of float32 values."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.zeros(x.shape, dtype=np.uint8)
+    _load().pa_oracle_e4m3_encode_array(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def e4m3_decode(c) -> np.ndarray:
+    """Values (fp64) of E4M3 codes."""
+    c = np.ascontiguousarray(c, dtype=np.uint8)
+    out = np.zeros(c.shape, dtype=np.float64)
+    _load().pa_oracle_e4m3_decode_array(_ptr(c), c.size, _ptr(out))
+    return out
+
+
+def append_fp8(k_new, v_new, slot_mapping, k_cache8, v_cache8, k_scale, v_scale) -> None:
+    """In place: encode token t's rows as e4m3(x / scale[g]) into slot
+    slot_mapping[t] (>= 0) of the fp8 caches: k_cache8 [NB][Hkv][16][D],
+    v_cache8 [NB][Hkv][D][16] (tokens in the transposed tile order)."""
+    k_new, v_new, slot_mapping = _u16(k_new), _u16(v_new), _i32(slot_mapping)
+    for c in (k_cache8, v_cache8):
+        if not (isinstance(c, np.ndarray) and c.dtype == np.uint8 and c.flags.c_contiguous):
+            raise TypeError("fp8 caches must be C-contiguous uint8 numpy arrays")
+    NB, Hkv, bs, D = k_cache8.shape
+    if bs != 16 or v_cache8.shape != (NB, Hkv, D, 16):
+        raise ValueError("fp8 caches are [NB][Hkv][16][D] and [NB][Hkv][D][16]")
+    ks = np.ascontiguousarray(k_scale, dtype=np.float32)
+    vs = np.ascontiguousarray(v_scale, dtype=np.float32)
+    T = slot_mapping.shape[0]
+    _check(_load().pa_oracle_append_fp8(_ptr(k_new), _ptr(v_new), _ptr(slot_mapping), T, _ptr(k_cache8),
+                                        _ptr(v_cache8), _ptr(ks), _ptr(vs), Hkv, D, NB))
+
+
+def decode_fp8(q, k_cache8, v_cache8, k_scale, v_scale, block_tables, context_lens, scale: float) -> np.ndarray:
+    """The decode over the dequantized fp8 caches (values e4m3(c) * scale[g]); fp64 [B][Hq][D]."""
+    q = _u16(q)
+    k8 = np.ascontiguousarray(k_cache8, dtype=np.uint8)
+    v8 = np.ascontiguousarray(v_cache8, dtype=np.uint8)
+    block_tables, context_lens = _i32(block_tables), _i32(context_lens)
+    B, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k8.shape
+    if D2 != D or bs != 16 or v8.shape != (NB, Hkv, D, 16) or block_tables.shape[0] != B:
+        raise ValueError("shape mismatch")
+    ks = np.ascontiguousarray(k_scale, dtype=np.float32)
+    vs = np.ascontiguousarray(v_scale, dtype=np.float32)
+    out = np.zeros((B, Hq, D), dtype=np.float64)
+    _check(_load().pa_oracle_decode_fp8(_ptr(q), _ptr(k8), _ptr(v8), _ptr(ks), _ptr(vs), _ptr(block_tables),
+                                        _ptr(context_lens), B, Hq, Hkv, D, NB, block_tables.shape[1],
+                                        float(scale), _ptr(out)))
+    return out

@@ -33,6 +33,20 @@
  * the documented layout): k_cache and v_cache are [NB][Hkv][bs][D] bf16,
  * row-major; block_tables is [B][M] int32; q and out are [B][Hq][D].
  *
+ * fp8 KV cache (the pages' quantization theme applied to the KV cache:
+ * MiniVLLM write-up, "量化层" and "量化支持"): each cached value is one
+ * OCP FP8 E4M3 code c (the "fn" variant: 4 exponent bits with bias 7, 3
+ * mantissa bits, no infinities, 0x7F/0xFF NaN, largest finite 448) with a
+ * per-kv-head scale, value = e4m3(c) * scale[g].  The append encodes
+ * x / scale[g] (one IEEE binary32 division of the widened bf16 value) by
+ * rounding to the nearest representable value, ties to even, and
+ * saturating magnitudes beyond 448 to 448.  Layouts (uint8):
+ *   k_cache8 [NB][Hkv][16][D]   token-major, like the bf16 cache;
+ *   v_cache8 [NB][Hkv][D][16]   each (block, head) tile transposed: row d
+ *                               holds the 16 tokens' values of column d at
+ *                               position pos(t) = 4*((t % 8) / 2) + 2*(t / 8) + t % 2.
+ * The fp8 decode is the formula above with K_t, V_t the dequantized values.
+ *
  * Parity pins: tests/test_oracle_pins.py checks every function here
  * against torch's scaled_dot_product_attention on contiguous K/V, block
  * permutation and block-size invariance, the closed forms for
@@ -266,5 +280,145 @@ int pa_oracle_append(const uint16_t *k_new, const uint16_t *v_new, const int32_t
             }
         }
     }
+    return rc;
+}
+
+/* ---------------------------------------------------------------------
+ * OCP FP8 E4M3 ("fn": no infinities, NaN = 0x7F / 0xFF, max finite 448).
+ * Normal codes: (1 + m/8) * 2^(e-7), e = 1..15 (e = 15, m = 7 is NaN);
+ * subnormal codes (e = 0): (m/8) * 2^-6.
+ * ------------------------------------------------------------------- */
+double pa_oracle_e4m3_decode(uint8_t c)
+{
+    const int e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return NAN;
+    const double mag = e == 0 ? ldexp((double)m, -9) : ldexp(8.0 + m, e - 10);
+    return (c & 0x80) ? -mag : mag;
+}
+
+/* Round half to even of a non-negative double to an integer (exact). */
+static double round_half_even(double v)
+{
+    double f = floor(v);
+    double r = v - f;
+    if (r > 0.5) return f + 1.0;
+    if (r < 0.5) return f;
+    return fmod(f, 2.0) == 0.0 ? f : f + 1.0;
+}
+
+/* Nearest E4M3 code to x (ties to even), |x| beyond 448 saturating to 448,
+ * NaN to 0x7F. */
+uint8_t pa_oracle_e4m3_encode(float x)
+{
+    if (isnan(x)) return 0x7F;
+    const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    if (a == 0.0) return sign;
+    if (a >= 448.0) return sign | 0x7E;
+    int ex;
+    frexp(a, &ex);                 /* a = f * 2^ex, f in [0.5, 1) */
+    int E = ex - 1;                /* a in [2^E, 2^(E+1)) */
+    if (E < -6) {                  /* subnormal range: multiples of 2^-9 */
+        double n = round_half_even(ldexp(a, 9));
+        if (n >= 8.0) return sign | 0x08;          /* rounded up to 2^-6 */
+        return sign | (uint8_t)n;
+    }
+    double n = round_half_even(ldexp(a, 3 - E)); /* in [8, 16] */
+    if (n == 16.0) { n = 8.0; E += 1; }
+    if (E > 8 || (E == 8 && n > 14.0)) return sign | 0x7E;  /* beyond 448 */
+    return sign | (uint8_t)(((E + 7) << 3) | ((int)n - 8));
+}
+
+void pa_oracle_e4m3_encode_array(const float *x, int64_t n, uint8_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = pa_oracle_e4m3_encode(x[i]);
+}
+
+void pa_oracle_e4m3_decode_array(const uint8_t *c, int64_t n, double *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = pa_oracle_e4m3_decode(c[i]);
+}
+
+static int64_t vt_pos(int64_t t) { return 4 * ((t % 8) / 2) + 2 * (t / 8) + t % 2; }
+
+/* Slot-mapped append into the fp8 caches (block size 16): the row of token
+ * t, kv head g is encoded as e4m3(x / scale[g]). */
+int pa_oracle_append_fp8(const uint16_t *k_new, const uint16_t *v_new, const int32_t *slot_mapping,
+                         int64_t T, uint8_t *k_cache, uint8_t *v_cache, const float *k_scale,
+                         const float *v_scale, int64_t Hkv, int64_t D, int64_t NB)
+{
+    const int64_t bs = 16;
+    if (T < 0 || Hkv <= 0 || D <= 0 || NB < 0) return PAO_ERR_ARG;
+    if (T > 0 && (!k_new || !v_new || !slot_mapping || !k_cache || !v_cache || !k_scale || !v_scale))
+        return PAO_ERR_ARG;
+    int rc = PAO_OK;
+    for (int64_t t = 0; t < T; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        int64_t block = slot / bs, offset = slot % bs;
+        if (block >= NB) { rc = PAO_ERR_SLOT; continue; }
+        for (int64_t g = 0; g < Hkv; ++g) {
+            int64_t src = (t * Hkv + g) * D;
+            int64_t tile = block * Hkv + g;
+            for (int64_t d = 0; d < D; ++d) {
+                float kx = (float)bf16_bits_to_double(k_new[src + d]);
+                float vx = (float)bf16_bits_to_double(v_new[src + d]);
+                k_cache[(tile * bs + offset) * D + d] = pa_oracle_e4m3_encode(kx / k_scale[g]);
+                v_cache[(tile * D + d) * bs + vt_pos(offset)] = pa_oracle_e4m3_encode(vx / v_scale[g]);
+            }
+        }
+    }
+    return rc;
+}
+
+/* fp8 decode, same formula as pa_oracle_decode on the dequantized values. */
+int pa_oracle_decode_fp8(const uint16_t *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                         const float *k_scale, const float *v_scale,
+                         const int32_t *block_tables, const int32_t *context_lens,
+                         int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t NB, int64_t M,
+                         double scale, double *out)
+{
+    const int64_t bs = 16;
+    if (!q || !k_cache || !v_cache || !k_scale || !v_scale || !block_tables || !context_lens || !out)
+        return PAO_ERR_ARG;
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || NB < 0 || M < 0 || Hq % Hkv != 0) return PAO_ERR_ARG;
+    const int64_t G = Hq / Hkv;
+    double *s_buf = (double *)malloc(sizeof(double) * (size_t)(M * bs > 0 ? M * bs : 1));
+    if (!s_buf) return PAO_ERR_NOMEM;
+    int rc = PAO_OK;
+    for (int64_t b = 0; b < B && rc == PAO_OK; ++b) {
+        const int64_t L = context_lens[b];
+        if (L < 0 || L > M * bs) { rc = PAO_ERR_LEN; break; }
+        for (int64_t h = 0; h < Hq && rc == PAO_OK; ++h) {
+            const int64_t g = h / G;
+            const uint16_t *qr = q + (b * Hq + h) * D;
+            double *o = out + (b * Hq + h) * D;
+            for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
+            if (L == 0) continue;
+            double mx = -INFINITY;
+            for (int64_t t = 0; t < L; ++t) {
+                int64_t block = block_tables[b * M + t / bs];
+                if (block < 0 || block >= NB) { rc = PAO_ERR_BLOCK; break; }
+                const uint8_t *k = k_cache + ((block * Hkv + g) * bs + t % bs) * D;
+                double dot = 0.0;
+                for (int64_t d = 0; d < D; ++d)
+                    dot += bf16_bits_to_double(qr[d]) * (pa_oracle_e4m3_decode(k[d]) * (double)k_scale[g]);
+                s_buf[t] = scale * dot;
+                if (s_buf[t] > mx) mx = s_buf[t];
+            }
+            if (rc != PAO_OK) break;
+            double l = 0.0;
+            for (int64_t t = 0; t < L; ++t) {
+                int64_t block = block_tables[b * M + t / bs];
+                const uint8_t *vt = v_cache + (block * Hkv + g) * D * bs;
+                double w = exp(s_buf[t] - mx);
+                l += w;
+                for (int64_t d = 0; d < D; ++d)
+                    o[d] += w * (pa_oracle_e4m3_decode(vt[d * bs + vt_pos(t % bs)]) * (double)v_scale[g]);
+            }
+            for (int64_t d = 0; d < D; ++d) o[d] /= l;
+        }
+    }
+    free(s_buf);
     return rc;
 }
