@@ -6,6 +6,7 @@ merge included).  Prints ONE JSON line on rank 0.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama32]
     python bench.py --impl reference ...   # the fp64 CPU oracle, timed on host cores
+    python bench.py --kv fp8 ...           # fp8 (E4M3) caches: append_fp8 + decode_fp8
 
 Metric: effective GB/s = algorithmic bytes / device time, where the
 algorithmic bytes of a step are the distinct K/V rows the decode must read
@@ -53,6 +54,8 @@ def _args():
     ap.add_argument("--workload", default="llama32",
                     choices=["tiny", "qwen3", "llama32", "longskew", "prefix"])
     ap.add_argument("--impl", default="pa", choices=["pa", "reference"])
+    ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8"],
+                    help="cache format: bf16, or fp8 E4M3 codes with per-kv-head scales")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -199,6 +202,52 @@ def cpu_baseline(w, dec_bytes: int, app_bytes: int, budget_s: float = 12.0):
                       f"{per_step * 1e3:.1f} ms each, fp64, {nthreads} threads"}
 
 
+def _fp8_scales(Hkv: int):
+    """The benchmark's per-kv-head K and V scales of the fp8 caches (an input
+    choice: they keep N(0,1) values and the x8 outliers inside E4M3's range)."""
+    g = torch.arange(Hkv, dtype=torch.float32)
+    return (g + 4) / 32, (g + 3) / 24
+
+
+def _fp8_step_bytes(w):
+    """Algorithmic bytes of one fp8 step: half the bf16 K/V bytes (one byte
+    per value) + q/out; the append reads bf16 rows and writes fp8 ones."""
+    from paged_kv_attention_36_b200 import workloads
+    dec = workloads.unique_kv_bytes(w) // 2 + workloads.qo_bytes(w)
+    n_valid = int((w.slot_mapping >= 0).sum().item())
+    per_tok = w.k_new.shape[1] * w.k_new.shape[2]
+    app = n_valid * per_tok * (2 * 2 + 2 * 1) + 4 * w.slot_mapping.numel()
+    return dec, app
+
+
+def _pool_rows(cache):
+    """[NB][Hkv][16][D] bf16 pool -> [NB*16][Hkv][D] rows, one per slot."""
+    NB, Hkv, bs, D = cache.shape
+    return cache.permute(0, 2, 1, 3).reshape(NB * bs, Hkv, D).contiguous()
+
+
+def run_reference_fp8(args, w):
+    import numpy as np
+    import oracle
+    from tests import paging
+    dec, app = _fp8_step_bytes(w)
+    nthreads = oracle.default_threads()
+    NB, Hkv, _, D = w.k_cache.shape
+    ks, vs = (t.numpy() for t in _fp8_scales(Hkv))
+    k8 = np.zeros((NB, Hkv, 16, D), np.uint8)
+    v8 = np.zeros((NB, Hkv, D, 16), np.uint8)
+    oracle.append_fp8(paging.bits(_pool_rows(w.k_cache)), paging.bits(_pool_rows(w.v_cache)),
+                      np.arange(NB * 16, dtype=np.int32), k8, v8, ks, vs)
+    qb = paging.bits(w.q)
+    bt, cl = w.block_tables.numpy(), w.context_lens.numpy()
+    kn, vn, sm = paging.bits(w.k_new), paging.bits(w.v_new), w.slot_mapping.numpy()
+
+    def step():
+        oracle.append_fp8(kn, vn, sm, k8, v8, ks, vs)
+        oracle.decode_fp8(qb, k8, v8, ks, vs, bt, cl, w.scale, nthreads=nthreads)
+    return step, dec, app, nthreads
+
+
 def run_reference(args, ws, rank):
     """--impl reference: the fp64 oracle on the host cores, rank 0 only."""
     if rank != 0:
@@ -207,16 +256,19 @@ def run_reference(args, ws, rank):
     import oracle
     from tests import paging
     w = workloads.make(args.workload)
-    dec, app = _step_bytes(w)
-    nthreads = oracle.default_threads()
-    kb, vb = paging.bits(w.k_cache).copy(), paging.bits(w.v_cache).copy()
-    qb = paging.bits(w.q)
-    bt, cl = w.block_tables.numpy(), w.context_lens.numpy()
-    kn, vn, sm = paging.bits(w.k_new), paging.bits(w.v_new), w.slot_mapping.numpy()
+    if args.kv == "fp8":
+        step, dec, app, nthreads = run_reference_fp8(args, w)
+    else:
+        dec, app = _step_bytes(w)
+        nthreads = oracle.default_threads()
+        kb, vb = paging.bits(w.k_cache).copy(), paging.bits(w.v_cache).copy()
+        qb = paging.bits(w.q)
+        bt, cl = w.block_tables.numpy(), w.context_lens.numpy()
+        kn, vn, sm = paging.bits(w.k_new), paging.bits(w.v_new), w.slot_mapping.numpy()
 
-    def step():
-        oracle.append(kn, vn, sm, kb, vb)
-        oracle.decode(qb, kb, vb, bt, cl, w.scale, nthreads=nthreads)
+        def step():
+            oracle.append(kn, vn, sm, kb, vb)
+            oracle.decode(qb, kb, vb, bt, cl, w.scale, nthreads=nthreads)
 
     for _ in range(args.warmup):
         step()
@@ -231,7 +283,7 @@ def run_reference(args, ws, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(per * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "description": w.spec.description},
+        "config": {"workload": args.workload, "description": w.spec.description, "kv": args.kv},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": nthreads, "kind": "oracle",
                          "sample": f"{args.steps} full steps of the '{args.workload}' batch"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -439,6 +491,148 @@ def run_pa(args, ws, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_pa_fp8(args, ws, rank, local):
+    """The fp8 step: pa_cache_append_fp8 then pa_decode_fp8 (two launches)."""
+    from paged_kv_attention_36_b200 import binding as pa
+    from paged_kv_attention_36_b200 import workloads
+
+    dev = torch.device("cuda", local if ws > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+    w = workloads.make(args.workload)
+    dec_bytes, app_bytes = _fp8_step_bytes(w)
+    step_bytes = dec_bytes + app_bytes
+    NB, Hkv, _, D = w.k_cache.shape
+    ks, vs = (t.to(dev) for t in _fp8_scales(Hkv))
+    # the fp8 pool: every slot of the bf16 pool encoded once (set-up, not timed)
+    k8 = torch.empty((NB, Hkv, 16, D), dtype=torch.uint8, device=dev)
+    v8 = torch.empty((NB, Hkv, D, 16), dtype=torch.uint8, device=dev)
+    pa.pa_cache_append_fp8(_pool_rows(w.k_cache).to(dev), _pool_rows(w.v_cache).to(dev),
+                           torch.arange(NB * 16, dtype=torch.int32, device=dev), k8, v8, ks, vs)
+    torch.cuda.synchronize(dev)
+    pool_bytes = 2 * k8.numel()
+    rotate = pool_bytes >= ROTATE_MIN_POOL
+    ncopies = max(2, -(-ROTATE_BYTES // pool_bytes)) if rotate else 1
+    caches = [(k8.clone(), v8.clone()) for _ in range(ncopies)]
+    del k8, v8
+    q, bt, cl = w.q.to(dev), w.block_tables.to(dev), w.context_lens.to(dev)
+    kn, vn, sm = w.k_new.to(dev), w.v_new.to(dev), w.slot_mapping.to(dev)
+    out = torch.empty_like(q)
+    dims = pa.pa_dims(q.shape[0], q.shape[1], Hkv, D, 16, NB, bt.shape[1])
+    wsp = pa.alloc_workspace(dims, device=dev)
+    flush = None if rotate else torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    app = [pa.prepare_append_fp8(kn, vn, sm, kc, vc, ks, vs, stream=stream) for kc, vc in caches]
+    dec = [pa.prepare_decode_fp8(q, kc, vc, ks, vs, bt, cl, w.scale, out, wsp, stream=stream) for kc, vc in caches]
+
+    def between():
+        if flush is not None:
+            flush.zero_()
+
+    W_ = max(3, args.warmup)
+    for k in range(W_):
+        app[k % ncopies]()
+        dec[k % ncopies]()
+        between()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    clocks = ClockSampler(dev.index, enabled=not args.no_clocks)
+    _barrier(ws)
+    torch.cuda.synchronize(dev)
+    for k in range(K):
+        c = k % ncopies
+        ev[k][0].record(stream)
+        app[c]()
+        ev[k][1].record(stream)
+        dec[c]()
+        ev[k][2].record(stream)
+        between()
+    torch.cuda.synchronize(dev)
+    _barrier(ws)
+    errs = pa.pa_device_errors(clear=True)
+    if errs:
+        raise RuntimeError(f"device error bits {errs:#x} during the benchmark")
+    total_ms = _max_over_ranks(sum(ev[k][0].elapsed_time(ev[k][2]) for k in range(K)), ws)
+    app_avg = _max_over_ranks(sum(ev[k][0].elapsed_time(ev[k][1]) for k in range(K)) / K, ws)
+    dec_avg = _max_over_ranks(sum(ev[k][1].elapsed_time(ev[k][2]) for k in range(K)) / K, ws)
+
+    host = {n: t.pin_memory() for n, t in (("q", w.q), ("bt", w.block_tables), ("cl", w.context_lens),
+                                            ("kn", w.k_new), ("vn", w.v_new), ("sm", w.slot_mapping))}
+    out_h = torch.empty(w.q.shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+    dev_in = {"q": q, "bt": bt, "cl": cl, "kn": kn, "vn": vn, "sm": sm}
+
+    def e2e_step(c):
+        for n, t in host.items():
+            dev_in[n].copy_(t, non_blocking=True)
+        app[c]()
+        dec[c]()
+        out_h.copy_(out, non_blocking=True)
+
+    for k in range(3):
+        e2e_step(k % ncopies)
+        between()
+    torch.cuda.synchronize(dev)
+    ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    _barrier(ws)
+    torch.cuda.synchronize(dev)
+    for k in range(K):
+        ee[k][0].record(stream)
+        e2e_step(k % ncopies)
+        ee[k][1].record(stream)
+        between()
+    torch.cuda.synchronize(dev)
+    _barrier(ws)
+    clk = clocks.stop()
+    e2e_total = _max_over_ranks(sum(ee[k][0].elapsed_time(ee[k][1]) for k in range(K)), ws)
+    if rank != 0:
+        return
+    peak, peak_kind = _peaks()
+    step_avg = total_ms / K
+    achieved = dec_bytes / (dec_avg * 1e-3) / 1e9
+    value = ws * K * step_bytes / (total_ms * 1e-3) / 1e9
+    l2 = (f"inputs larger than L2: {ncopies} copies of the {pool_bytes / 1e6:.0f} MB fp8 cache rotated, "
+          f"no flush" if rotate else "flushed between steps (256 MB write, outside the timed events)")
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": ws, "steps": K, "warmup": W_,
+        "ms_per_step": round(step_avg, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "storage_dtype": "e4m3", "data": "synthetic",
+        "config": {"workload": args.workload, "description": w.spec.description, "kv": "fp8-e4m3",
+                   "num_seqs": w.spec.num_seqs, "q_heads": w.spec.num_q_heads, "kv_heads": w.spec.num_kv_heads,
+                   "head_dim": w.spec.head_dim, "block_size": 16,
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU", "l2": l2,
+                   "unique_kv_bytes": workloads.unique_kv_bytes(w) // 2},
+        "step_us": round(step_avg * 1e3, 2),
+        "decode_us": round(dec_avg * 1e3, 2),
+        "append_us": round(app_avg * 1e3, 2),
+        "decode_only_gbs": round(achieved, 1),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                     "kernel": "pa::decode_kernel<..., Fp8MmaMath> (pa_decode_fp8)",
+                     "traffic": _traffic(args.workload + ":fp8"),
+                     "algorithmic_bytes_per_launch": dec_bytes},
+        "e2e": {"value": round(ws * K * step_bytes / (e2e_total * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_total / K, 5)},
+        "gpu_launches": 2 * K,
+        "clocks": clk,
+    }
+    if ws == 1 and not args.no_cpu_baseline:
+        step, cdec, capp, nthreads = run_reference_fp8(args, w)
+        n, t0 = 0, time.perf_counter()
+        while True:
+            step()
+            n += 1
+            el = time.perf_counter() - t0
+            if el >= 12.0 or n >= 50:
+                break
+        line["cpu_baseline"] = {"value": round((cdec + capp) / (el / n) / 1e9, 4), "unit": "GB/s",
+                                "cores": nthreads, "kind": "oracle",
+                                "sample": f"{n} full fp8 steps (append + decode) of the '{w.spec.name}' batch, "
+                                          f"{el / n * 1e3:.1f} ms each, fp64, {nthreads} threads"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = _args()
     ws, rank, local = _dist()
@@ -448,7 +642,10 @@ def main():
         else:
             if not torch.cuda.is_available():
                 raise SystemExit("bench.py needs a CUDA device for --impl pa")
-            run_pa(args, ws, rank, local)
+            if args.kv == "fp8":
+                run_pa_fp8(args, ws, rank, local)
+            else:
+                run_pa(args, ws, rank, local)
     finally:
         if ws > 1:
             import torch.distributed as dist

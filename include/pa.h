@@ -256,6 +256,36 @@ PA_API pa_status pa_decode_shared_prefix(const void* k_new, const void* v_new, c
                                          void* stream);
 
 /*
+ * fp8 KV cache (OCP FP8 E4M3 codes with one scale per kv head for K and one
+ * for V; the pages' quantization theme applied to the KV cache, MiniVLLM
+ * write-up, "量化层" / "量化支持").  A cached value is e4m3(code) * scale[g]:
+ *   k_cache [NB][Hkv][16][D] uint8   token-major, as the bf16 cache;
+ *   v_cache [NB][Hkv][D][16] uint8   each (block, kv head) tile transposed:
+ *            row d holds the 16 tokens' codes of column d, token t at byte
+ *            4*((t % 8) / 2) + 2*(t / 8) + t % 2 of the row;
+ *   k_scale, v_scale [Hkv] float32 (device).  block_size must be 16.
+ * Half the bytes of the bf16 cache per token; the decode is the formula at
+ * the top of this file on the dequantized values.
+ *
+ * pa_cache_append_fp8: the slot-mapped append (as pa_cache_append) of bf16
+ * rows, each value encoded as the E4M3 code nearest to x / scale[g] (an
+ * IEEE fp32 division; ties to even; magnitudes beyond 448 saturate to 448).
+ * D must be a multiple of 8.
+ *
+ * pa_decode_fp8: pa_decode over fp8 caches (tensor-core policy; head_dim 64
+ * or 128, Hq/Hkv in {1, 2, 4, 8}).  q is bf16 and is converted to f16 for
+ * the products, so |q| must stay below 65504; softmax state and sums are
+ * fp32.  Workspace as for pa_decode (pa_decode_workspace_bytes).
+ */
+PA_API pa_status pa_cache_append_fp8(const void* k_new, const void* v_new, const int32_t* slot_mapping,
+                                     int32_t num_tokens, void* k_cache, void* v_cache, const float* k_scale,
+                                     const float* v_scale, const pa_dims* dims, void* stream);
+PA_API pa_status pa_decode_fp8(const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
+                               const float* v_scale, const int32_t* block_tables, const int32_t* context_lens,
+                               float scale, void* out, const pa_dims* dims, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/*
  * Reads (and, if `clear` != 0, resets) the device error word of the
  * current device.  Synchronous: waits for all prior work on the device.
  */

@@ -64,7 +64,7 @@ def _load():
         lib.pa_oracle_e4m3_decode_array.restype = None
         lib.pa_oracle_append_fp8.argtypes = [vp, vp, vp, i64, vp, vp, vp, vp, i64, i64, i64]
         lib.pa_oracle_append_fp8.restype = i32
-        lib.pa_oracle_decode_fp8.argtypes = [vp] * 7 + [i64] * 6 + [dbl, vp]
+        lib.pa_oracle_decode_fp8.argtypes = [vp] * 7 + [i64] * 6 + [dbl, vp, i32]
         lib.pa_oracle_decode_fp8.restype = i32
         _lib = lib
     return _lib
@@ -205,7 +205,8 @@ def append_fp8(k_new, v_new, slot_mapping, k_cache8, v_cache8, k_scale, v_scale)
                                         _ptr(v_cache8), _ptr(ks), _ptr(vs), Hkv, D, NB))
 
 
-def decode_fp8(q, k_cache8, v_cache8, k_scale, v_scale, block_tables, context_lens, scale: float) -> np.ndarray:
+def decode_fp8(q, k_cache8, v_cache8, k_scale, v_scale, block_tables, context_lens, scale: float,
+               nthreads: int | None = None) -> np.ndarray:
     """The decode over the dequantized fp8 caches (values e4m3(c) * scale[g]); fp64 [B][Hq][D]."""
     q = _u16(q)
     k8 = np.ascontiguousarray(k_cache8, dtype=np.uint8)
@@ -220,5 +221,5 @@ def decode_fp8(q, k_cache8, v_cache8, k_scale, v_scale, block_tables, context_le
     out = np.zeros((B, Hq, D), dtype=np.float64)
     _check(_load().pa_oracle_decode_fp8(_ptr(q), _ptr(k8), _ptr(v8), _ptr(ks), _ptr(vs), _ptr(block_tables),
                                         _ptr(context_lens), B, Hq, Hkv, D, NB, block_tables.shape[1],
-                                        float(scale), _ptr(out)))
+                                        float(scale), _ptr(out), int(nthreads or default_threads())))
     return out

@@ -371,54 +371,89 @@ int pa_oracle_append_fp8(const uint16_t *k_new, const uint16_t *v_new, const int
     return rc;
 }
 
-/* fp8 decode, same formula as pa_oracle_decode on the dequantized values. */
+/* fp8 decode, same formula as pa_oracle_decode on the dequantized values
+ * (codes looked up in a table built from pa_oracle_e4m3_decode), threaded
+ * over (b, h) rows. */
+typedef struct {
+    const uint16_t *q;
+    const uint8_t *k_cache, *v_cache;
+    const float *k_scale, *v_scale;
+    const int32_t *block_tables, *context_lens;
+    int64_t B, Hq, Hkv, D, NB, M;
+    double scale;
+    const double *table;
+    double *out;
+    int64_t first, stride;
+    int status;
+} fp8_job_t;
+
+static void *decode_fp8_worker(void *arg)
+{
+    fp8_job_t *j = (fp8_job_t *)arg;
+    const int64_t bs = 16, G = j->Hq / j->Hkv, D = j->D;
+    double *s_buf = (double *)malloc(sizeof(double) * (size_t)(j->M * bs > 0 ? j->M * bs : 1));
+    if (!s_buf) { j->status = PAO_ERR_NOMEM; return NULL; }
+    j->status = PAO_OK;
+    for (int64_t row = j->first; row < j->B * j->Hq; row += j->stride) {
+        const int64_t b = row / j->Hq, h = row % j->Hq, g = h / G;
+        const int64_t L = j->context_lens[b];
+        const uint16_t *qr = j->q + row * D;
+        double *o = j->out + row * D;
+        for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
+        if (L == 0) continue;
+        const double ks = (double)j->k_scale[g], vs = (double)j->v_scale[g];
+        double mx = -INFINITY;
+        for (int64_t t = 0; t < L; ++t) {
+            const int64_t block = j->block_tables[b * j->M + t / bs];
+            if (block < 0 || block >= j->NB) { j->status = PAO_ERR_BLOCK; break; }
+            const uint8_t *k = j->k_cache + ((block * j->Hkv + g) * bs + t % bs) * D;
+            double dot = 0.0;
+            for (int64_t d = 0; d < D; ++d) dot += bf16_bits_to_double(qr[d]) * (j->table[k[d]] * ks);
+            s_buf[t] = j->scale * dot;
+            if (s_buf[t] > mx) mx = s_buf[t];
+        }
+        if (j->status != PAO_OK) break;
+        double l = 0.0;
+        for (int64_t t = 0; t < L; ++t) {
+            const int64_t block = j->block_tables[b * j->M + t / bs];
+            const uint8_t *vt = j->v_cache + (block * j->Hkv + g) * D * bs;
+            const double w = exp(s_buf[t] - mx);
+            l += w;
+            const int64_t pos = vt_pos(t % bs);
+            for (int64_t d = 0; d < D; ++d) o[d] += w * (j->table[vt[d * bs + pos]] * vs);
+        }
+        for (int64_t d = 0; d < D; ++d) o[d] /= l;
+    }
+    free(s_buf);
+    return NULL;
+}
+
 int pa_oracle_decode_fp8(const uint16_t *q, const uint8_t *k_cache, const uint8_t *v_cache,
                          const float *k_scale, const float *v_scale,
                          const int32_t *block_tables, const int32_t *context_lens,
                          int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t NB, int64_t M,
-                         double scale, double *out)
+                         double scale, double *out, int nthreads)
 {
-    const int64_t bs = 16;
     if (!q || !k_cache || !v_cache || !k_scale || !v_scale || !block_tables || !context_lens || !out)
         return PAO_ERR_ARG;
     if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || NB < 0 || M < 0 || Hq % Hkv != 0) return PAO_ERR_ARG;
-    const int64_t G = Hq / Hkv;
-    double *s_buf = (double *)malloc(sizeof(double) * (size_t)(M * bs > 0 ? M * bs : 1));
-    if (!s_buf) return PAO_ERR_NOMEM;
-    int rc = PAO_OK;
-    for (int64_t b = 0; b < B && rc == PAO_OK; ++b) {
-        const int64_t L = context_lens[b];
-        if (L < 0 || L > M * bs) { rc = PAO_ERR_LEN; break; }
-        for (int64_t h = 0; h < Hq && rc == PAO_OK; ++h) {
-            const int64_t g = h / G;
-            const uint16_t *qr = q + (b * Hq + h) * D;
-            double *o = out + (b * Hq + h) * D;
-            for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
-            if (L == 0) continue;
-            double mx = -INFINITY;
-            for (int64_t t = 0; t < L; ++t) {
-                int64_t block = block_tables[b * M + t / bs];
-                if (block < 0 || block >= NB) { rc = PAO_ERR_BLOCK; break; }
-                const uint8_t *k = k_cache + ((block * Hkv + g) * bs + t % bs) * D;
-                double dot = 0.0;
-                for (int64_t d = 0; d < D; ++d)
-                    dot += bf16_bits_to_double(qr[d]) * (pa_oracle_e4m3_decode(k[d]) * (double)k_scale[g]);
-                s_buf[t] = scale * dot;
-                if (s_buf[t] > mx) mx = s_buf[t];
-            }
-            if (rc != PAO_OK) break;
-            double l = 0.0;
-            for (int64_t t = 0; t < L; ++t) {
-                int64_t block = block_tables[b * M + t / bs];
-                const uint8_t *vt = v_cache + (block * Hkv + g) * D * bs;
-                double w = exp(s_buf[t] - mx);
-                l += w;
-                for (int64_t d = 0; d < D; ++d)
-                    o[d] += w * (pa_oracle_e4m3_decode(vt[d * bs + vt_pos(t % bs)]) * (double)v_scale[g]);
-            }
-            for (int64_t d = 0; d < D; ++d) o[d] /= l;
-        }
+    for (int64_t b = 0; b < B; ++b)
+        if (context_lens[b] < 0 || context_lens[b] > M * 16) return PAO_ERR_LEN;
+    double table[256];
+    for (int c = 0; c < 256; ++c) table[c] = pa_oracle_e4m3_decode((uint8_t)c);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    pthread_t tid[256];
+    fp8_job_t jobs[256];
+    for (int i = 0; i < nthreads; ++i) {
+        jobs[i] = (fp8_job_t){q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                              B, Hq, Hkv, D, NB, M, scale, table, out, i, nthreads, PAO_OK};
+        if (nthreads == 1) decode_fp8_worker(&jobs[i]);
+        else pthread_create(&tid[i], NULL, decode_fp8_worker, &jobs[i]);
     }
-    free(s_buf);
-    return rc;
+    if (nthreads > 1)
+        for (int i = 0; i < nthreads; ++i) pthread_join(tid[i], NULL);
+    for (int i = 0; i < nthreads; ++i)
+        if (jobs[i].status != PAO_OK) return jobs[i].status;
+    return PAO_OK;
 }

@@ -65,6 +65,10 @@ def _load(path: str = LIB_PATH):
     lib.pa_decode_shared_prefix.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, f32, vp, vp, i32, i32,
                                             vp, dp, vp, sz, vp]
     lib.pa_decode_shared_prefix.restype = i32
+    lib.pa_cache_append_fp8.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, dp, vp]
+    lib.pa_cache_append_fp8.restype = i32
+    lib.pa_decode_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, f32, vp, dp, vp, sz, vp]
+    lib.pa_decode_fp8.restype = i32
     lib.pa_decode_static_ws.argtypes = [vp, vp, vp, vp, vp, f32, vp, dp, vp]
     lib.pa_decode_static_ws.restype = i32
     lib.pa_device_errors.argtypes = [ctypes.POINTER(i32), i32]
@@ -79,8 +83,8 @@ lib = _load()
 # Every symbol include/pa.h declares.
 EXPORTS = ("pa_cache_append", "pa_decode_workspace_bytes", "pa_decode_default_ctas", "pa_decode",
            "pa_append_decode", "pa_decode_partials", "pa_decode_static_ws",
-           "pa_decode_shared_prefix_workspace_bytes", "pa_decode_shared_prefix", "pa_device_errors",
-           "pa_status_string")
+           "pa_decode_shared_prefix_workspace_bytes", "pa_decode_shared_prefix", "pa_cache_append_fp8",
+           "pa_decode_fp8", "pa_device_errors", "pa_status_string")
 
 PA_ERR_SCRATCH_LIMIT = -7
 PA_STATIC_SCRATCH_BYTES = 4 << 20  # include/pa.h
@@ -324,6 +328,84 @@ def prepare_decode_shared_prefix(q, k_cache, v_cache, block_tables, context_lens
                                      max_group_size, out, workspace, stream)
     p = Prepared(lib.pa_decode_shared_prefix, args, "pa_decode_shared_prefix")
     p._keep = keep
+    return p
+
+
+# ---- fp8 (E4M3) caches -------------------------------------------------------
+
+def _fp8_cache_args(k_cache8, v_cache8, k_scale, v_scale):
+    _need(k_cache8, torch.uint8, "k_cache", 4)
+    _need(v_cache8, torch.uint8, "v_cache", 4)
+    NB, Hkv, bs, D = k_cache8.shape
+    if bs != 16 or tuple(v_cache8.shape) != (NB, Hkv, D, 16):
+        raise ValueError("fp8 caches are k [NB][Hkv][16][D] and v [NB][Hkv][D][16] (uint8)")
+    for t, n in ((k_scale, "k_scale"), (v_scale, "v_scale")):
+        _need(t, torch.float32, n, 1)
+        if t.shape[0] != Hkv:
+            raise ValueError(f"{n} must have one scale per kv head")
+    return NB, Hkv, D
+
+
+def pa_cache_append_fp8(k_new, v_new, slot_mapping, k_cache8, v_cache8, k_scale, v_scale, stream=None) -> None:
+    """Encode each new bf16 row as E4M3 codes of x / scale[kv head] into its
+    slot of the fp8 caches (see include/pa.h for the layouts)."""
+    NB, Hkv, D = _fp8_cache_args(k_cache8, v_cache8, k_scale, v_scale)
+    for t, n in ((k_new, "k_new"), (v_new, "v_new")):
+        _need(t, torch.bfloat16, n, 3)
+    _need(slot_mapping, torch.int32, "slot_mapping", 1)
+    T = slot_mapping.shape[0]
+    if k_new.shape != v_new.shape or k_new.shape[0] != T or k_new.shape[1:] != (Hkv, D):
+        raise ValueError("k_new/v_new must be [T][Hkv][D] of the cache")
+    dims = pa_dims(0, Hkv, Hkv, D, 16, NB, 0)
+    _check(lib.pa_cache_append_fp8(_ptr(k_new), _ptr(v_new), _ptr(slot_mapping), T, _ptr(k_cache8),
+                                   _ptr(v_cache8), _ptr(k_scale), _ptr(v_scale), ctypes.byref(dims),
+                                   _stream(stream)), "pa_cache_append_fp8")
+
+
+def _decode_fp8_args(q, k_cache8, v_cache8, k_scale, v_scale, block_tables, context_lens, out):
+    NB, Hkv, D = _fp8_cache_args(k_cache8, v_cache8, k_scale, v_scale)
+    _need(q, torch.bfloat16, "q", 3)
+    _need(out, torch.bfloat16, "out", 3)
+    _need(block_tables, torch.int32, "block_tables", 2)
+    _need(context_lens, torch.int32, "context_lens", 1)
+    B, Hq, D2 = q.shape
+    if D2 != D or out.shape != q.shape or block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise ValueError("decode shapes disagree")
+    return pa_dims(B, Hq, Hkv, D, 16, NB, block_tables.shape[1])
+
+
+def pa_decode_fp8(q, k_cache8, v_cache8, k_scale, v_scale, block_tables, context_lens, scale: float, out,
+                  workspace=None, stream=None) -> None:
+    """Paged decode over fp8 (E4M3) caches with per-kv-head scales."""
+    dims = _decode_fp8_args(q, k_cache8, v_cache8, k_scale, v_scale, block_tables, context_lens, out)
+    if workspace is None:
+        workspace = alloc_workspace(dims, device=q.device)
+    _need(workspace, torch.uint8, "workspace", 1)
+    _check(lib.pa_decode_fp8(_ptr(q), _ptr(k_cache8), _ptr(v_cache8), _ptr(k_scale), _ptr(v_scale),
+                             _ptr(block_tables), _ptr(context_lens), float(scale), _ptr(out), ctypes.byref(dims),
+                             _ptr(workspace), workspace.numel(), _stream(stream)), "pa_decode_fp8")
+
+
+def prepare_append_fp8(k_new, v_new, slot_mapping, k_cache8, v_cache8, k_scale, v_scale, stream=None) -> "Prepared":
+    NB, Hkv, D = _fp8_cache_args(k_cache8, v_cache8, k_scale, v_scale)
+    dims = pa_dims(0, Hkv, Hkv, D, 16, NB, 0)
+    p = Prepared(lib.pa_cache_append_fp8,
+                 (_ptr(k_new), _ptr(v_new), _ptr(slot_mapping), slot_mapping.shape[0], _ptr(k_cache8),
+                  _ptr(v_cache8), _ptr(k_scale), _ptr(v_scale), ctypes.byref(dims), _stream(stream)),
+                 "pa_cache_append_fp8")
+    p._keep = (dims, k_new, v_new, slot_mapping, k_cache8, v_cache8, k_scale, v_scale)
+    return p
+
+
+def prepare_decode_fp8(q, k_cache8, v_cache8, k_scale, v_scale, block_tables, context_lens, scale: float, out,
+                       workspace, stream=None) -> "Prepared":
+    dims = _decode_fp8_args(q, k_cache8, v_cache8, k_scale, v_scale, block_tables, context_lens, out)
+    _need(workspace, torch.uint8, "workspace", 1)
+    p = Prepared(lib.pa_decode_fp8,
+                 (_ptr(q), _ptr(k_cache8), _ptr(v_cache8), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+                  _ptr(context_lens), float(scale), _ptr(out), ctypes.byref(dims), _ptr(workspace),
+                  workspace.numel(), _stream(stream)), "pa_decode_fp8")
+    p._keep = (dims, q, k_cache8, v_cache8, k_scale, v_scale, block_tables, context_lens, out, workspace)
     return p
 
 

@@ -26,8 +26,9 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
-// The math policies: tensor-core (default) or fp32 CUDA-core.
-enum class MathKind { kMma, kSimt };
+// The math policies: tensor-core (default) or fp32 CUDA-core for bf16
+// caches; tensor-core for fp8 (E4M3) caches.
+enum class MathKind { kMma, kSimt, kFp8 };
 
 #ifndef PA_MAX_RING
 #define PA_MAX_RING 64
@@ -35,9 +36,9 @@ enum class MathKind { kMma, kSimt };
 // Deepest ring of stages whose CTA fits in shared memory, a multiple of
 // the most stages a page can take (with 32 KB stages: 7 at head_dim 64,
 // 6 at 128).
-template <int D>
+template <int D, int EB = 2>
 constexpr int ring_fit() {
-    using C1 = pa::DecodeCfg<D, kBlockSize, 1>;
+    using C1 = pa::DecodeCfg<D, kBlockSize, 1, EB>;
     int r = PA_MAX_RING;
     while (r > 1 && C1::kSmemBytes + (r - 1) * (C1::kStage + 16) > 232448) --r;
     r -= r % C1::kMaxSpl;
@@ -47,22 +48,22 @@ constexpr int ring_fit() {
 // Fixed cost of finishing a segment, expressed as K+V bytes that could be
 // streamed meanwhile, in pages of `heads` kv heads (rounded down);
 // PA_SEG_WEIGHT_BYTES overrides it.
-int32_t seg_weight_pages(int head_dim, int heads) {
+int32_t seg_weight_pages(int head_dim, int heads, int eb) {
     static const long long bytes = [] {
         const char* e = std::getenv("PA_SEG_WEIGHT_BYTES");
         return e ? std::atoll(e) : 32768LL;
     }();
-    const long long page = 2LL * kBlockSize * head_dim * 2 * heads;
+    const long long page = 2LL * kBlockSize * head_dim * eb * heads;
     return int32_t(bytes / page);
 }
 
-// kv heads per ring stage: as many whole K+V tiles as a stage holds.
-int heads_per_stage_max(int D) { return PA_STAGE_K_BYTES / (kBlockSize * D * 2); }
+// kv heads per ring stage: as many whole K+V tiles (eb bytes per value) as a stage holds.
+int heads_per_stage_max(int D, int eb) { return PA_STAGE_K_BYTES / (kBlockSize * D * eb); }
 
 // kv heads per head group: the largest divisor of Hkv that is at most 8
 // (one consumer warp per head) and splits into 1, 2, 4 or 8 equal stages.
-int heads_per_group(int Hkv, int D) {
-    const int hs = heads_per_stage_max(D);
+int heads_per_group(int Hkv, int D, int eb) {
+    const int hs = heads_per_stage_max(D, eb);
     for (int h = pa::kDecodeWarps; h > 1; --h) {
         if (Hkv % h) continue;
         for (int spl = 1; spl <= pa::kDecodeWarps; spl *= 2)
@@ -82,7 +83,7 @@ MathKind math_kind() {
 bool supported(int D, int G, MathKind mk) {
     if (D != 64 && D != 128) return false;
     if (G != 1 && G != 2 && G != 4 && G != 8) return false;
-    return mk == MathKind::kMma || G * D <= 256;
+    return mk != MathKind::kSimt || G * D <= 256;
 }
 
 std::mutex g_mu;
@@ -114,14 +115,15 @@ struct WsLayout {
 };
 
 WsLayout ws_layout(const pa_dims& d, int grid) {
-    const size_t hG = size_t(heads_per_group(d.num_kv_heads, d.head_dim)) * (d.num_q_heads / d.num_kv_heads);
+    // partial slots hold the query heads of one head group, at most min(Hkv, 8) kv heads (any cache format)
+    const size_t hg_max = size_t(d.num_kv_heads < pa::kDecodeWarps ? d.num_kv_heads : pa::kDecodeWarps);
+    const size_t hG = hg_max * (d.num_q_heads / d.num_kv_heads);
     WsLayout w;
     w.counters = 0;
     w.part_o = align_up(size_t(d.num_seqs) * d.num_kv_heads * 4, 256);
     w.part_ml = align_up(w.part_o + size_t(grid) * 2 * hG * d.head_dim * 4, 256);
     w.slot_sync = align_up(w.part_ml + size_t(grid) * 2 * hG * 8, 256);
-    w.grid_bar = align_up(w.slot_sync + size_t(grid) * 2 * heads_per_group(d.num_kv_heads, d.head_dim) * 4,
-                          256);
+    w.grid_bar = align_up(w.slot_sync + size_t(grid) * 2 * hg_max * 4, 256);
     w.total = w.grid_bar + 256;
     return w;
 }
@@ -180,15 +182,37 @@ bool make_cache_map(CUtensorMap* map, const void* base, int64_t tiles, int D, in
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// An fp8 cache seen as a 4-D uint8 tensor {128 bytes, D/8 lines, 1, NB*Hkv
+// tiles} (rank 4 like the bf16 maps, so that the decode's 4-D tiled load
+// {0, 0, 0, tile} serves both): one (block, kv head) tile is 16*D bytes =
+// D/8 lines of 128 bytes (K: 16 tokens of D codes; V: D rows of 16 tokens).
+// One box is `heads` consecutive tiles whole.  K takes the 128-byte swizzle
+// (a line holds one token at head_dim 128, two at 64); V^T rows are 16
+// bytes and need none.
+bool make_fp8_map(CUtensorMap* map, const void* base, int64_t tiles, int D, int heads, bool swizzle) {
+    auto fn = encode_tiled();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {128, cuuint64_t(D / 8), 1, cuuint64_t(tiles)};
+    cuuint64_t strides[3] = {128, cuuint64_t(16) * D, cuuint64_t(16) * D};
+    cuuint32_t box[4] = {128, cuuint32_t(D / 8), 1, cuuint32_t(heads)};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+              PA_L2_PROMOTION, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // pdl: launched as a programmatic dependent of the kernel before it in the
 // stream (prefix_kernel), so that its set-up overlaps that kernel's end.
 template <MathKind MK, int D, int G, bool DUMP, bool APPEND>
 pa_status launch_decode(const pa::DecodeParams& p, int grid, cudaStream_t stream, bool pdl) {
-    constexpr int R = ring_fit<D>();
-    using Cfg = pa::DecodeCfg<D, kBlockSize, R>;
+    constexpr int EB = MK == MathKind::kFp8 ? 1 : 2;
+    constexpr int R = ring_fit<D, EB>();
+    using Cfg = pa::DecodeCfg<D, kBlockSize, R, EB>;
     auto kern = [] {
         if constexpr (MK == MathKind::kMma)
             return pa::decode_kernel<D, G, kBlockSize, R, DUMP, APPEND, pa::MmaMath>;
+        else if constexpr (MK == MathKind::kFp8)
+            return pa::decode_kernel<D, G, kBlockSize, R, DUMP, APPEND, pa::Fp8MmaMath>;
         else
             return pa::decode_kernel<D, G, kBlockSize, R, DUMP, APPEND, pa::SimtMath>;
     }();
@@ -228,7 +252,9 @@ pa_status launch_decode(const pa::DecodeParams& p, int grid, cudaStream_t stream
 // The SIMT policy is built only for G*D <= 256 (its per-lane state grows with G*D).
 template <MathKind MK, int D, int G, bool DUMP, bool APPEND>
 pa_status launch_built(const pa::DecodeParams& p, int grid, cudaStream_t s, bool pdl) {
-    if constexpr (MK == MathKind::kMma || G * D <= 256)
+    if constexpr (MK == MathKind::kFp8 && (DUMP || APPEND))
+        return PA_ERR_UNSUPPORTED;  // fp8: the plain decode only
+    else if constexpr (MK != MathKind::kSimt || G * D <= 256)
         return launch_decode<MK, D, G, DUMP, APPEND>(p, grid, s, pdl);
     else
         return PA_ERR_UNSUPPORTED;
@@ -325,12 +351,13 @@ pa_status dispatch_prefix(int D, int G, const pa::PrefixParams& p, dim3 grid, cu
 // Shared validation of pa_decode and pa_decode_partials; fills p.
 pa_status prepare_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
                          const int32_t* context_lens, float scale, void* out, const pa_dims* dims, int grid,
-                         void* workspace, size_t workspace_bytes, pa::DecodeParams& p) {
+                         void* workspace, size_t workspace_bytes, pa::DecodeParams& p, int eb = 2) {
     if (!dims) return PA_ERR_NULL;
     if (!dims_ok(dims)) return PA_ERR_SHAPE;
     const pa_dims& d = *dims;
     const int G = d.num_q_heads / d.num_kv_heads;
-    if (d.block_size != kBlockSize || !supported(d.head_dim, G, math_kind())) return PA_ERR_UNSUPPORTED;
+    if (d.block_size != kBlockSize || !supported(d.head_dim, G, eb == 1 ? MathKind::kFp8 : math_kind()))
+        return PA_ERR_UNSUPPORTED;
     if (d.num_seqs == 0) return PA_OK;
     // at least one block, so that a bad block id can be redirected to block 0
     if (d.num_blocks == 0) return PA_ERR_SHAPE;
@@ -346,14 +373,17 @@ pa_status prepare_decode(const void* q, const void* k_cache, const void* v_cache
     p = pa::DecodeParams{};
     const int64_t rows = int64_t(d.num_blocks) * d.num_kv_heads * d.block_size;
     if (rows >= (int64_t(1) << 31)) return PA_ERR_SHAPE;  // TMA coordinates are int32
-    const int HG = heads_per_group(d.num_kv_heads, d.head_dim);
+    const int HG = heads_per_group(d.num_kv_heads, d.head_dim, eb);
     int SPL = 1;
-    while (HG / SPL > heads_per_stage_max(d.head_dim) || HG % SPL) SPL *= 2;
+    while (HG / SPL > heads_per_stage_max(d.head_dim, eb) || HG % SPL) SPL *= 2;
     const int HS = HG / SPL;
     const int64_t tiles = int64_t(d.num_blocks) * d.num_kv_heads;
-    if (!make_cache_map(&p.tmap_k, k_cache, tiles, d.head_dim, d.block_size, HS) ||
-        !make_cache_map(&p.tmap_v, v_cache, tiles, d.head_dim, d.block_size, HS))
-        return PA_ERR_CUDA;
+    const bool maps_ok =
+        eb == 2 ? make_cache_map(&p.tmap_k, k_cache, tiles, d.head_dim, d.block_size, HS) &&
+                      make_cache_map(&p.tmap_v, v_cache, tiles, d.head_dim, d.block_size, HS)
+                : make_fp8_map(&p.tmap_k, k_cache, tiles, d.head_dim, HS, true) &&
+                      make_fp8_map(&p.tmap_v, v_cache, tiles, d.head_dim, HS, false);
+    if (!maps_ok) return PA_ERR_CUDA;
     p.q = static_cast<const uint8_t*>(q);
     p.block_tables = block_tables;
     p.context_lens = context_lens;
@@ -370,7 +400,7 @@ pa_status prepare_decode(const void* q, const void* k_cache, const void* v_cache
     p.SPL = SPL;
     p.SPL_LOG = SPL == 1 ? 0 : SPL == 2 ? 1 : SPL == 4 ? 2 : 3;
     p.min_pages = kMinPagesPerCta;
-    p.seg_weight = seg_weight_pages(d.head_dim, HG);
+    p.seg_weight = seg_weight_pages(d.head_dim, HG, eb);
     p.counters = reinterpret_cast<int32_t*>(ws + w.counters);
     p.part_o = reinterpret_cast<float*>(ws + w.part_o);
     p.part_ml = reinterpret_cast<float2*>(ws + w.part_ml);
@@ -639,6 +669,53 @@ pa_status pa_decode_static_ws(const void* q, const void* k_cache, const void* v_
         cudaMemsetAsync(p.slot_sync, 0, w.grid_bar - w.slot_sync, s) != cudaSuccess)
         return PA_ERR_CUDA;
     return dispatch_decode<false>(dims->head_dim, dims->num_q_heads / dims->num_kv_heads, p, grid, s);
+}
+
+pa_status pa_cache_append_fp8(const void* k_new, const void* v_new, const int32_t* slot_mapping, int32_t num_tokens,
+                              void* k_cache, void* v_cache, const float* k_scale, const float* v_scale,
+                              const pa_dims* dims, void* stream) {
+    if (!dims) return PA_ERR_NULL;
+    const pa_dims& d = *dims;
+    if (num_tokens < 0 || d.num_kv_heads <= 0 || d.head_dim <= 0 || d.block_size <= 0 || d.num_blocks < 0)
+        return PA_ERR_SHAPE;
+    if (d.block_size != kBlockSize || d.head_dim % 8 != 0) return PA_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return PA_OK;
+    if (!k_new || !v_new || !slot_mapping || !k_cache || !v_cache || !k_scale || !v_scale) return PA_ERR_NULL;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned4(slot_mapping) || !aligned4(k_scale) || !aligned4(v_scale))
+        return PA_ERR_ALIGN;
+    pa::AppendFp8Params p;
+    p.k_new = static_cast<const uint4*>(k_new);
+    p.v_new = static_cast<const uint4*>(v_new);
+    p.slot_mapping = slot_mapping;
+    p.k_cache = static_cast<uint8_t*>(k_cache);
+    p.v_cache = static_cast<uint8_t*>(v_cache);
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.chunks_per_row = d.head_dim / 8;
+    p.num_chunks = int64_t(num_tokens) * d.num_kv_heads * p.chunks_per_row;
+    p.kv_heads = d.num_kv_heads;
+    p.num_blocks = d.num_blocks;
+    const int64_t blocks = (p.num_chunks + pa::kAppendThreads - 1) / pa::kAppendThreads;
+    if (blocks > 0x7fffffff) return PA_ERR_SHAPE;
+    pa::append_fp8_kernel<<<unsigned(blocks), pa::kAppendThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_decode_fp8(const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
+                        const float* v_scale, const int32_t* block_tables, const int32_t* context_lens, float scale,
+                        void* out, const pa_dims* dims, void* workspace, size_t workspace_bytes, void* stream) {
+    pa::DecodeParams p;
+    const int grid = sm_count();
+    const pa_status st = prepare_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, dims, grid,
+                                        workspace, workspace_bytes, p, /*eb=*/1);
+    if (st != PA_OK || dims->num_seqs == 0) return st;
+    if (!k_scale || !v_scale) return PA_ERR_NULL;
+    if (!aligned4(k_scale) || !aligned4(v_scale)) return PA_ERR_ALIGN;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    return dispatch_d_g<MathKind::kFp8, false, false>(dims->head_dim, dims->num_q_heads / dims->num_kv_heads, p,
+                                                      grid, static_cast<cudaStream_t>(stream), false);
 }
 
 pa_status pa_device_errors(int32_t* errors_out, int32_t clear) {

@@ -49,4 +49,68 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendParams p) 
     p.v_cache[dst] = vv;
 }
 
+// ---- fp8 (E4M3) caches --------------------------------------------------------
+// k_cache8 [NB][Hkv][16][D] (token-major) and v_cache8 [NB][Hkv][D][16]: each
+// (block, kv head) V tile is stored transposed, row d holding the 16 tokens'
+// column-d codes, token t at position 4*((t % 8) / 2) + 2*(t / 8) + t % 2.  This
+// order lets the decode's tensor-core fragments of V^T come from a plain
+// ldmatrix of 8-byte groups (two tokens t, t+1 then t+8, t+9 per 4 bytes).
+// Codes are e4m3(x / scale[g]): fp32 division, nearest code, ties to even,
+// saturating at +-448.
+struct AppendFp8Params {
+    const uint4* k_new;           // [T][Hkv][D] bf16, 16-byte chunks
+    const uint4* v_new;
+    const int32_t* slot_mapping;  // [T]
+    uint8_t* k_cache;             // [NB][Hkv][16][D] e4m3
+    uint8_t* v_cache;             // [NB][Hkv][D][16] e4m3
+    const float* k_scale;         // [Hkv]
+    const float* v_scale;         // [Hkv]
+    int64_t num_chunks;           // T * Hkv * D / 8
+    int32_t chunks_per_row;       // D / 8
+    int32_t kv_heads;
+    int32_t num_blocks;
+};
+
+__device__ __forceinline__ int vt_position(int t) { return 4 * ((t & 7) >> 1) + 2 * (t >> 3) + (t & 1); }
+
+__global__ void __launch_bounds__(kAppendThreads) append_fp8_kernel(AppendFp8Params p) {
+    const int64_t idx = int64_t(blockIdx.x) * kAppendThreads + threadIdx.x;
+    if (idx >= p.num_chunks) return;
+    const int64_t per_token = int64_t(p.kv_heads) * p.chunks_per_row;
+    const int64_t t = idx / per_token;
+    const int64_t rem = idx - t * per_token;
+    const int32_t slot = __ldg(p.slot_mapping + t);
+    if (slot < 0) return;
+    const int64_t block = slot >> 4;
+    const int offset = slot & 15;
+    if (block >= p.num_blocks) {
+        if (rem == 0) raise_error(PA_DEVERR_SLOT);
+        return;
+    }
+    const int g = int(rem / p.chunks_per_row);
+    const int c = int(rem - int64_t(g) * p.chunks_per_row);
+    const int D = p.chunks_per_row * 8;
+    const int64_t tile = block * p.kv_heads + g;
+    const float ks = __ldg(p.k_scale + g), vs = __ldg(p.v_scale + g);
+    const uint4 kv = __ldg(p.k_new + idx), vv = __ldg(p.v_new + idx);
+    const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w}, vw[4] = {vv.x, vv.y, vv.z, vv.w};
+    uint16_t k8[4], v8[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 kf = bf16x2_to_float2(kw[j]), vf = bf16x2_to_float2(vw[j]);
+        k8[j] = f32x2_to_e4m3x2(__fdiv_rn(kf.x, ks), __fdiv_rn(kf.y, ks));
+        v8[j] = f32x2_to_e4m3x2(__fdiv_rn(vf.x, vs), __fdiv_rn(vf.y, vs));
+    }
+    // K: 8 consecutive codes of row `offset`
+    *reinterpret_cast<uint2*>(p.k_cache + (tile * 16 + offset) * D + c * 8) =
+        make_uint2(uint32_t(k8[0]) | (uint32_t(k8[1]) << 16), uint32_t(k8[2]) | (uint32_t(k8[3]) << 16));
+    // V: one code in each of the rows c*8 .. c*8+7 of the transposed tile
+    uint8_t* vrow = p.v_cache + (tile * D + c * 8) * 16 + vt_position(offset);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        vrow[(2 * j) * 16] = uint8_t(v8[j] & 0xff);
+        vrow[(2 * j + 1) * 16] = uint8_t(v8[j] >> 8);
+    }
+}
+
 }  // namespace pa

@@ -108,6 +108,9 @@ struct DecodeParams {
     int32_t prefix_splits;              // key ranges of the prefix partials
     const float* prefix_o;              // [splits][B][Hq][D]
     const float2* prefix_ml;            // [splits][B][Hq] (max logit base 2, exp-sum)
+    // fp8 caches: value = e4m3 code * scale[kv head] (null for bf16 caches)
+    const float* k_scale;               // [Hkv]
+    const float* v_scale;               // [Hkv]
 };
 
 // One segment of a CTA's share, handed from the producer to the consumers.
@@ -151,10 +154,12 @@ struct SimtMath {
     static constexpr bool kZeroMaskedV = false;  // masked rows are skipped
     static_assert(D % 64 == 0 && BS % 4 == 0, "layout");
 
+    static constexpr int kElemBytes = 2;  // bf16 caches
     float2 q2[G][NCH][4];
     float2 acc[G][NCH][4];
     float m[G];
     float l[G];
+    float oscale = 1.f;  // output scale (1 for bf16 caches)
 
     // q of the G query heads of one kv head (G rows of D bf16, global
     // memory), pre-scaled by scale * log2(e).
@@ -330,7 +335,7 @@ struct SimtMath {
         if (tg != 0) return;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-            const float inv = 1.f / l[h];
+            const float inv = oscale / l[h];
 #pragma unroll
             for (int i = 0; i < NCH; ++i) {
                 uint4 v;
@@ -384,10 +389,12 @@ struct MmaMath {
     static constexpr int KS = D / 16;  // k-steps of Q.K = m-tiles of O^T
     static constexpr bool kZeroMaskedV = true;  // 0 * NaN would poison the mma
 
+    static constexpr int kElemBytes = 2;  // bf16 caches
     uint32_t qb[KS][2];  // Q^T as B fragments (bf16 pairs)
     float acc[KS][4];    // O^T accumulator tiles
     float m[2], l[2];    // heads h0, h0 + 1 of this lane (l: this lane's rows only)
     float qscale;
+    float oscale = 1.f;  // output scale (1 for bf16 caches)
 
     // q of the G query heads of one kv head (G rows of D bf16, global
     // memory) as B fragments; the logits are scaled by scale * log2(e) later.
@@ -537,7 +544,7 @@ struct MmaMath {
         for (int e = 0; e < 2; ++e) {
             const int h = h0 + e;
             if (h >= G) continue;
-            const float inv = 1.f / l[e];
+            const float inv = oscale / l[e];
 #pragma unroll
             for (int mt = 0; mt < KS; ++mt) {
                 out[h * D + 16 * mt + d0] = __float2bfloat16_rn(acc[mt][e] * inv);
@@ -573,13 +580,132 @@ struct MmaMath {
 };
 
 // ===========================================================================
+// fp8 (E4M3) caches on the tensor cores.  K tiles arrive as [16 tokens][D]
+// codes in 128-byte lines (128-byte swizzle; at head_dim 64 a line holds two
+// tokens), V tiles transposed as [D][16] codes in 16-byte rows with the
+// token order of pa_append.cuh.  A plain ldmatrix of 8 rows x 16 bytes gives
+// each lane 4 consecutive codes of one row; each half converts exactly to an
+// f16x2.  With Q^T's d order permuted the same way (k slots 2c, 2c+1 <- d
+// 4c, 4c+1 and 2c+8, 2c+9 <- d 4c+2, 4c+3 within each 16) the K fragments
+// feed mma.sync m16n8k16 (f16 in, fp32 accumulate); for V^T the stored
+// token order makes the same conversion give tokens 2c, 2c+1, 2c+8, 2c+9,
+// the natural fragment order, so P^T is the bf16 policy's, in f16.  Tokens
+// past the context are zeroed in the V^T fragments (0 * NaN would poison
+// the sum).  The kv head's K scale is folded into qscale and its V scale
+// into oscale; the state, merges and outputs are MmaMath's.
+template <int D, int G, int BS>
+struct Fp8MmaMath : MmaMath<D, G, BS> {
+    using Base = MmaMath<D, G, BS>;
+    using Base::KS;
+    using Base::qb;
+    using Base::acc;
+    using Base::m;
+    using Base::l;
+    using Base::qscale;
+    static constexpr bool kZeroMaskedV = false;  // masked in the fragments
+    static constexpr int kElemBytes = 1;
+    static_assert(D == 64 || D == 128, "128-byte K lines hold one or two tokens");
+
+    __device__ __forceinline__ void load_q_global(const uint8_t* gq, int lane, float qs_scale) {
+        qscale = qs_scale;
+        const int h = lane >> 2, c = lane & 3;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            if (h < G) {
+                const uint2 w = __ldg(reinterpret_cast<const uint2*>(gq + (h * D + 16 * ks + 4 * c) * 2));
+                const float2 a = bf16x2_to_float2(w.x), b = bf16x2_to_float2(w.y);
+                qb[ks][0] = float2_to_f16x2(a.x, a.y);
+                qb[ks][1] = float2_to_f16x2(b.x, b.y);
+            } else {
+                qb[ks][0] = qb[ks][1] = 0u;
+            }
+        }
+    }
+
+    // Byte offset of 16-byte chunk ch (d 16ch .. 16ch+15) of token t in a K tile.
+    static __device__ __forceinline__ int k_off(int t, int ch) {
+        const int line = D == 128 ? t : (t >> 1);
+        const int lch = D == 128 ? ch : (((t & 1) << 2) + ch);
+        return (line << 7) + ((lch ^ (line & 7)) << 4);
+    }
+    static __device__ __forceinline__ uint32_t lo(uint32_t r) { return e4m3x2_to_f16x2(uint16_t(r & 0xffffu)); }
+    static __device__ __forceinline__ uint32_t hi(uint32_t r) { return e4m3x2_to_f16x2(uint16_t(r >> 16)); }
+
+    __device__ __forceinline__ void page(const uint8_t* kt, const uint8_t* vt, int nvalid, int lane) {
+        const int mi = lane >> 3, r8 = lane & 7, c = lane & 3;
+        // ---- S^T = K . Q^T, two k-steps per ldmatrix ----
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+            const int t = r8 + ((mi & 1) << 3);
+#pragma unroll
+            for (int j = 0; j < KS / 2; ++j) {
+                uint32_t r[4];
+                ldmatrix_x4(r, kt + k_off(t, 2 * j + (mi >> 1)));
+                const uint32_t a0[4] = {lo(r[0]), lo(r[1]), hi(r[0]), hi(r[1])};
+                mma_f16_16816(s, a0, qb[2 * j][0], qb[2 * j][1]);
+                const uint32_t a1[4] = {lo(r[2]), lo(r[3]), hi(r[2]), hi(r[3])};
+                mma_f16_16816(s, a1, qb[2 * j + 1][0], qb[2 * j + 1][1]);
+            }
+        }
+        const int t0 = lane >> 2;
+        const bool v0 = t0 < nvalid, v1 = (t0 + 8) < nvalid;
+        s[0] = v0 ? s[0] * qscale : -INFINITY;
+        s[1] = v0 ? s[1] * qscale : -INFINITY;
+        s[2] = v1 ? s[2] * qscale : -INFINITY;
+        s[3] = v1 ? s[3] * qscale : -INFINITY;
+        // ---- online softmax over the 16 tokens of each head column ----
+        float mx0 = fmaxf(s[0], s[2]), mx1 = fmaxf(s[1], s[3]);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+        }
+        if (__any_sync(0xffffffffu, mx0 > m[0] || mx1 > m[1])) {
+            const float n0 = fmaxf(m[0], mx0), n1 = fmaxf(m[1], mx1);
+            const float a0 = exp2f(m[0] - n0), a1 = exp2f(m[1] - n1);
+            m[0] = n0;
+            m[1] = n1;
+            l[0] *= a0;
+            l[1] *= a1;
+#pragma unroll
+            for (int i = 0; i < KS; ++i) {
+                acc[i][0] *= a0;
+                acc[i][1] *= a1;
+                acc[i][2] *= a0;
+                acc[i][3] *= a1;
+            }
+        }
+        const float p0 = exp2f(s[0] - m[0]), p1 = exp2f(s[1] - m[1]);
+        const float p2 = exp2f(s[2] - m[0]), p3 = exp2f(s[3] - m[1]);
+        l[0] += p0 + p2;
+        l[1] += p1 + p3;
+        // ---- P^T as f16 B fragments ----
+        const uint32_t b0 = movmatrix_trans(float2_to_f16x2(p0, p1));
+        const uint32_t b1 = movmatrix_trans(float2_to_f16x2(p2, p3));
+        // ---- O^T += V^T . P^T, two m-tiles (32 rows of V^T) per ldmatrix;
+        // this lane's tokens: 2c, 2c+1 (low halves) and 2c+8, 2c+9 (high) ----
+        const uint32_t mlo = (2 * c < nvalid ? 0x0000ffffu : 0u) | (2 * c + 1 < nvalid ? 0xffff0000u : 0u);
+        const uint32_t mhi = (2 * c + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * c + 9 < nvalid ? 0xffff0000u : 0u);
+#pragma unroll
+        for (int j = 0; j < KS / 2; ++j) {
+            uint32_t r[4];
+            ldmatrix_x4(r, vt + (32 * j + lane) * 16);
+            const uint32_t a0[4] = {lo(r[0]) & mlo, lo(r[1]) & mlo, hi(r[0]) & mhi, hi(r[1]) & mhi};
+            mma_f16_16816(acc[2 * j], a0, b0, b1);
+            const uint32_t a1[4] = {lo(r[2]) & mlo, lo(r[3]) & mlo, hi(r[2]) & mhi, hi(r[3]) & mhi};
+            mma_f16_16816(acc[2 * j + 1], a1, b0, b1);
+        }
+    }
+};
+
+// ===========================================================================
 // Consumer warps of a decode CTA: warp w < HG owns kv head hg*HG + w.
 constexpr int kDecodeWarps = 8;
 
-template <int D, int BS, int R>
+template <int D, int BS, int R, int EB = 2>
 struct DecodeCfg {
     static constexpr int NW = kDecodeWarps;
-    static constexpr int kRow = D * 2;              // bytes of one K or V row
+    static constexpr int kRow = D * EB;             // bytes of one K or V row (EB bytes per value)
     static constexpr int kTile = BS * kRow;         // one (block, kv head) tile
     static constexpr int kPanel = BS * 128;         // one 64-column panel of a tile
     static constexpr int kStageK = PA_STAGE_K_BYTES;  // K tiles of up to kHeadsPerStage heads of one block
@@ -598,7 +724,7 @@ struct DecodeCfg {
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kMiscBytes = 256;
     static constexpr int kSmemBytes = kMiscOff + kMiscBytes + 1024;  // + alignment slack
-    static_assert(kTile % 1024 == 0 && kStage % 1024 == 0, "TMA tile alignment");
+    static_assert(kTile % 1024 == 0 && kStage % 1024 == 0, "TMA tile alignment (128-byte swizzle)");
     static_assert(kBarOff % 8 == 0, "mbarrier alignment");
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
@@ -701,7 +827,7 @@ constexpr int kMergeMaxPieces = 64;
 
 template <int D, int G>
 __device__ __noinline__ void merge_pieces(const DecodeParams& p, int k0, int off, int stride, int n, int HG,
-                                          int warp, int lane, __nv_bfloat16* out) {
+                                          int warp, int lane, __nv_bfloat16* out, float oscale = 1.f) {
     auto base = [&](int i) -> int64_t {
         const int leaf = off + i * stride;
         return ((int64_t(k0 + leaf) * 2 + (leaf == 0 ? 1 : 0)) * HG + warp) * G;
@@ -773,7 +899,7 @@ __device__ __noinline__ void merge_pieces(const DecodeParams& p, int k0, int off
 #pragma unroll
         for (int hh = 1; hh < G; ++hh)
             if (hh == h) ls = lsum[hh];
-        const float inv = 1.f / ls;
+        const float inv = (out ? oscale : 1.f) / ls;
         if (out) {
             *reinterpret_cast<uint2*>(out + h * D + dd) = make_uint2(float2_to_bf16x2(a[t].x * inv, a[t].y * inv),
                                                                      float2_to_bf16x2(a[t].z * inv, a[t].w * inv));
@@ -796,7 +922,7 @@ __device__ __noinline__ void merge_pieces(const DecodeParams& p, int k0, int off
 
 template <int D, int G, int BS, int R, bool DUMP, bool APPEND, template <int, int, int> class Math>
 __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
-    using Cfg = DecodeCfg<D, BS, R>;
+    using Cfg = DecodeCfg<D, BS, R, Math<D, G, BS>::kElemBytes>;
     constexpr int NW = Cfg::NW;
     constexpr int S = Cfg::kSegSlots;
     constexpr int NT = Cfg::kThreads;
@@ -1091,7 +1217,8 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
         if (d.npg == 0) break;
         const int g = d.hg * HG + warp;  // this warp's kv head
         const int64_t row = int64_t(d.b) * p.Hq + int64_t(g) * G;  // its first query head
-        st.load_q_global(p.q + row * (D * 2), lane, p.qscale);
+        st.load_q_global(p.q + row * (D * 2), lane, p.k_scale ? p.qscale * __ldg(p.k_scale + g) : p.qscale);
+        st.oscale = p.v_scale ? __ldg(p.v_scale + g) : 1.f;
         st.reset();
         // The piece that starts at b's first own page carries the shared
         // prefix: the partial of prefix key range 0 is loaded now and folded
@@ -1211,7 +1338,7 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
             __syncwarp();
             if (nk <= kMergeFanIn) {
                 if (ticket(top, nk, lane)) {
-                    merge_pieces<D, G>(p, d.k0, 0, 1, nk, HG, warp, lane, p.out + row * D);
+                    merge_pieces<D, G>(p, d.k0, 0, 1, nk, HG, warp, lane, p.out + row * D, st.oscale);
                     if (lane == 0) *top = 0;
                 }
             } else {
@@ -1226,7 +1353,7 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
                     __threadfence();
                     __syncwarp();
                     if (ticket(top, runs, lane)) {
-                        merge_pieces<D, G>(p, d.k0, 0, kMergeFanIn, runs, HG, warp, lane, p.out + row * D);
+                        merge_pieces<D, G>(p, d.k0, 0, kMergeFanIn, runs, HG, warp, lane, p.out + row * D, st.oscale);
                         if (lane == 0) *top = 0;
                     }
                 }

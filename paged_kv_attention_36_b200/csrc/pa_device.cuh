@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cuda.h>  // CUtensorMap (the type only; the library does not link libcuda)
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "../../include/pa.h"
@@ -114,17 +115,6 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
 }
 
 // ---- tiled TMA (tensor map) load global -> shared --------------------------
-// 3-D box at coordinates {x, y, z} of the tensor map `tmap` (a __grid_constant__
-// kernel parameter), completing on `bar`.  x must be 16-byte aligned (x = 0 here).
-__device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, int x, int y, int z, uint64_t* bar,
-                                            uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(smem_dst)),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)), "l"(policy)
-        : "memory");
-}
-
 // 4-D box at coordinates {x, y, z, w} of `tmap`, completing on `bar`.  x must
 // be 16-byte aligned (x = 0 here).
 __device__ __forceinline__ void tma_load_4d(void* smem_dst, const void* tmap, int x, int y, int z, int w,
@@ -133,15 +123,6 @@ __device__ __forceinline__ void tma_load_4d(void* smem_dst, const void* tmap, in
         "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
         " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar)), "l"(policy)
-        : "memory");
-}
-
-// Asks L2 to fetch a 3-D box of `tmap` ahead of a later tiled load of it.
-__device__ __forceinline__ void tma_prefetch_3d(const void* tmap, int x, int y, int z, uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.prefetch.tensor.3d.L2.global.tile.L2::cache_hint [%0, {%1, %2, %3}], %4;" ::"l"(
-            reinterpret_cast<uint64_t>(tmap)),
-        "r"(x), "r"(y), "r"(z), "l"(policy)
         : "memory");
 }
 
@@ -212,6 +193,36 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
         "{%0, %1, %2, %3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// c[16x8 f32] += a[16x16 f16, row-major] * b[16x8 f16, col-major]
+__device__ __forceinline__ void mma_f16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// ---- fp8 (OCP E4M3) ----------------------------------------------------------
+// Two E4M3 codes (the low byte is the first element) -> f16x2 (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+    return r;
+}
+
+// Nearest E4M3 codes of two floats (ties to even, saturating at +-448); the
+// first one in the low byte.
+__device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float first, float second) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(second), "f"(first));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t float2_to_f16x2(float a, float b) {
+    __half2 h = __floats2half2_rn(a, b);  // a in the low half
+    return *reinterpret_cast<uint32_t*>(&h);
 }
 
 // ---- data movement and conversion ------------------------------------------
