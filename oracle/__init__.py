@@ -66,6 +66,8 @@ def _load():
         lib.pa_oracle_append_fp8.restype = i32
         lib.pa_oracle_decode_fp8.argtypes = [vp] * 7 + [i64] * 6 + [dbl, vp, i32]
         lib.pa_oracle_decode_fp8.restype = i32
+        lib.pa_oracle_prefill.argtypes = [vp] * 6 + [i64] * 7 + [dbl, vp, i32]
+        lib.pa_oracle_prefill.restype = i32
         _lib = lib
     return _lib
 
@@ -222,4 +224,24 @@ def decode_fp8(q, k_cache8, v_cache8, k_scale, v_scale, block_tables, context_le
     _check(_load().pa_oracle_decode_fp8(_ptr(q), _ptr(k8), _ptr(v8), _ptr(ks), _ptr(vs), _ptr(block_tables),
                                         _ptr(context_lens), B, Hq, Hkv, D, NB, block_tables.shape[1],
                                         float(scale), _ptr(out), int(nthreads or default_threads())))
+    return out
+
+
+def prefill(q, cu_q_lens, k_cache, v_cache, block_tables, context_lens, scale: float,
+            nthreads: int | None = None) -> np.ndarray:
+    """Multi-query (chunked prefill) attention: q [total][Hq][D] u16 holds, for
+    sequence b, rows cu_q_lens[b] .. cu_q_lens[b+1]-1, its last q_len_b
+    tokens; token i (position L_b - q_len_b + i) attends to tokens 0 .. its
+    position.  fp64 [total][Hq][D]."""
+    q, k_cache, v_cache = _u16(q), _u16(k_cache), _u16(v_cache)
+    block_tables, context_lens, cu = _i32(block_tables), _i32(context_lens), _i32(cu_q_lens)
+    total, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_cache.shape
+    B, M = block_tables.shape
+    if D2 != D or cu.shape[0] != B + 1 or int(cu[-1]) != total:
+        raise ValueError("shape mismatch")
+    out = np.zeros((total, Hq, D), dtype=np.float64)
+    _check(_load().pa_oracle_prefill(_ptr(q), _ptr(cu), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                                     _ptr(context_lens), B, Hq, Hkv, D, bs, NB, M, float(scale), _ptr(out),
+                                     int(nthreads or default_threads())))
     return out

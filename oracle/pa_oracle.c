@@ -47,6 +47,14 @@
  *                               position pos(t) = 4*((t % 8) / 2) + 2*(t / 8) + t % 2.
  * The fp8 decode is the formula above with K_t, V_t the dequantized values.
  *
+ * Multi-query (chunked prefill) attention over the paged cache, the step
+ * beside decode in the pages' engines (miniVLLM docs index, "What is
+ * miniVLLM?": flash attention for prefill; Mini-SGLang write-up, "Key
+ * optimizations": chunked prefill): sequence b brings q_len_b query tokens
+ * (rows cu_q_lens[b] .. cu_q_lens[b+1]-1 of q[total][Hq][D]), which are the
+ * last q_len_b of its L_b cached tokens; query token i (position
+ * p = L_b - q_len_b + i) attends causally to tokens t = 0 .. p.
+ *
  * Parity pins: tests/test_oracle_pins.py checks every function here
  * against torch's scaled_dot_product_attention on contiguous K/V, block
  * permutation and block-size invariance, the closed forms for
@@ -94,16 +102,14 @@ static const uint16_t *cache_row(const problem_t *p, const uint16_t *cache,
     return cache + ((block * p->Hkv + g) * p->bs + offset) * p->D;
 }
 
-/* Attention of query head h of sequence b over tokens [t0, t1).
- * Writes the normalised output o[D]; *m_out = max logit, *l_out = sum of
- * exp(s - m).  An empty range gives o = 0, m = -inf, l = 0. */
-static int attend_range(const problem_t *p, int64_t b, int64_t h,
-                        int64_t t0, int64_t t1, double *s_buf,
-                        double *o, double *m_out, double *l_out)
+/* Attention of the query row q (D bf16 values) against kv head g of
+ * sequence b over tokens [t0, t1).  Writes the normalised output o[D];
+ * *m_out = max logit, *l_out = sum of exp(s - m).  An empty range gives
+ * o = 0, m = -inf, l = 0. */
+static int attend_tokens(const problem_t *p, int64_t b, int64_t g, const uint16_t *q,
+                         int64_t t0, int64_t t1, double *s_buf,
+                         double *o, double *m_out, double *l_out)
 {
-    const int64_t G = p->Hq / p->Hkv;
-    const int64_t g = h / G;
-    const uint16_t *q = p->q + (b * p->Hq + h) * p->D;
     for (int64_t d = 0; d < p->D; ++d) o[d] = 0.0;
     if (t1 <= t0) {
         *m_out = -INFINITY;
@@ -134,6 +140,15 @@ static int attend_range(const problem_t *p, int64_t b, int64_t h,
     *m_out = m;
     *l_out = l;
     return PAO_OK;
+}
+
+/* Query head h of sequence b (its row of q[B][Hq][D]) over tokens [t0, t1). */
+static int attend_range(const problem_t *p, int64_t b, int64_t h,
+                        int64_t t0, int64_t t1, double *s_buf,
+                        double *o, double *m_out, double *l_out)
+{
+    const int64_t G = p->Hq / p->Hkv;
+    return attend_tokens(p, b, h / G, p->q + (b * p->Hq + h) * p->D, t0, t1, s_buf, o, m_out, l_out);
 }
 
 /* ---------------------------------------------------------------------
@@ -450,6 +465,70 @@ int pa_oracle_decode_fp8(const uint16_t *q, const uint8_t *k_cache, const uint8_
                               B, Hq, Hkv, D, NB, M, scale, table, out, i, nthreads, PAO_OK};
         if (nthreads == 1) decode_fp8_worker(&jobs[i]);
         else pthread_create(&tid[i], NULL, decode_fp8_worker, &jobs[i]);
+    }
+    if (nthreads > 1)
+        for (int i = 0; i < nthreads; ++i) pthread_join(tid[i], NULL);
+    for (int i = 0; i < nthreads; ++i)
+        if (jobs[i].status != PAO_OK) return jobs[i].status;
+    return PAO_OK;
+}
+
+/* ---------------------------------------------------------------------
+ * Multi-query (chunked prefill) attention, threaded over query rows.
+ * ------------------------------------------------------------------- */
+typedef struct {
+    const problem_t *p;
+    const int32_t *cu_q_lens;
+    double *out;
+    int64_t total_rows, first, stride;
+    int status;
+} prefill_job_t;
+
+static void *prefill_worker(void *arg)
+{
+    prefill_job_t *job = (prefill_job_t *)arg;
+    const problem_t *p = job->p;
+    const int64_t G = p->Hq / p->Hkv;
+    double *s_buf = (double *)malloc(sizeof(double) * (size_t)(p->M * p->bs > 0 ? p->M * p->bs : 1));
+    if (!s_buf) { job->status = PAO_ERR_NOMEM; return NULL; }
+    job->status = PAO_OK;
+    int64_t b = 0;
+    for (int64_t row = job->first; row < job->total_rows; row += job->stride) {
+        const int64_t tok = row / p->Hq, h = row % p->Hq;
+        while (job->cu_q_lens[b + 1] <= tok) ++b;          /* sequence of query token `tok` */
+        const int64_t q_len = job->cu_q_lens[b + 1] - job->cu_q_lens[b];
+        const int64_t pos = p->context_lens[b] - q_len + (tok - job->cu_q_lens[b]);
+        double m, l;
+        int rc = attend_tokens(p, b, h / G, p->q + row * p->D, 0, pos + 1, s_buf,
+                               job->out + row * p->D, &m, &l);
+        if (rc != PAO_OK) { job->status = rc; break; }
+    }
+    free(s_buf);
+    return NULL;
+}
+
+int pa_oracle_prefill(const uint16_t *q, const int32_t *cu_q_lens, const uint16_t *k_cache,
+                      const uint16_t *v_cache, const int32_t *block_tables, const int32_t *context_lens,
+                      int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t bs, int64_t NB, int64_t M,
+                      double scale, double *out, int nthreads)
+{
+    problem_t p = {q, k_cache, v_cache, block_tables, context_lens, B, Hq, Hkv, D, bs, NB, M, scale};
+    int rc = check_problem(&p);
+    if (rc != PAO_OK) return rc;
+    if (!cu_q_lens || !out || cu_q_lens[0] != 0) return PAO_ERR_ARG;
+    for (int64_t b = 0; b < B; ++b) {
+        const int64_t q_len = cu_q_lens[b + 1] - cu_q_lens[b];
+        if (q_len < 0 || q_len > context_lens[b]) return PAO_ERR_LEN;
+    }
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    pthread_t tid[256];
+    prefill_job_t jobs[256];
+    const int64_t total_rows = (int64_t)cu_q_lens[B] * Hq;
+    for (int i = 0; i < nthreads; ++i) {
+        jobs[i] = (prefill_job_t){&p, cu_q_lens, out, total_rows, i, nthreads, PAO_OK};
+        if (nthreads == 1) prefill_worker(&jobs[i]);
+        else pthread_create(&tid[i], NULL, prefill_worker, &jobs[i]);
     }
     if (nthreads > 1)
         for (int i = 0; i < nthreads; ++i) pthread_join(tid[i], NULL);
