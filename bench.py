@@ -54,6 +54,8 @@ def _args():
     ap.add_argument("--workload", default="llama32",
                     choices=["tiny", "qwen3", "llama32", "longskew", "prefix"])
     ap.add_argument("--impl", default="pa", choices=["pa", "reference"])
+    ap.add_argument("--mode", default="decode", choices=["decode", "prefill"],
+                    help="decode step (the default), or multi-query chunked prefill over the cache")
     ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8"],
                     help="cache format: bf16, or fp8 E4M3 codes with per-kv-head scales")
     ap.add_argument("--no-clocks", action="store_true")
@@ -633,11 +635,130 @@ def run_pa_fp8(args, ws, rank, local):
     print(json.dumps(line), flush=True)
 
 
+PREFILL_METRIC = "paged chunked-prefill attention TFLOP/s (causal, over the cache)"
+
+
+def run_prefill(args, ws, rank, local, reference: bool):
+    """--mode prefill: pa_prefill on a chunked-prefill batch with the head
+    shapes of --workload; value = algorithmic TFLOP/s (4*D per query row and
+    visible key).  The reference arm times the oracle on a bounded sample."""
+    from paged_kv_attention_36_b200 import workloads
+    wl = args.workload if args.workload in ("llama32", "qwen3") else "llama32"
+    pb = workloads.make_prefill(wl)
+    flops = workloads.prefill_flops(pb)
+    if reference:
+        if rank != 0:
+            return
+        import numpy as np
+        import oracle
+        from tests import paging
+        nthreads = oracle.default_threads()
+        sub = 2  # a bounded sample: the first two sequences of the batch
+        cu = pb.cu_q_lens[: sub + 1].numpy()
+        sb = workloads.PrefillBatch(pb.q[: int(cu[-1])], pb.cu_q_lens[: sub + 1], pb.k_cache, pb.v_cache,
+                                    pb.block_tables[:sub], pb.context_lens[:sub], pb.scale, pb.description)
+        sflops = workloads.prefill_flops(sb)
+        args_ = (paging.bits(sb.q), cu, paging.bits(pb.k_cache), paging.bits(pb.v_cache),
+                 sb.block_tables.numpy(), sb.context_lens.numpy(), pb.scale)
+        for _ in range(max(1, min(args.warmup, 1))):
+            oracle.prefill(*args_, nthreads=nthreads)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            oracle.prefill(*args_, nthreads=nthreads)
+        per = (time.perf_counter() - t0) / args.steps
+        value = sflops / per / 1e12
+        print(json.dumps({
+            "impl": "reference", "metric": PREFILL_METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"prefill-{wl}", "description": pb.description},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": nthreads, "kind": "oracle",
+                             "sample": f"the first {sub} of {pb.cu_q_lens.shape[0] - 1} sequences per step"},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }), flush=True)
+        return
+    from paged_kv_attention_36_b200 import binding as pa
+    dev = torch.device("cuda", local if ws > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+    t = {k: getattr(pb, k).to(dev) for k in ("q", "cu_q_lens", "k_cache", "v_cache", "block_tables", "context_lens")}
+    out = torch.empty_like(t["q"])
+    stream = torch.cuda.current_stream(dev)
+    call = pa.prepare_prefill(t["q"], t["cu_q_lens"], pb.max_q_len, t["k_cache"], t["v_cache"], t["block_tables"],
+                              t["context_lens"], pb.scale, out, stream=stream)
+    W_ = max(3, args.warmup)
+    for _ in range(W_):
+        call()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    clocks = ClockSampler(dev.index, enabled=not args.no_clocks)
+    _barrier(ws)
+    torch.cuda.synchronize(dev)
+    for k in range(K):
+        ev[k][0].record(stream)
+        call()
+        ev[k][1].record(stream)
+    torch.cuda.synchronize(dev)
+    _barrier(ws)
+    clk = clocks.stop()
+    errs = pa.pa_device_errors(clear=True)
+    if errs:
+        raise RuntimeError(f"device error bits {errs:#x} during the benchmark")
+    total_ms = _max_over_ranks(sum(ev[k][0].elapsed_time(ev[k][1]) for k in range(K)), ws)
+    # end to end: q and the batch metadata from pinned host memory, out back
+    host = {n: getattr(pb, n).pin_memory() for n in ("q", "cu_q_lens", "block_tables", "context_lens")}
+    out_h = torch.empty(pb.q.shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+    ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    torch.cuda.synchronize(dev)
+    for k in range(K):
+        ee[k][0].record(stream)
+        for n, x in host.items():
+            t[n].copy_(x, non_blocking=True)
+        call()
+        out_h.copy_(out, non_blocking=True)
+        ee[k][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = _max_over_ranks(sum(ee[k][0].elapsed_time(ee[k][1]) for k in range(K)), ws)
+    if rank != 0:
+        return
+    avg = total_ms / K
+    achieved = flops / (avg * 1e-3) / 1e12
+    pk_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    peak, kind = 1590.0, "fallback"
+    if os.path.exists(pk_path):
+        with open(pk_path) as f:
+            pk = json.load(f)
+        if "bf16_tflops" in pk:
+            peak, kind = float(pk["bf16_tflops"]), "measured"
+    print(json.dumps({
+        "metric": PREFILL_METRIC, "value": round(ws * achieved, 2), "unit": "TFLOP/s", "n_gpus": ws, "steps": K,
+        "warmup": W_, "ms_per_step": round(avg, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "storage_dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"prefill-{wl}", "description": pb.description, "flops_per_step": flops,
+                   "l2": (f"no flush: the {2 * pb.k_cache.numel() * 2 / 1e6:.0f} MB of K/V are re-read by every "
+                          "row tile of a sequence, through L2 by design")},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": kind,
+                     "kernel": "pa::prefill_kernel (mma.sync m16n8k16; P.V as two bf16 products)",
+                     "traffic": None},
+        "e2e": {"value": round(ws * flops / (e2e_ms / K * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / K, 5)},
+        "gpu_launches": K,
+        "clocks": clk,
+    }), flush=True)
+
+
 def main():
     args = _args()
     ws, rank, local = _dist()
     try:
-        if args.impl == "reference":
+        if args.mode == "prefill":
+            if args.impl != "reference" and not torch.cuda.is_available():
+                raise SystemExit("bench.py needs a CUDA device for --impl pa")
+            run_prefill(args, ws, rank, local, reference=args.impl == "reference")
+        elif args.impl == "reference":
             run_reference(args, ws, rank)
         else:
             if not torch.cuda.is_available():

@@ -286,6 +286,32 @@ PA_API pa_status pa_decode_fp8(const void* q, const void* k_cache, const void* v
                                size_t workspace_bytes, void* stream);
 
 /*
+ * Multi-query (chunked prefill) attention over the paged cache, the step
+ * beside decode in the pages' engines (miniVLLM docs index, "What is
+ * miniVLLM?": flash attention for prefill; Mini-SGLang write-up, "Key
+ * optimizations": chunked prefill).  Sequence b brings
+ * q_len_b = cu_q_lens[b+1] - cu_q_lens[b] query tokens, rows cu_q_lens[b] ..
+ * cu_q_lens[b+1]-1 of q [total][Hq][D] (bf16), which are the LAST q_len_b of
+ * its context_lens[b] cached tokens (append their K/V rows first, e.g. with
+ * pa_cache_append).  Query token i, at position p = L_b - q_len_b + i,
+ * attends causally to tokens 0 .. p:
+ *     out[cu_q_lens[b] + i][h] = sum_{t <= p} softmax_t(scale * q . K_t) V_t
+ * (bf16, round to nearest even; fp32 products, sums and softmax state).
+ *   - cu_q_lens [B+1] int32 (device), cu_q_lens[0] = 0, non-decreasing;
+ *     max_q_len (host) >= every q_len_b (it sizes the grid; rows past it
+ *     are not computed).  q_len_b > L_b sets PA_DEVERR_CONTEXT (the
+ *     sequence's output is then unspecified).
+ *   - Shapes and alignment as for pa_decode (block_size 16, head_dim 64 or
+ *     128, Hq/Hkv in {1, 2, 4, 8}); out [total][Hq][D].  No workspace.
+ * One CTA per (sequence, 128-row tile, kv head) streams the sequence's
+ * pages up to the tile's last position and computes the row tile against
+ * each page on the tensor cores (mma.sync m16n8k16).
+ */
+PA_API pa_status pa_prefill(const void* q, const int32_t* cu_q_lens, int32_t max_q_len, const void* k_cache,
+                            const void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
+                            float scale, void* out, const pa_dims* dims, void* stream);
+
+/*
  * Reads (and, if `clear` != 0, resets) the device error word of the
  * current device.  Synchronous: waits for all prior work on the device.
  */

@@ -69,6 +69,8 @@ def _load(path: str = LIB_PATH):
     lib.pa_cache_append_fp8.restype = i32
     lib.pa_decode_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, f32, vp, dp, vp, sz, vp]
     lib.pa_decode_fp8.restype = i32
+    lib.pa_prefill.argtypes = [vp, vp, i32, vp, vp, vp, vp, f32, vp, dp, vp]
+    lib.pa_prefill.restype = i32
     lib.pa_decode_static_ws.argtypes = [vp, vp, vp, vp, vp, f32, vp, dp, vp]
     lib.pa_decode_static_ws.restype = i32
     lib.pa_device_errors.argtypes = [ctypes.POINTER(i32), i32]
@@ -84,7 +86,7 @@ lib = _load()
 EXPORTS = ("pa_cache_append", "pa_decode_workspace_bytes", "pa_decode_default_ctas", "pa_decode",
            "pa_append_decode", "pa_decode_partials", "pa_decode_static_ws",
            "pa_decode_shared_prefix_workspace_bytes", "pa_decode_shared_prefix", "pa_cache_append_fp8",
-           "pa_decode_fp8", "pa_device_errors", "pa_status_string")
+           "pa_decode_fp8", "pa_prefill", "pa_device_errors", "pa_status_string")
 
 PA_ERR_SCRATCH_LIMIT = -7
 PA_STATIC_SCRATCH_BYTES = 4 << 20  # include/pa.h
@@ -406,6 +408,43 @@ def prepare_decode_fp8(q, k_cache8, v_cache8, k_scale, v_scale, block_tables, co
                   _ptr(context_lens), float(scale), _ptr(out), ctypes.byref(dims), _ptr(workspace),
                   workspace.numel(), _stream(stream)), "pa_decode_fp8")
     p._keep = (dims, q, k_cache8, v_cache8, k_scale, v_scale, block_tables, context_lens, out, workspace)
+    return p
+
+
+def _prefill_args(q, cu_q_lens, k_cache, v_cache, block_tables, context_lens, out):
+    _need(q, torch.bfloat16, "q", 3)
+    _need(out, torch.bfloat16, "out", 3)
+    _need(cu_q_lens, torch.int32, "cu_q_lens", 1)
+    _need(k_cache, torch.bfloat16, "k_cache", 4)
+    _need(v_cache, torch.bfloat16, "v_cache", 4)
+    _need(block_tables, torch.int32, "block_tables", 2)
+    _need(context_lens, torch.int32, "context_lens", 1)
+    B = block_tables.shape[0]
+    if out.shape != q.shape or cu_q_lens.shape[0] != B + 1 or context_lens.shape[0] != B or \
+            k_cache.shape != v_cache.shape or k_cache.shape[3] != q.shape[2]:
+        raise ValueError("prefill shapes disagree")
+    NB, Hkv, bs, D = k_cache.shape
+    return pa_dims(B, q.shape[1], Hkv, D, bs, NB, block_tables.shape[1])
+
+
+def pa_prefill(q, cu_q_lens, max_q_len: int, k_cache, v_cache, block_tables, context_lens, scale: float, out,
+               stream=None) -> None:
+    """Multi-query (chunked prefill) attention over the paged cache: the
+    rows cu_q_lens[b] .. cu_q_lens[b+1]-1 of q are the last tokens of
+    sequence b's context and attend causally (see include/pa.h)."""
+    dims = _prefill_args(q, cu_q_lens, k_cache, v_cache, block_tables, context_lens, out)
+    _check(lib.pa_prefill(_ptr(q), _ptr(cu_q_lens), int(max_q_len), _ptr(k_cache), _ptr(v_cache),
+                          _ptr(block_tables), _ptr(context_lens), float(scale), _ptr(out), ctypes.byref(dims),
+                          _stream(stream)), "pa_prefill")
+
+
+def prepare_prefill(q, cu_q_lens, max_q_len: int, k_cache, v_cache, block_tables, context_lens, scale: float,
+                    out, stream=None) -> "Prepared":
+    dims = _prefill_args(q, cu_q_lens, k_cache, v_cache, block_tables, context_lens, out)
+    p = Prepared(lib.pa_prefill,
+                 (_ptr(q), _ptr(cu_q_lens), int(max_q_len), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                  _ptr(context_lens), float(scale), _ptr(out), ctypes.byref(dims), _stream(stream)), "pa_prefill")
+    p._keep = (dims, q, cu_q_lens, k_cache, v_cache, block_tables, context_lens, out)
     return p
 
 

@@ -12,6 +12,7 @@
 #include "pa_append.cuh"
 #include "pa_decode.cuh"
 #include "pa_device.cuh"
+#include "pa_prefill.cuh"
 #include "pa_prefix.cuh"
 
 namespace {
@@ -343,6 +344,36 @@ pa_status dispatch_prefix(int D, int G, const pa::PrefixParams& p, dim3 grid, cu
             case 2: return launch_prefix<128, 2>(p, grid, s);
             case 4: return launch_prefix<128, 4>(p, grid, s);
             case 8: return launch_prefix<128, 8>(p, grid, s);
+        }
+    }
+    return PA_ERR_UNSUPPORTED;
+}
+
+// ---- multi-query (chunked prefill) attention -----------------------------------
+template <int D, int G>
+pa_status launch_prefill(const pa::PrefillParams& p, dim3 grid, cudaStream_t stream) {
+    using Cfg = pa::PrefixCfg<D, kPrefixNW, kPrefixStages>;
+    auto kern = pa::prefill_kernel<D, G, kPrefixNW, kPrefixStages>;
+    static unsigned attr_done[kMaxDevices];
+    if (!set_smem_once(kern, Cfg::kSmemBytes, attr_done)) return PA_ERR_CUDA;
+    kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status dispatch_prefill(int D, int G, const pa::PrefillParams& p, dim3 grid, cudaStream_t s) {
+    if (D == 64) {
+        switch (G) {
+            case 1: return launch_prefill<64, 1>(p, grid, s);
+            case 2: return launch_prefill<64, 2>(p, grid, s);
+            case 4: return launch_prefill<64, 4>(p, grid, s);
+            case 8: return launch_prefill<64, 8>(p, grid, s);
+        }
+    } else if (D == 128) {
+        switch (G) {
+            case 1: return launch_prefill<128, 1>(p, grid, s);
+            case 2: return launch_prefill<128, 2>(p, grid, s);
+            case 4: return launch_prefill<128, 4>(p, grid, s);
+            case 8: return launch_prefill<128, 8>(p, grid, s);
         }
     }
     return PA_ERR_UNSUPPORTED;
@@ -716,6 +747,45 @@ pa_status pa_decode_fp8(const void* q, const void* k_cache, const void* v_cache,
     p.v_scale = v_scale;
     return dispatch_d_g<MathKind::kFp8, false, false>(dims->head_dim, dims->num_q_heads / dims->num_kv_heads, p,
                                                       grid, static_cast<cudaStream_t>(stream), false);
+}
+
+pa_status pa_prefill(const void* q, const int32_t* cu_q_lens, int32_t max_q_len, const void* k_cache,
+                     const void* v_cache, const int32_t* block_tables, const int32_t* context_lens, float scale,
+                     void* out, const pa_dims* dims, void* stream) {
+    if (!dims) return PA_ERR_NULL;
+    if (!dims_ok(dims) || max_q_len < 0) return PA_ERR_SHAPE;
+    const pa_dims& d = *dims;
+    const int G = d.num_q_heads / d.num_kv_heads;
+    if (d.block_size != kBlockSize || !supported(d.head_dim, G, MathKind::kMma)) return PA_ERR_UNSUPPORTED;
+    if (d.num_seqs == 0 || max_q_len == 0) return PA_OK;
+    if (d.num_blocks == 0) return PA_ERR_SHAPE;
+    if (!q || !cu_q_lens || !k_cache || !v_cache || !block_tables || !context_lens || !out) return PA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(out) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned4(cu_q_lens) ||
+        !aligned4(block_tables) || !aligned4(context_lens))
+        return PA_ERR_ALIGN;
+    const int64_t rows = int64_t(d.num_blocks) * d.num_kv_heads * d.block_size;
+    if (rows >= (int64_t(1) << 31)) return PA_ERR_SHAPE;
+    const int64_t tiles = (int64_t(max_q_len) * G + 16 * kPrefixNW - 1) / (16 * kPrefixNW);
+    if (int64_t(d.num_seqs) * tiles > 0x7fffffffLL || d.num_kv_heads > 65535) return PA_ERR_SHAPE;
+    pa::PrefillParams p;
+    const int64_t cache_tiles = int64_t(d.num_blocks) * d.num_kv_heads;
+    if (!make_cache_map(&p.tmap_k, k_cache, cache_tiles, d.head_dim, d.block_size, 1) ||
+        !make_cache_map(&p.tmap_v, v_cache, cache_tiles, d.head_dim, d.block_size, 1))
+        return PA_ERR_CUDA;
+    p.q = static_cast<const uint8_t*>(q);
+    p.cu_q_lens = cu_q_lens;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.B = d.num_seqs;
+    p.Hq = d.num_q_heads;
+    p.Hkv = d.num_kv_heads;
+    p.NB = d.num_blocks;
+    p.M = d.max_blocks_per_seq;
+    p.tiles_per_seq = int32_t(tiles);
+    p.qscale = scale * kLog2e;
+    return dispatch_prefill(d.head_dim, G, p, dim3(unsigned(d.num_seqs * tiles), unsigned(d.num_kv_heads)),
+                            static_cast<cudaStream_t>(stream));
 }
 
 pa_status pa_device_errors(int32_t* errors_out, int32_t clear) {

@@ -32,6 +32,140 @@
 
 namespace pa {
 
+// Sixteen query rows of one warp against staged (block, kv head) tiles of 16
+// tokens (128-byte-swizzled panels, see tile_off), FlashAttention-2
+// fragment flow on mma.sync m16n8k16 (bf16 in, fp32 accumulate).  Lane l
+// holds rows lr = l/4 and lr+8 of the 16: its query fragments, and the
+// accumulator columns 8*nt + 2*(l%4), +1 of both rows.
+template <int D>
+struct RowTile {
+    static constexpr int KS = D / 16;
+    uint32_t qa[KS][4];
+    float o[D / 8][4];
+    float m0, m1, l0, l1;  // rows lr and lr + 8: running max (base 2), running sum
+
+    // row0 / row1: the D bf16 query values of rows lr and lr+8, or nullptr (zeros)
+    __device__ __forceinline__ void load_q(const uint8_t* row0, const uint8_t* row1, int lane) {
+        const int lc = (lane & 3) * 2;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const uint32_t* row = reinterpret_cast<const uint32_t*>(e ? row1 : row0);
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                qa[ks][e] = row ? __ldg(row + (16 * ks + lc) / 2) : 0u;          // a0a1 / a2a3: columns lc, lc+1
+                qa[ks][2 + e] = row ? __ldg(row + (16 * ks + lc + 8) / 2) : 0u;  // a4a5 / a6a7: columns + 8
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+        m0 = m1 = -INFINITY;
+        l0 = l1 = 0.f;
+    }
+
+    // One page: tokens [0, lim0) count for row lr and [0, lim1) for row lr+8
+    // (the others are masked out of the softmax); V rows at or past vvalid
+    // hold no data and are zeroed in the fragments (0 * NaN would poison).
+    // Every row must have had a counted token by its first page.
+    __device__ __forceinline__ void page(const uint8_t* kt, const uint8_t* vt, int lim0, int lim1, int vvalid,
+                                         float qscale, int lane) {
+        const int lc = (lane & 3) * 2;
+        // ---- S = Q . K^T, two n8 tiles of tokens ----
+        float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        {
+            const int t = (lane & 7) + ((lane >> 4) << 3);
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                uint32_t kb[4];
+                ldmatrix_x4(kb, kt + tile_off(t, 2 * ks + ((lane >> 3) & 1)));
+                mma_bf16_16816(s[0], qa[ks], kb[0], kb[1]);
+                mma_bf16_16816(s[1], qa[ks], kb[2], kb[3]);
+            }
+        }
+        // s[nt][0..1]: row lr, tokens 8nt + lc, +1; s[nt][2..3]: row lr + 8
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const int tok = 8 * nt + lc + (x & 1);
+                const int lim = x < 2 ? lim0 : lim1;
+                s[nt][x] = tok < lim ? s[nt][x] * qscale : -INFINITY;
+            }
+        // ---- online softmax per row (the 4 lanes of a row hold its 16 tokens) ----
+        float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+        float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+        if (__any_sync(0xffffffffu, mx0 > m0 || mx1 > m1)) {
+            const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+            const float a0 = exp2f(m0 - n0), a1 = exp2f(m1 - n1);
+            m0 = n0;
+            m1 = n1;
+            l0 *= a0;
+            l1 *= a1;
+#pragma unroll
+            for (int nt = 0; nt < D / 8; ++nt) {
+                o[nt][0] *= a0;
+                o[nt][1] *= a0;
+                o[nt][2] *= a1;
+                o[nt][3] *= a1;
+            }
+        }
+        float pr[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            pr[nt][0] = exp2f(s[nt][0] - m0);
+            pr[nt][1] = exp2f(s[nt][1] - m0);
+            pr[nt][2] = exp2f(s[nt][2] - m1);
+            pr[nt][3] = exp2f(s[nt][3] - m1);
+            l0 += pr[nt][0] + pr[nt][1];
+            l1 += pr[nt][2] + pr[nt][3];
+        }
+        // ---- P as the A operand (k = the page's 16 tokens): bf16 high part and remainder ----
+        // a0a1: (row lr, tokens lc..lc+1) = tile 0 top; a2a3: row lr+8; a4a5 / a6a7: tile 1
+        uint32_t ph[4], pl[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const int nt = x >> 1, half = x & 1;
+            const float u = pr[nt][2 * half], v = pr[nt][2 * half + 1];
+            ph[x] = float2_to_bf16x2(u, v);
+            const float2 f = bf16x2_to_float2(ph[x]);
+            pl[x] = float2_to_bf16x2(u - f.x, v - f.y);
+        }
+        // ---- O += P . V; V fragment b0b1 holds tokens lc, lc+1, b2b3 tokens lc+8, lc+9 ----
+        uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+        if (vvalid < 16) {
+            mlo = (lc < vvalid ? 0x0000ffffu : 0u) | (lc + 1 < vvalid ? 0xffff0000u : 0u);
+            mhi = (lc + 8 < vvalid ? 0x0000ffffu : 0u) | (lc + 9 < vvalid ? 0xffff0000u : 0u);
+        }
+        {
+            const int t = (lane & 7) + (((lane >> 3) & 1) << 3);
+#pragma unroll
+            for (int nd = 0; nd < D / 16; ++nd) {
+                uint32_t vb[4];
+                ldmatrix_x4_trans(vb, vt + tile_off(t, 2 * nd + (lane >> 4)));
+                vb[0] &= mlo;
+                vb[1] &= mhi;
+                vb[2] &= mlo;
+                vb[3] &= mhi;
+                mma_bf16_16816(o[2 * nd], ph, vb[0], vb[1]);
+                mma_bf16_16816(o[2 * nd], pl, vb[0], vb[1]);
+                mma_bf16_16816(o[2 * nd + 1], ph, vb[2], vb[3]);
+                mma_bf16_16816(o[2 * nd + 1], pl, vb[2], vb[3]);
+            }
+        }
+    }
+
+    // Sums l over the 4 lanes of each row.
+    __device__ __forceinline__ void finish() {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    }
+};
+
 struct PrefixParams {
     CUtensorMap tmap_k;
     CUtensorMap tmap_v;
@@ -76,7 +210,6 @@ __host__ __device__ __forceinline__ int prefix_split_pages(int P, int splits) { 
 template <int D, int G, int NW, int RS>
 __global__ void __launch_bounds__((NW + 1) * 32, 1) prefix_kernel(const __grid_constant__ PrefixParams p) {
     using Cfg = PrefixCfg<D, NW, RS>;
-    constexpr int KS = D / 16;
     static_assert(Cfg::kRows % G == 0, "a tile holds whole members");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -201,122 +334,40 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) prefix_kernel(const __grid_c
     // rows wr0 .. wr0+15 of the group; row r = (member first + r / G, head g*G + r % G)
     const int wr0 = row0 + warp * 16;
     const int lr = lane >> 2, lc = (lane & 3) * 2;
-    uint32_t qa[KS][4];
+    RowTile<D> rt;
+    {
+        const uint8_t* rows[2];
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-        const int r = wr0 + lr + 8 * e;
-        const uint32_t* row = nullptr;
-        if (r < nrows)
-            row = reinterpret_cast<const uint32_t*>(p.q + (int64_t(first + r / G) * p.Hq + g * G + r % G) * Cfg::kRow);
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-            qa[ks][e] = row ? __ldg(row + (16 * ks + lc) / 2) : 0u;          // a0a1 / a2a3: columns lc, lc+1
-            qa[ks][2 + e] = row ? __ldg(row + (16 * ks + lc + 8) / 2) : 0u;  // a4a5 / a6a7: columns + 8
+        for (int e = 0; e < 2; ++e) {
+            const int r = wr0 + lr + 8 * e;
+            rows[e] = r < nrows ? p.q + (int64_t(first + r / G) * p.Hq + g * G + r % G) * Cfg::kRow : nullptr;
         }
+        rt.load_q(rows[0], rows[1], lane);
     }
-    float o[D / 8][4];
-#pragma unroll
-    for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // rows lr and lr + 8
-
     for (int i = 0; i < npages; ++i) {
         const int slot = i % RS;
         if (!mbar_wait(&full[slot], uint32_t(i / RS) & 1, abort)) return;
         const uint8_t* kt = smem + slot * Cfg::kPage;
-        const uint8_t* vt = kt + Cfg::kTile;
-        // ---- S = Q . K^T, two n8 tiles of tokens ----
-        float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        {
-            const int t = (lane & 7) + ((lane >> 4) << 3);
-#pragma unroll
-            for (int ks = 0; ks < KS; ++ks) {
-                uint32_t kb[4];
-                ldmatrix_x4(kb, kt + tile_off(t, 2 * ks + ((lane >> 3) & 1)));
-                mma_bf16_16816(s[0], qa[ks], kb[0], kb[1]);
-                mma_bf16_16816(s[1], qa[ks], kb[2], kb[3]);
-            }
-        }
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int x = 0; x < 4; ++x) s[nt][x] *= p.qscale;
-        // ---- online softmax per row (the 4 lanes of a row hold its 16 tokens) ----
-        float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
-        float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        if (__any_sync(0xffffffffu, mx0 > m0 || mx1 > m1)) {
-            const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-            const float a0 = exp2f(m0 - n0), a1 = exp2f(m1 - n1);
-            m0 = n0;
-            m1 = n1;
-            l0 *= a0;
-            l1 *= a1;
-#pragma unroll
-            for (int nt = 0; nt < D / 8; ++nt) {
-                o[nt][0] *= a0;
-                o[nt][1] *= a0;
-                o[nt][2] *= a1;
-                o[nt][3] *= a1;
-            }
-        }
-        float pr[2][4];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            pr[nt][0] = exp2f(s[nt][0] - m0);
-            pr[nt][1] = exp2f(s[nt][1] - m0);
-            pr[nt][2] = exp2f(s[nt][2] - m1);
-            pr[nt][3] = exp2f(s[nt][3] - m1);
-            l0 += pr[nt][0] + pr[nt][1];
-            l1 += pr[nt][2] + pr[nt][3];
-        }
-        // ---- P as the A operand (k = the page's 16 tokens): bf16 high part and remainder ----
-        // a0a1: (row lr, tokens lc..lc+1) = tile 0 top; a2a3: row lr+8; a4a5 / a6a7: tile 1
-        uint32_t ph[4], pl[4];
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            const int nt = x >> 1, half = x & 1;
-            const float u = pr[nt][2 * half], v = pr[nt][2 * half + 1];
-            ph[x] = float2_to_bf16x2(u, v);
-            const float2 f = bf16x2_to_float2(ph[x]);
-            pl[x] = float2_to_bf16x2(u - f.x, v - f.y);
-        }
-        // ---- O += P . V ----
-        {
-            const int t = (lane & 7) + (((lane >> 3) & 1) << 3);
-#pragma unroll
-            for (int nd = 0; nd < D / 16; ++nd) {
-                uint32_t vb[4];
-                ldmatrix_x4_trans(vb, vt + tile_off(t, 2 * nd + (lane >> 4)));
-                mma_bf16_16816(o[2 * nd], ph, vb[0], vb[1]);
-                mma_bf16_16816(o[2 * nd], pl, vb[0], vb[1]);
-                mma_bf16_16816(o[2 * nd + 1], ph, vb[2], vb[3]);
-                mma_bf16_16816(o[2 * nd + 1], pl, vb[2], vb[3]);
-            }
-        }
+        rt.page(kt, kt + Cfg::kTile, 16, 16, 16, p.qscale, lane);  // shared pages are whole
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[slot]);
     }
 
     // ---- the partials of the valid rows ----
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    rt.finish();
     const int64_t plane = int64_t(blockIdx.z) * p.B;
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
         const int r = wr0 + lr + 8 * e;
         if (r >= nrows) continue;
         const int64_t idx = (plane + first + r / G) * p.Hq + g * G + r % G;
-        const float l = e ? l1 : l0, inv = 1.f / l;
+        const float l = e ? rt.l1 : rt.l0, inv = 1.f / l;
         float* dst = p.prefix_o + idx * D;
 #pragma unroll
         for (int nt = 0; nt < D / 8; ++nt)
-            *reinterpret_cast<float2*>(dst + nt * 8 + lc) = make_float2(o[nt][2 * e] * inv, o[nt][2 * e + 1] * inv);
-        if ((lane & 3) == 0) p.prefix_ml[idx] = make_float2(e ? m1 : m0, l);
+            *reinterpret_cast<float2*>(dst + nt * 8 + lc) =
+                make_float2(rt.o[nt][2 * e] * inv, rt.o[nt][2 * e + 1] * inv);
+        if ((lane & 3) == 0) p.prefix_ml[idx] = make_float2(e ? rt.m1 : rt.m0, l);
     }
 
     // ---- checks of the caller's grouping (kv head 0 only): each member holds

@@ -322,3 +322,62 @@ def make_grouped(name: str, groups, suffix_lens, *, tail_lens=(), seed: int | No
     w.group_offsets = torch.tensor(offsets, dtype=torch.int32)
     w.group_prefix_pages = torch.tensor([P for _, P in groups], dtype=torch.int32)
     return w
+
+
+@dataclasses.dataclass
+class PrefillBatch:
+    """A chunked-prefill batch: sequence b's last q_len[b] cached tokens are
+    its queries, rows cu_q_lens[b] .. cu_q_lens[b+1]-1 of q."""
+    q: torch.Tensor             # [total][Hq][D] bf16
+    cu_q_lens: torch.Tensor     # [B + 1] int32
+    k_cache: torch.Tensor       # [NB][Hkv][16][D] bf16
+    v_cache: torch.Tensor
+    block_tables: torch.Tensor  # [B][M] int32
+    context_lens: torch.Tensor  # [B] int32 (prior context + the chunk)
+    scale: float
+    description: str
+
+    @property
+    def max_q_len(self) -> int:
+        return int((self.cu_q_lens[1:] - self.cu_q_lens[:-1]).max().item())
+
+
+def make_prefill(name: str = "llama32", num_seqs: int = 16, chunk: int = 512, prior=(512, 3584),
+                 seed: int | None = None) -> PrefillBatch:
+    """Chunked prefill with the head shapes of configuration `name`: each of
+    `num_seqs` sequences has a prior context U[prior] and a new chunk of
+    `chunk` tokens (cached already), blocks scattered over a shuffled pool."""
+    spec = SPECS[name]
+    g = torch.Generator().manual_seed((spec.seed + 2000) if seed is None else seed)
+    Hq, Hkv, D, bs = spec.num_q_heads, spec.num_kv_heads, spec.head_dim, spec.block_size
+    prior_lens = torch.randint(prior[0], prior[1] + 1, (num_seqs,), generator=g, dtype=torch.int64)
+    lens = prior_lens + chunk
+    pages = _pages(lens, bs)
+    NB = int(pages.sum().item())
+    perm = torch.randperm(NB, generator=g).tolist()
+    lists, cursor = [], 0
+    for b in range(num_seqs):
+        n = int(pages[b].item())
+        lists.append(perm[cursor:cursor + n])
+        cursor += n
+    bt = build_tables(lists, int(pages.max().item()))
+    k_cache = _randn_bf16(g, (NB, Hkv, bs, D))
+    v_cache = _randn_bf16(g, (NB, Hkv, bs, D))
+    q = _randn_bf16(g, (num_seqs * chunk, Hq, D))
+    cu = torch.arange(0, num_seqs + 1, dtype=torch.int32) * chunk
+    desc = (f"chunked prefill, {spec.name} heads ({Hq} q / {Hkv} kv, head_dim {D}): {num_seqs} sequences, "
+            f"{chunk}-token chunks after prior contexts U[{prior[0]},{prior[1]}], causal, block 16")
+    return PrefillBatch(q=q, cu_q_lens=cu, k_cache=k_cache, v_cache=v_cache, block_tables=bt,
+                        context_lens=lens.to(torch.int32), scale=1.0 / math.sqrt(D), description=desc)
+
+
+def prefill_flops(b: PrefillBatch) -> int:
+    """Multiply-adds x 2 of QK and PV: 4 * D flops per (query row, visible key)."""
+    Hq, D = b.q.shape[1], b.q.shape[2]
+    total = 0
+    for i in range(b.cu_q_lens.shape[0] - 1):
+        n = int(b.cu_q_lens[i + 1] - b.cu_q_lens[i])
+        L = int(b.context_lens[i])
+        # query j sees L - n + j + 1 keys
+        total += n * (L - n + 1) + n * (n - 1) // 2
+    return 4 * D * Hq * total
