@@ -155,6 +155,7 @@ struct SimtMath {
     static_assert(D % 64 == 0 && BS % 4 == 0, "layout");
 
     static constexpr int kElemBytes = 2;  // bf16 caches
+    static constexpr bool kPairPages = false;
     float2 q2[G][NCH][4];
     float2 acc[G][NCH][4];
     float m[G];
@@ -390,6 +391,7 @@ struct MmaMath {
     static constexpr bool kZeroMaskedV = true;  // 0 * NaN would poison the mma
 
     static constexpr int kElemBytes = 2;  // bf16 caches
+    static constexpr bool kPairPages = false;
     uint32_t qb[KS][2];  // Q^T as B fragments (bf16 pairs)
     float acc[KS][4];    // O^T accumulator tiles
     float m[2], l[2];    // heads h0, h0 + 1 of this lane (l: this lane's rows only)
@@ -604,6 +606,7 @@ struct Fp8MmaMath : MmaMath<D, G, BS> {
     using Base::qscale;
     static constexpr bool kZeroMaskedV = false;  // masked in the fragments
     static constexpr int kElemBytes = 1;
+    static constexpr bool kPairPages = true;     // page2(): two pages per softmax update
     static_assert(D == 64 || D == 128, "128-byte K lines hold one or two tokens");
 
     __device__ __forceinline__ void load_q_global(const uint8_t* gq, int lane, float qs_scale) {
@@ -696,6 +699,97 @@ struct Fp8MmaMath : MmaMath<D, G, BS> {
             mma_f16_16816(acc[2 * j + 1], a1, b0, b1);
         }
     }
+
+    // Two pages at once (nv1 == 0: the second is absent): both S products in
+    // flight together, one max / rescale over the 32 tokens, then both P.V.
+    __device__ __forceinline__ void page2(const uint8_t* kt0, const uint8_t* vt0, int nv0, const uint8_t* kt1,
+                                          const uint8_t* vt1, int nv1, int lane) {
+        const int mi = lane >> 3, r8 = lane & 7, c = lane & 3;
+        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+            const int t = r8 + ((mi & 1) << 3);
+#pragma unroll
+            for (int j = 0; j < KS / 2; ++j) {
+                uint32_t r[4], u[4];
+                ldmatrix_x4(r, kt0 + k_off(t, 2 * j + (mi >> 1)));
+                ldmatrix_x4(u, kt1 + k_off(t, 2 * j + (mi >> 1)));
+                const uint32_t a0[4] = {lo(r[0]), lo(r[1]), hi(r[0]), hi(r[1])};
+                const uint32_t c0[4] = {lo(u[0]), lo(u[1]), hi(u[0]), hi(u[1])};
+                mma_f16_16816(s0, a0, qb[2 * j][0], qb[2 * j][1]);
+                mma_f16_16816(s1, c0, qb[2 * j][0], qb[2 * j][1]);
+                const uint32_t a1[4] = {lo(r[2]), lo(r[3]), hi(r[2]), hi(r[3])};
+                const uint32_t c1[4] = {lo(u[2]), lo(u[3]), hi(u[2]), hi(u[3])};
+                mma_f16_16816(s0, a1, qb[2 * j + 1][0], qb[2 * j + 1][1]);
+                mma_f16_16816(s1, c1, qb[2 * j + 1][0], qb[2 * j + 1][1]);
+            }
+        }
+        const int t0 = lane >> 2;
+        const bool v00 = t0 < nv0, v01 = (t0 + 8) < nv0, v10 = t0 < nv1, v11 = (t0 + 8) < nv1;
+        s0[0] = v00 ? s0[0] * qscale : -INFINITY;
+        s0[1] = v00 ? s0[1] * qscale : -INFINITY;
+        s0[2] = v01 ? s0[2] * qscale : -INFINITY;
+        s0[3] = v01 ? s0[3] * qscale : -INFINITY;
+        s1[0] = v10 ? s1[0] * qscale : -INFINITY;
+        s1[1] = v10 ? s1[1] * qscale : -INFINITY;
+        s1[2] = v11 ? s1[2] * qscale : -INFINITY;
+        s1[3] = v11 ? s1[3] * qscale : -INFINITY;
+        // ---- one online-softmax step over the 32 tokens of each head column ----
+        float mx0 = fmaxf(fmaxf(s0[0], s0[2]), fmaxf(s1[0], s1[2]));
+        float mx1 = fmaxf(fmaxf(s0[1], s0[3]), fmaxf(s1[1], s1[3]));
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+        }
+        if (__any_sync(0xffffffffu, mx0 > m[0] || mx1 > m[1])) {
+            const float n0 = fmaxf(m[0], mx0), n1 = fmaxf(m[1], mx1);
+            const float a0 = exp2f(m[0] - n0), a1 = exp2f(m[1] - n1);
+            m[0] = n0;
+            m[1] = n1;
+            l[0] *= a0;
+            l[1] *= a1;
+#pragma unroll
+            for (int i = 0; i < KS; ++i) {
+                acc[i][0] *= a0;
+                acc[i][1] *= a1;
+                acc[i][2] *= a0;
+                acc[i][3] *= a1;
+            }
+        }
+        const float p00 = exp2f(s0[0] - m[0]), p01 = exp2f(s0[1] - m[1]);
+        const float p02 = exp2f(s0[2] - m[0]), p03 = exp2f(s0[3] - m[1]);
+        const float p10 = exp2f(s1[0] - m[0]), p11 = exp2f(s1[1] - m[1]);
+        const float p12 = exp2f(s1[2] - m[0]), p13 = exp2f(s1[3] - m[1]);
+        l[0] += (p00 + p02) + (p10 + p12);
+        l[1] += (p01 + p03) + (p11 + p13);
+        const uint32_t b00 = movmatrix_trans(float2_to_f16x2(p00, p01));
+        const uint32_t b01 = movmatrix_trans(float2_to_f16x2(p02, p03));
+        const uint32_t b10 = movmatrix_trans(float2_to_f16x2(p10, p11));
+        const uint32_t b11 = movmatrix_trans(float2_to_f16x2(p12, p13));
+        uint32_t ml0 = 0xffffffffu, mh0 = 0xffffffffu, ml1 = 0xffffffffu, mh1 = 0xffffffffu;
+        if (nv0 < 16) {
+            ml0 = (2 * c < nv0 ? 0x0000ffffu : 0u) | (2 * c + 1 < nv0 ? 0xffff0000u : 0u);
+            mh0 = (2 * c + 8 < nv0 ? 0x0000ffffu : 0u) | (2 * c + 9 < nv0 ? 0xffff0000u : 0u);
+        }
+        if (nv1 < 16) {
+            ml1 = (2 * c < nv1 ? 0x0000ffffu : 0u) | (2 * c + 1 < nv1 ? 0xffff0000u : 0u);
+            mh1 = (2 * c + 8 < nv1 ? 0x0000ffffu : 0u) | (2 * c + 9 < nv1 ? 0xffff0000u : 0u);
+        }
+#pragma unroll
+        for (int j = 0; j < KS / 2; ++j) {
+            uint32_t r[4], u[4];
+            ldmatrix_x4(r, vt0 + (32 * j + lane) * 16);
+            ldmatrix_x4(u, vt1 + (32 * j + lane) * 16);
+            const uint32_t a0[4] = {lo(r[0]) & ml0, lo(r[1]) & ml0, hi(r[0]) & mh0, hi(r[1]) & mh0};
+            mma_f16_16816(acc[2 * j], a0, b00, b01);
+            const uint32_t a1[4] = {lo(r[2]) & ml0, lo(r[3]) & ml0, hi(r[2]) & mh0, hi(r[3]) & mh0};
+            mma_f16_16816(acc[2 * j + 1], a1, b00, b01);
+            const uint32_t c0[4] = {lo(u[0]) & ml1, lo(u[1]) & ml1, hi(u[0]) & mh1, hi(u[1]) & mh1};
+            mma_f16_16816(acc[2 * j], c0, b10, b11);
+            const uint32_t c1[4] = {lo(u[2]) & ml1, lo(u[3]) & ml1, hi(u[2]) & mh1, hi(u[3]) & mh1};
+            mma_f16_16816(acc[2 * j + 1], c1, b10, b11);
+        }
+    }
 };
 
 // ===========================================================================
@@ -708,7 +802,9 @@ struct DecodeCfg {
     static constexpr int kRow = D * EB;             // bytes of one K or V row (EB bytes per value)
     static constexpr int kTile = BS * kRow;         // one (block, kv head) tile
     static constexpr int kPanel = BS * 128;         // one 64-column panel of a tile
-    static constexpr int kStageK = PA_STAGE_K_BYTES;  // K tiles of up to kHeadsPerStage heads of one block
+    // K tiles of up to kHeadsPerStage heads of one block: PA_STAGE_K_BYTES, or
+    // less when all NW heads' tiles are smaller (fp8 at head_dim 64)
+    static constexpr int kStageK = PA_STAGE_K_BYTES < NW * kTile ? PA_STAGE_K_BYTES : NW * kTile;
     static constexpr int kStage = 2 * kStageK;        // then their V tiles
     static constexpr int kHeadsPerStage = kStageK / kTile;
     static constexpr int kMaxSpl = NW / kHeadsPerStage > 1 ? NW / kHeadsPerStage : 1;  // stages per page, at most
@@ -1232,6 +1328,27 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
 
         // (R is a multiple of SPL, so the stages of each warp recur in the
         // same slots and every parity wait is exact)
+        if constexpr (MathT::kPairPages) {
+            // two pages per softmax step (one stage per page: SPL == 1 here)
+            for (int k = 0; k < d.npg; k += 2) {
+                const uint32_t i0 = stage_base + uint32_t(k), i1 = i0 + 1;
+                const bool two = k + 1 < d.npg;
+                const int slot0 = int(i0 % R), slot1 = int(i1 % R);
+                if (!mbar_wait(&full[slot0], (i0 / R) & 1, abort)) return;
+                if (two && !mbar_wait(&full[slot1], (i1 / R) & 1, abort)) return;
+                const uint8_t* kt0 = ring + slot0 * Cfg::kStage + pos * Cfg::kTile;
+                const uint8_t* kt1 = two ? ring + slot1 * Cfg::kStage + pos * Cfg::kTile : kt0;
+                const int nr0 = d.L - (d.j0 + k) * BS, nr1 = d.L - (d.j0 + k + 1) * BS;
+                const int nv0 = nr0 < BS ? nr0 : BS;
+                const int nv1 = two ? (nr1 < BS ? nr1 : BS) : 0;
+                st.page2(kt0, kt0 + Cfg::kStageK, nv0, kt1, kt1 + Cfg::kStageK, nv1, lane);
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&empty[slot0]);
+                    if (two) mbar_arrive(&empty[slot1]);
+                }
+            }
+        } else
         for (int k = 0; k < d.npg; ++k) {
             const uint32_t i = stage_base + uint32_t(k * SPL + sub);
             const int slot = int(i % R);
