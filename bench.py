@@ -741,7 +741,9 @@ def run_prefill(args, ws, rank, local, reference: bool):
                           "row tile of a sequence, through L2 by design")},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "peak_kind": kind,
-                     "kernel": "pa::prefill_kernel (mma.sync m16n8k16; P.V as two bf16 products)",
+                     "kernel": ("pa::prefill_kernel (mma.sync m16n8k16; P.V as two bf16 products)"
+                                if os.environ.get("PA_PREFILL_MMA") == "sync" else
+                                "pa::prefill_tc_kernel (tcgen05.mma, S/P and O in TMEM, TMA-fed K/V)"),
                      "traffic": None},
         "e2e": {"value": round(ws * flops / (e2e_ms / K * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / K, 5)},

@@ -13,6 +13,7 @@
 #include "pa_decode.cuh"
 #include "pa_device.cuh"
 #include "pa_prefill.cuh"
+#include "pa_prefill_tc.cuh"
 #include "pa_prefix.cuh"
 
 namespace {
@@ -177,6 +178,21 @@ bool make_cache_map(CUtensorMap* map, const void* base, int64_t tiles, int D, in
     cuuint64_t dims[4] = {64, cuuint64_t(bs), cuuint64_t(D / 64), cuuint64_t(tiles)};
     cuuint64_t strides[3] = {cuuint64_t(D) * 2, 128, cuuint64_t(bs) * D * 2};
     cuuint32_t box[4] = {64, cuuint32_t(bs), cuuint32_t(D / 64), cuuint32_t(heads)};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, PA_L2_PROMOTION,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The same 4-D view with a box of one 64-wide panel of one (block, kv head)
+// tile: {64, 16, 1, 1} at {0, 0, panel, tile}, so a block of pages lands as
+// [panel][tokens][128 bytes] (the tcgen05 operand layout).
+bool make_panel_map(CUtensorMap* map, const void* base, int64_t tiles, int D, int bs) {
+    auto fn = encode_tiled();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {64, cuuint64_t(bs), cuuint64_t(D / 64), cuuint64_t(tiles)};
+    cuuint64_t strides[3] = {cuuint64_t(D) * 2, 128, cuuint64_t(bs) * D * 2};
+    cuuint32_t box[4] = {64, cuuint32_t(bs), 1, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, PA_L2_PROMOTION,
@@ -358,6 +374,48 @@ pa_status launch_prefill(const pa::PrefillParams& p, dim3 grid, cudaStream_t str
     if (!set_smem_once(kern, Cfg::kSmemBytes, attr_done)) return PA_ERR_CUDA;
     kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+// tcgen05 prefill: BN keys per block, KS blocks in the ring.
+constexpr int kTcBN = 128;
+template <int D> constexpr int tc_stages() { return D == 64 ? 4 : 3; }
+
+template <int D, int G>
+pa_status launch_prefill_tc(const pa::PrefillParams& p, dim3 grid, cudaStream_t stream) {
+    using Cfg = pa::TcPrefillCfg<D, kTcBN, tc_stages<D>()>;
+    auto kern = pa::prefill_tc_kernel<D, G, kTcBN, tc_stages<D>()>;
+    static unsigned attr_done[kMaxDevices];
+    if (!set_smem_once(kern, Cfg::kSmemBytes, attr_done)) return PA_ERR_CUDA;
+    kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status dispatch_prefill_tc(int D, int G, const pa::PrefillParams& p, dim3 grid, cudaStream_t s) {
+    if (D == 64) {
+        switch (G) {
+            case 1: return launch_prefill_tc<64, 1>(p, grid, s);
+            case 2: return launch_prefill_tc<64, 2>(p, grid, s);
+            case 4: return launch_prefill_tc<64, 4>(p, grid, s);
+            case 8: return launch_prefill_tc<64, 8>(p, grid, s);
+        }
+    } else if (D == 128) {
+        switch (G) {
+            case 1: return launch_prefill_tc<128, 1>(p, grid, s);
+            case 2: return launch_prefill_tc<128, 2>(p, grid, s);
+            case 4: return launch_prefill_tc<128, 4>(p, grid, s);
+            case 8: return launch_prefill_tc<128, 8>(p, grid, s);
+        }
+    }
+    return PA_ERR_UNSUPPORTED;
+}
+
+// PA_PREFILL_MMA=sync selects the warp-level mma.sync kernel (kept for comparison).
+bool prefill_use_mma_sync() {
+    static const bool v = [] {
+        const char* e = std::getenv("PA_PREFILL_MMA");
+        return e && std::strcmp(e, "sync") == 0;
+    }();
+    return v;
 }
 
 pa_status dispatch_prefill(int D, int G, const pa::PrefillParams& p, dim3 grid, cudaStream_t s) {
@@ -769,9 +827,13 @@ pa_status pa_prefill(const void* q, const int32_t* cu_q_lens, int32_t max_q_len,
     if (int64_t(d.num_seqs) * tiles > 0x7fffffffLL || d.num_kv_heads > 65535) return PA_ERR_SHAPE;
     pa::PrefillParams p;
     const int64_t cache_tiles = int64_t(d.num_blocks) * d.num_kv_heads;
-    if (!make_cache_map(&p.tmap_k, k_cache, cache_tiles, d.head_dim, d.block_size, 1) ||
-        !make_cache_map(&p.tmap_v, v_cache, cache_tiles, d.head_dim, d.block_size, 1))
-        return PA_ERR_CUDA;
+    const bool sync_mma = prefill_use_mma_sync();
+    const bool maps_ok =
+        sync_mma ? make_cache_map(&p.tmap_k, k_cache, cache_tiles, d.head_dim, d.block_size, 1) &&
+                       make_cache_map(&p.tmap_v, v_cache, cache_tiles, d.head_dim, d.block_size, 1)
+                 : make_panel_map(&p.tmap_k, k_cache, cache_tiles, d.head_dim, d.block_size) &&
+                       make_panel_map(&p.tmap_v, v_cache, cache_tiles, d.head_dim, d.block_size);
+    if (!maps_ok) return PA_ERR_CUDA;
     p.q = static_cast<const uint8_t*>(q);
     p.cu_q_lens = cu_q_lens;
     p.block_tables = block_tables;
@@ -784,8 +846,9 @@ pa_status pa_prefill(const void* q, const int32_t* cu_q_lens, int32_t max_q_len,
     p.M = d.max_blocks_per_seq;
     p.tiles_per_seq = int32_t(tiles);
     p.qscale = scale * kLog2e;
-    return dispatch_prefill(d.head_dim, G, p, dim3(unsigned(d.num_seqs * tiles), unsigned(d.num_kv_heads)),
-                            static_cast<cudaStream_t>(stream));
+    const dim3 grid(unsigned(d.num_seqs * tiles), unsigned(d.num_kv_heads));
+    return sync_mma ? dispatch_prefill(d.head_dim, G, p, grid, static_cast<cudaStream_t>(stream))
+                    : dispatch_prefill_tc(d.head_dim, G, p, grid, static_cast<cudaStream_t>(stream));
 }
 
 pa_status pa_device_errors(int32_t* errors_out, int32_t clear) {

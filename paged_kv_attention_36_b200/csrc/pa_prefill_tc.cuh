@@ -1,0 +1,357 @@
+// pa_prefill_tc.cuh -- multi-query (chunked prefill) attention over the paged
+// KV cache on the tcgen05 tensor cores.
+//
+// Same contract as prefill_kernel (pa_prefill.cuh): sequence b's last q_len_b
+// cached tokens are the query rows, row (token i, query head g*G + j) of kv
+// head g attends to the tokens at or before position L_b - q_len_b + i.  A CTA
+// owns 128 such rows (one M = 128 tile) of one (sequence, kv head) and walks
+// the sequence's pages in blocks of BN tokens (BN / 16 pages):
+//
+//   S_j = Q K_j^T        tcgen05.mma, A = Q (shared memory), B = K_j (shared
+//                        memory), fp32 accumulator in TMEM (two buffers, so
+//                        S_{j+1} is computed while S_j is in the softmax)
+//   P_j = 2^(S_j*c - m)  softmax warpgroup: thread i owns row i (TMEM lane i),
+//                        masks, keeps the running max m and sum l, writes P_j
+//                        as bf16 over the first half of S_j's columns
+//   O  += P_j V_j        tcgen05.mma, A = P_j (TMEM), B = V_j (shared memory,
+//                        MN-major), fp32 accumulator in TMEM, one MMA per page
+//
+// The running max is raised lazily: O and l are rescaled only when a row's
+// block maximum exceeds the max in use by more than 2^8 (P stays <= 256, well
+// inside bf16 and fp32), so most blocks skip the TMEM round trip of O.
+//
+// Warps: 0 streams K and V pages (one 2-D tiled TMA copy per page and 64-wide
+// panel) into a ring of KS blocks; 1 allocates TMEM and one of its threads
+// issues every MMA; 2-5 (one per TMEM lane quarter) load Q, run the softmax
+// and write the output.  Completion flows through mbarriers: TMA -> kv_full
+// -> MMA -> s_full -> softmax -> p_full -> MMA -> pv_done / kv_empty.
+//
+// The staged layout of a block is [D/64 panels][BN tokens][128 bytes] with the
+// 128-byte swizzle, for K and V alike: K is then the K-major B operand of
+// Q K^T (8-token groups 1024 bytes apart) and V the MN-major B operand of
+// P V (64-wide panels of head_dim BN*128 bytes apart).  Q has the same
+// [D/64][128 rows][128 bytes] layout.  V rows past the context in the
+// sequence's last page are zeroed in shared memory before P V reads them, so
+// an unused slot's bits (NaN included) cannot reach the output through a zero
+// probability.
+#pragma once
+
+#include "pa_prefill.cuh"
+#include "pa_tcgen05.cuh"
+
+namespace pa {
+
+template <int D, int BN, int KS>
+struct TcPrefillCfg {
+    static constexpr int kBM = 128;                 // query rows of a CTA
+    static constexpr int kPanels = D / 64;
+    static constexpr int kPanelQ = kBM * 128;       // bytes of one 64-wide panel of Q
+    static constexpr int kPanelKV = BN * 128;       // bytes of one 64-wide panel of a K or V block
+    static constexpr int kQBytes = kPanels * kPanelQ;
+    static constexpr int kKBytes = kPanels * kPanelKV;
+    static constexpr int kStage = 2 * kKBytes;      // K block then V block
+    static constexpr int kPages = BN / 16;          // pages per block
+    static constexpr int kPageBytes = 16 * D * 2;   // one (block, kv head) tile
+    static constexpr int kStageOff = kQBytes;
+    static constexpr int kBarOff = kStageOff + KS * kStage;
+    static constexpr int kNumBars = 1 + 2 * KS + 2 + 2 + 2 + 1;
+    static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;  // + TMEM slot, alignment slack
+    static constexpr int kThreads = 6 * 32;
+    static constexpr int kColsUsed = 2 * BN + D;   // S buffers, then O
+    static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
+                                   : kColsUsed <= 256 ? 256 : 512;
+    static_assert(BN % 64 == 0 && BN <= 256, "block of whole 64-token halves");
+    static_assert(kColsUsed <= 512, "TMEM columns");
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+    static_assert(kPanelKV % 1024 == 0 && kPanelQ % 1024 == 0, "swizzle atoms 1024-byte aligned");
+};
+
+template <int D, int G, int BN, int KS>
+__global__ void __launch_bounds__(6 * 32, 1) prefill_tc_kernel(const __grid_constant__ PrefillParams p) {
+    using Cfg = TcPrefillCfg<D, BN, KS>;
+    static_assert(Cfg::kBM % G == 0, "a tile holds whole tokens");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint8_t* qs = smem;
+    uint8_t* stages = smem + Cfg::kStageOff;
+    uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
+    uint64_t* kv_full = q_full + 1;
+    uint64_t* kv_empty = kv_full + KS;
+    uint64_t* s_full = kv_empty + KS;
+    uint64_t* p_full = s_full + 2;
+    uint64_t* pv_done = p_full + 2;
+    uint64_t* drain = pv_done + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    __shared__ int s_abort;
+    volatile int* abort = &s_abort;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = blockIdx.y;
+
+    // ---- the sequence, its query rows and the tokens this tile needs ----
+    const int b = int(blockIdx.x) / p.tiles_per_seq;
+    const int tile = int(blockIdx.x) - b * p.tiles_per_seq;
+    if (b >= p.B) return;
+    const bool report = tile == 0 && g == 0 && threadIdx.x == 0;
+    int32_t L = __ldg(p.context_lens + b);
+    const int64_t cap = int64_t(p.M) * 16;
+    if (L < 0 || L > cap) {
+        if (report) raise_error(PA_DEVERR_CONTEXT);
+        L = L < 0 ? 0 : int32_t(cap);
+    }
+    const int32_t q0 = __ldg(p.cu_q_lens + b);
+    int32_t q_len = __ldg(p.cu_q_lens + b + 1) - q0;
+    if (q_len < 0 || q_len > L) {  // queries must be cached tokens of the sequence
+        if (report) raise_error(PA_DEVERR_CONTEXT);
+        q_len = q_len < 0 ? 0 : L;
+    }
+    const int nrows = q_len * G;
+    const int row0 = tile * Cfg::kBM;
+    if (row0 >= nrows) return;  // whole CTA, before any barrier or TMEM use
+    const int first_pos = L - q_len;  // position of query token 0
+    const int last_row = (row0 + Cfg::kBM < nrows ? row0 + Cfg::kBM : nrows) - 1;
+    const int n_need = first_pos + last_row / G + 1;  // tokens 0 .. n_need-1 are visible to some row
+    const int pages = (n_need + 15) / 16;
+    const int nblk = (n_need + BN - 1) / BN;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 128);
+        for (int s = 0; s < KS; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&p_full[i], 128);
+            mbar_init(&pv_done[i], 1);
+        }
+        mbar_init(drain, 1);
+        s_abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, Cfg::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t t_o = tmem + 2 * BN;  // O columns; S buffer i at tmem + i*BN
+
+    if (warp == 0) {
+        // ======================= producer warp =======================
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_k)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_v)) : "memory");
+        }
+        const uint64_t pol = policy_evict_normal();  // the sequence's other row tiles read these pages too
+        const int32_t* bt = p.block_tables + int64_t(b) * p.M;
+        int j = 0;
+        for (; j < nblk; ++j) {
+            const int s = j % KS;
+            if (j >= KS && !__all_sync(0xffffffffu, mbar_wait(&kv_empty[s], uint32_t(j / KS - 1) & 1, abort)))
+                break;
+            const int pg0 = j * Cfg::kPages;
+            const int npg = pages - pg0 < Cfg::kPages ? pages - pg0 : Cfg::kPages;
+            if (lane == 0) mbar_arrive_expect_tx(&kv_full[s], uint32_t(npg * 2 * Cfg::kPageBytes));
+            __syncwarp();
+            if (lane < npg) {
+                int32_t blk = __ldg(bt + pg0 + lane);
+                if (blk < 0 || blk >= p.NB) {
+                    raise_error(PA_DEVERR_BLOCK_ID);
+                    blk = 0;
+                }
+                const int t = blk * p.Hkv + g;
+                uint8_t* kd = stages + s * Cfg::kStage + lane * 2048;
+#pragma unroll
+                for (int c = 0; c < Cfg::kPanels; ++c) {
+                    tma_load_4d(kd + c * Cfg::kPanelKV, &p.tmap_k, 0, 0, c, t, &kv_full[s], pol);
+                    tma_load_4d(kd + Cfg::kKBytes + c * Cfg::kPanelKV, &p.tmap_v, 0, 0, c, t, &kv_full[s], pol);
+                }
+            }
+        }
+        // every copy issued lands before shared memory is released
+        if (lane == 0)
+            for (int i = (j > KS ? j - KS : 0); i < j; ++i)
+                mbar_wait(&kv_full[i % KS], uint32_t(i / KS) & 1, nullptr, 20000000ull);
+    } else if (warp == 1) {
+        // ===================== MMA issue (one thread) =====================
+        if (lane == 0) {
+            constexpr uint32_t id_qk = idesc_bf16_f32(128, BN, false);
+            constexpr uint32_t id_pv = idesc_bf16_f32(128, D, true);
+            const uint32_t qa = smem_u32(qs);
+            const uint32_t st0 = smem_u32(stages);
+            bool ok = mbar_wait(q_full, 0, abort);
+            for (int j = 0; ok && j <= nblk; ++j) {
+                if (j < nblk) {
+                    const int s = j % KS, bb = j & 1;
+                    ok = mbar_wait(&kv_full[s], uint32_t(j / KS) & 1, abort);
+                    if (ok && j >= 2) ok = mbar_wait(&pv_done[bb], uint32_t((j - 2) >> 1) & 1, abort);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t kb = st0 + s * Cfg::kStage;
+#pragma unroll
+                    for (int c = 0; c < Cfg::kPanels; ++c)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_ss(tmem + bb * BN, sw128_desc(qa + c * Cfg::kPanelQ + kk * 32, 16, 1024),
+                                    sw128_desc(kb + c * Cfg::kPanelKV + kk * 32, 16, 1024), id_qk,
+                                    uint32_t(c | kk));
+                    umma_commit(&s_full[bb]);
+                }
+                if (j >= 1) {
+                    const int jp = j - 1, sp = jp % KS, bp = jp & 1;
+                    ok = mbar_wait(&p_full[bp], uint32_t(jp >> 1) & 1, abort);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const int npg = pages - jp * Cfg::kPages < Cfg::kPages ? pages - jp * Cfg::kPages : Cfg::kPages;
+                    const uint32_t vb = st0 + sp * Cfg::kStage + Cfg::kKBytes;
+                    for (int pg = 0; pg < npg; ++pg)
+                        umma_ts(t_o, tmem + bp * BN + pg * 8, sw128_desc(vb + pg * 2048, Cfg::kPanelKV, 1024), id_pv,
+                                uint32_t(jp | pg));
+                    umma_commit(&kv_empty[sp]);
+                    umma_commit(&pv_done[bp]);
+                }
+            }
+            // no MMA may still run when TMEM and shared memory are released
+            umma_commit(drain);
+            mbar_wait(drain, 0, nullptr, 20000000ull);
+        }
+        __syncwarp();
+    } else {
+        // ========================= softmax warpgroup =========================
+        const int qw = warp & 3;                // TMEM lane quarter of this warp
+        const int row = qw * 32 + lane;         // this thread's row of the tile
+        const int gt = (warp - 2) * 32 + lane;  // 0..127 within the warpgroup
+        const uint32_t lanes = uint32_t(qw * 32) << 16;
+        const int r = row0 + row;
+        const bool valid = r < nrows;
+        const int lim = valid ? first_pos + r / G + 1 : 1;  // keys 0 .. lim-1 are visible to this row
+        const int64_t orow = valid ? (int64_t(q0 + r / G) * p.Hq + g * G + r % G) * D : 0;
+
+        // Q row into shared memory (128-byte swizzle: 16-byte chunk c of row t at c ^ (t % 8))
+        {
+            const uint4* src = reinterpret_cast<const uint4*>(p.q + orow * 2);
+#pragma unroll
+            for (int ch = 0; ch < D / 8; ++ch) {
+                const uint4 v = valid ? __ldg(src + ch) : make_uint4(0u, 0u, 0u, 0u);
+                *reinterpret_cast<uint4*>(qs + (ch >> 3) * Cfg::kPanelQ + row * 128 + (((ch & 7) ^ (row & 7)) << 4)) =
+                    v;
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(q_full);
+        }
+
+        // the sequence's last page, when it is staged and ends inside the context
+        const int rem = L & 15;
+        const int last_pg = (L - 1) >> 4;
+        const int zero_blk = (rem != 0 && last_pg < pages) ? last_pg / Cfg::kPages : -1;
+
+        const float c = p.qscale;
+        float m = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nblk; ++j) {
+            const int bb = j & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[bb], uint32_t(j >> 1) & 1, abort));
+            if (!ok) break;
+            tc_fence_after();
+            float s[BN];
+#pragma unroll
+            for (int k = 0; k < BN / 32; ++k)
+                tmem_ld32(tmem + lanes + bb * BN + 32 * k, *reinterpret_cast<float(*)[32]>(&s[32 * k]));
+            // scaled logits (log2 units); keys past the row's position -> -inf
+            const int n0 = j * BN;
+#pragma unroll
+            for (int i = 0; i < BN; ++i) s[i] *= c;
+            if (n0 + BN > lim) {
+#pragma unroll
+                for (int i = 0; i < BN; ++i)
+                    if (n0 + i >= lim) s[i] = -INFINITY;
+            }
+            float m_blk = s[0];
+#pragma unroll
+            for (int i = 1; i < BN; ++i) m_blk = fmaxf(m_blk, s[i]);
+            const float m_new = fmaxf(m, m_blk);
+            if (__any_sync(0xffffffffu, m_new > m + 8.f)) {
+                const float alpha = ex2_approx(m - m_new);  // 0 while m = -inf
+                if (j > 0) {
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait(&pv_done[(j - 1) & 1], uint32_t((j - 1) >> 1) & 1, abort));
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < D / 32; ++k) {
+                        float o[32];
+                        tmem_ld32(t_o + lanes + 32 * k, o);
+                        uint32_t w[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(o[i] * alpha);
+                        tmem_st32(t_o + lanes + 32 * k, w);
+                    }
+                }
+                l *= alpha;
+                m = m_new;
+            }
+            // P = 2^(s*c - m) as bf16 pairs over the first BN/2 columns of the buffer
+            float sum = 0.f;
+#pragma unroll
+            for (int k = 0; k < BN / 64; ++k) {
+                uint32_t w[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float p0 = ex2_approx(s[64 * k + 2 * i] - m);
+                    const float p1 = ex2_approx(s[64 * k + 2 * i + 1] - m);
+                    sum += p0 + p1;
+                    w[i] = float2_to_bf16x2(p0, p1);
+                }
+                tmem_st32(tmem + lanes + bb * BN + 32 * k, w);
+            }
+            l += sum;
+            tmem_st_wait();
+            if (j == zero_blk) {
+                // V rows rem .. 15 of the last page hold no token of the context
+                uint8_t* vz = stages + (j % KS) * Cfg::kStage + Cfg::kKBytes + (last_pg % Cfg::kPages) * 2048;
+                const int pieces = (16 - rem) * 8;  // 16-byte pieces per panel
+                for (int i = gt; i < pieces * Cfg::kPanels; i += 128) {
+                    const int pc = i / pieces, rr = i - pc * pieces;
+                    *reinterpret_cast<uint4*>(vz + pc * Cfg::kPanelKV + (rem + (rr >> 3)) * 128 + ((rr & 7) << 4)) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+                fence_proxy_async_smem();
+            }
+            tc_fence_before();
+            mbar_arrive(&p_full[bb]);
+        }
+
+        // ---- output: O / l as bf16 ----
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(nblk - 1) & 1], uint32_t((nblk - 1) >> 1) & 1, abort));
+        if (ok) {
+            tc_fence_after();
+            const float inv = 1.f / l;
+            uint4* dst = reinterpret_cast<uint4*>(p.out + orow);
+#pragma unroll
+            for (int k = 0; k < D / 32; ++k) {
+                float o[32];
+                tmem_ld32(t_o + lanes + 32 * k, o);
+                if (valid) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[4 * k + q] = make_uint4(float2_to_bf16x2(o[8 * q] * inv, o[8 * q + 1] * inv),
+                                                    float2_to_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
+                                                    float2_to_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
+                                                    float2_to_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+                }
+            }
+        }
+    }
+
+    // ---- release TMEM once every warp's tcgen05 work has finished ----
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, Cfg::kTmemCols);
+    }
+}
+
+}  // namespace pa
