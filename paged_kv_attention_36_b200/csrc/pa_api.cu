@@ -376,18 +376,39 @@ pa_status launch_prefill(const pa::PrefillParams& p, dim3 grid, cudaStream_t str
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-// tcgen05 prefill: BN keys per block, KS blocks in the ring.
-constexpr int kTcBN = 128;
-template <int D> constexpr int tc_stages() { return D == 64 ? 4 : 3; }
+// tcgen05 prefill configurations: BN keys per block, KS blocks in the ring,
+// CPS CTAs per SM.
+template <int D, int BN> constexpr int tc_stages() {
+    return BN == 128 ? (D == 64 ? 4 : 3) : (D == 64 ? 5 : 2);
+}
 
-template <int D, int G>
+template <int D, int G, int BN>
 pa_status launch_prefill_tc(const pa::PrefillParams& p, dim3 grid, cudaStream_t stream) {
-    using Cfg = pa::TcPrefillCfg<D, kTcBN, tc_stages<D>()>;
-    auto kern = pa::prefill_tc_kernel<D, G, kTcBN, tc_stages<D>()>;
+    constexpr int KS = tc_stages<D, BN>(), CPS = BN == 128 ? 1 : 2;
+    // S buffers: as many as TMEM holds next to O for CPS CTAs per SM
+    constexpr int NS = (3 * BN + D) * CPS <= 512 ? 3 : 2;
+    using Cfg = pa::TcPrefillCfg<D, BN, KS, NS>;
+    static_assert(CPS * (Cfg::kSmemBytes + 1024) <= 233472, "CTAs per SM by shared memory");
+    static_assert(CPS * Cfg::kTmemCols <= 512, "CTAs per SM by TMEM columns");
+    auto kern = pa::prefill_tc_kernel<D, G, BN, KS, CPS, NS>;
     static unsigned attr_done[kMaxDevices];
     if (!set_smem_once(kern, Cfg::kSmemBytes, attr_done)) return PA_ERR_CUDA;
     kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+// PA_PREFILL_BN=64|128 picks the block size (keys per softmax step).
+int prefill_bn() {
+    static const int v = [] {
+        const char* e = std::getenv("PA_PREFILL_BN");
+        return (e && std::atoi(e) == 128) ? 128 : 64;
+    }();
+    return v;
+}
+
+template <int D, int G>
+pa_status launch_prefill_tc(const pa::PrefillParams& p, dim3 grid, cudaStream_t s) {
+    return prefill_bn() == 128 ? launch_prefill_tc<D, G, 128>(p, grid, s) : launch_prefill_tc<D, G, 64>(p, grid, s);
 }
 
 pa_status dispatch_prefill_tc(int D, int G, const pa::PrefillParams& p, dim3 grid, cudaStream_t s) {

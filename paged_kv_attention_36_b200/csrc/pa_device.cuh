@@ -88,6 +88,52 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// try_wait that suspends the thread (up to suspend_ns) until the phase
+// completes instead of returning at once.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+        : "memory");
+    return done != 0;
+}
+
+// mbar_wait for warps that share a scheduler with busy warps: the waiting
+// thread sleeps on the barrier rather than polling it, so it takes no issue
+// slots from them.  Same bound and abort behaviour as mbar_wait (abort is
+// seen within one suspension, <= 50 us).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                uint64_t limit_ns = kWaitLimitNs) {
+    if (mbar_test_wait(bar, parity)) return true;  // non-blocking probe: most waits are already satisfied
+    if (mbar_try_wait_suspend(bar, parity, 50000u)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait_suspend(bar, parity, 50000u)) return true;
+        if (abort && *abort) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            raise_error(PA_DEVERR_TIMEOUT);
+            if (abort) *abort = 1;
+            return false;
+        }
+    }
+}
+
 // ---- 1-D bulk copy global -> shared, completing on an mbarrier ------------
 // Both addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {

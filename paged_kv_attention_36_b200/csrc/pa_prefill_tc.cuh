@@ -8,7 +8,7 @@
 // the sequence's pages in blocks of BN tokens (BN / 16 pages):
 //
 //   S_j = Q K_j^T        tcgen05.mma, A = Q (shared memory), B = K_j (shared
-//                        memory), fp32 accumulator in TMEM (two buffers, so
+//                        memory), fp32 accumulator in TMEM (NS buffers, so
 //                        S_{j+1} is computed while S_j is in the softmax)
 //   P_j = 2^(S_j*c - m)  softmax warpgroup: thread i owns row i (TMEM lane i),
 //                        masks, keeps the running max m and sum l, writes P_j
@@ -20,11 +20,18 @@
 // block maximum exceeds the max in use by more than 2^8 (P stays <= 256, well
 // inside bf16 and fp32), so most blocks skip the TMEM round trip of O.
 //
+// CPS CTAs share an SM (TMEM columns and shared memory are sized for it),
+// so one CTA's prologue and epilogue overlap another's main loop.
+//
 // Warps: 0 streams K and V pages (one 2-D tiled TMA copy per page and 64-wide
 // panel) into a ring of KS blocks; 1 allocates TMEM and one of its threads
 // issues every MMA; 2-5 (one per TMEM lane quarter) load Q, run the softmax
-// and write the output.  Completion flows through mbarriers: TMA -> kv_full
-// -> MMA -> s_full -> softmax -> p_full -> MMA -> pv_done / kv_empty.
+// and write the output.  Completion flows through mbarriers: TMA -> k_full
+// -> MMA -> s_full -> softmax -> p_full (+ TMA -> v_full) -> MMA -> v_empty
+// (which also tells the softmax that O holds block j's P V).
+// K and V halves of a ring stage are refilled separately (k_empty once Q K^T
+// has read it, v_empty once P V has), and K is loaded one block ahead of V,
+// so each has a full softmax step more of lead than a shared stage would give.
 //
 // The staged layout of a block is [D/64 panels][BN tokens][128 bytes] with the
 // 128-byte swizzle, for K and V alike: K is then the K-major B operand of
@@ -41,7 +48,7 @@
 
 namespace pa {
 
-template <int D, int BN, int KS>
+template <int D, int BN, int KS, int NS>
 struct TcPrefillCfg {
     static constexpr int kBM = 128;                 // query rows of a CTA
     static constexpr int kPanels = D / 64;
@@ -54,10 +61,10 @@ struct TcPrefillCfg {
     static constexpr int kPageBytes = 16 * D * 2;   // one (block, kv head) tile
     static constexpr int kStageOff = kQBytes;
     static constexpr int kBarOff = kStageOff + KS * kStage;
-    static constexpr int kNumBars = 1 + 2 * KS + 2 + 2 + 2 + 1;
+    static constexpr int kNumBars = 1 + 4 * KS + 2 * NS + 1;
     static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;  // + TMEM slot, alignment slack
     static constexpr int kThreads = 6 * 32;
-    static constexpr int kColsUsed = 2 * BN + D;   // S buffers, then O
+    static constexpr int kColsUsed = NS * BN + D;  // S buffers, then O
     static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
                                    : kColsUsed <= 256 ? 256 : 512;
     static_assert(BN % 64 == 0 && BN <= 256, "block of whole 64-token halves");
@@ -66,21 +73,22 @@ struct TcPrefillCfg {
     static_assert(kPanelKV % 1024 == 0 && kPanelQ % 1024 == 0, "swizzle atoms 1024-byte aligned");
 };
 
-template <int D, int G, int BN, int KS>
-__global__ void __launch_bounds__(6 * 32, 1) prefill_tc_kernel(const __grid_constant__ PrefillParams p) {
-    using Cfg = TcPrefillCfg<D, BN, KS>;
+template <int D, int G, int BN, int KS, int CPS, int NS>
+__global__ void __launch_bounds__(6 * 32, CPS) prefill_tc_kernel(const __grid_constant__ PrefillParams p) {
+    using Cfg = TcPrefillCfg<D, BN, KS, NS>;
     static_assert(Cfg::kBM % G == 0, "a tile holds whole tokens");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* qs = smem;
     uint8_t* stages = smem + Cfg::kStageOff;
     uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
-    uint64_t* kv_full = q_full + 1;
-    uint64_t* kv_empty = kv_full + KS;
-    uint64_t* s_full = kv_empty + KS;
-    uint64_t* p_full = s_full + 2;
-    uint64_t* pv_done = p_full + 2;
-    uint64_t* drain = pv_done + 2;
+    uint64_t* k_full = q_full + 1;  // K and V halves of a stage fill and drain separately
+    uint64_t* v_full = k_full + KS;
+    uint64_t* k_empty = v_full + KS;
+    uint64_t* v_empty = k_empty + KS;
+    uint64_t* s_full = v_empty + KS;
+    uint64_t* p_full = s_full + NS;
+    uint64_t* drain = p_full + NS;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     __shared__ int s_abort;
     volatile int* abort = &s_abort;
@@ -116,13 +124,14 @@ __global__ void __launch_bounds__(6 * 32, 1) prefill_tc_kernel(const __grid_cons
     if (threadIdx.x == 0) {
         mbar_init(q_full, 128);
         for (int s = 0; s < KS; ++s) {
-            mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
+            mbar_init(&k_full[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+            mbar_init(&v_empty[s], 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NS; ++i) {
             mbar_init(&s_full[i], 1);
             mbar_init(&p_full[i], 128);
-            mbar_init(&pv_done[i], 1);
         }
         mbar_init(drain, 1);
         s_abort = 0;
@@ -136,7 +145,7 @@ __global__ void __launch_bounds__(6 * 32, 1) prefill_tc_kernel(const __grid_cons
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t t_o = tmem + 2 * BN;  // O columns; S buffer i at tmem + i*BN
+    const uint32_t t_o = tmem + NS * BN;  // O columns; S buffer i at tmem + i*BN
 
     if (warp == 0) {
         // ======================= producer warp =======================
@@ -146,80 +155,116 @@ __global__ void __launch_bounds__(6 * 32, 1) prefill_tc_kernel(const __grid_cons
         }
         const uint64_t pol = policy_evict_normal();  // the sequence's other row tiles read these pages too
         const int32_t* bt = p.block_tables + int64_t(b) * p.M;
-        int j = 0;
-        for (; j < nblk; ++j) {
+        // K of block j, or V: its stage half is free once the MMA that read
+        // it (Q K^T, or P V) has completed
+        auto load = [&](int j, bool v, int32_t blk) -> bool {
             const int s = j % KS;
-            if (j >= KS && !__all_sync(0xffffffffu, mbar_wait(&kv_empty[s], uint32_t(j / KS - 1) & 1, abort)))
-                break;
-            const int pg0 = j * Cfg::kPages;
-            const int npg = pages - pg0 < Cfg::kPages ? pages - pg0 : Cfg::kPages;
-            if (lane == 0) mbar_arrive_expect_tx(&kv_full[s], uint32_t(npg * 2 * Cfg::kPageBytes));
+            uint64_t* full = v ? &v_full[s] : &k_full[s];
+            if (j >= KS &&
+                !__all_sync(0xffffffffu, mbar_wait_sleep(v ? &v_empty[s] : &k_empty[s], uint32_t(j / KS - 1) & 1, abort)))
+                return false;
+            const int npg = pages - j * Cfg::kPages < Cfg::kPages ? pages - j * Cfg::kPages : Cfg::kPages;
+            if (lane == 0) mbar_arrive_expect_tx(full, uint32_t(npg * Cfg::kPageBytes));
             __syncwarp();
             if (lane < npg) {
-                int32_t blk = __ldg(bt + pg0 + lane);
                 if (blk < 0 || blk >= p.NB) {
                     raise_error(PA_DEVERR_BLOCK_ID);
                     blk = 0;
                 }
                 const int t = blk * p.Hkv + g;
-                uint8_t* kd = stages + s * Cfg::kStage + lane * 2048;
+                uint8_t* dst = stages + s * Cfg::kStage + (v ? Cfg::kKBytes : 0) + lane * 2048;
 #pragma unroll
-                for (int c = 0; c < Cfg::kPanels; ++c) {
-                    tma_load_4d(kd + c * Cfg::kPanelKV, &p.tmap_k, 0, 0, c, t, &kv_full[s], pol);
-                    tma_load_4d(kd + Cfg::kKBytes + c * Cfg::kPanelKV, &p.tmap_v, 0, 0, c, t, &kv_full[s], pol);
-                }
+                for (int c = 0; c < Cfg::kPanels; ++c)
+                    tma_load_4d(dst + c * Cfg::kPanelKV, v ? &p.tmap_v : &p.tmap_k, 0, 0, c, t, full, pol);
             }
+            return true;
+        };
+        // lane i's page of block t (read one block ahead, so the table load
+        // overlaps the waits)
+        auto page_of = [&](int t) -> int32_t {
+            const int pg = t * Cfg::kPages + lane;
+            return (t < nblk && lane < Cfg::kPages && pg < pages) ? __ldg(bt + pg) : 0;
+        };
+        // K runs one block ahead of V: V_j is read one softmax step after K_j
+        int nk = 0, nv = 0;  // blocks whose K (V) copies were issued
+        int32_t blk_cur = page_of(0), blk_prev = 0;
+        for (int t = 0; t <= nblk; ++t) {
+            const int32_t blk_next = page_of(t + 1);
+            if (t < nblk) {
+                if (!load(t, false, blk_cur)) break;
+                nk = t + 1;
+            }
+            if (t >= 1) {
+                if (!load(t - 1, true, blk_prev)) break;
+                nv = t;
+            }
+            blk_prev = blk_cur;
+            blk_cur = blk_next;
         }
         // every copy issued lands before shared memory is released
-        if (lane == 0)
-            for (int i = (j > KS ? j - KS : 0); i < j; ++i)
-                mbar_wait(&kv_full[i % KS], uint32_t(i / KS) & 1, nullptr, 20000000ull);
+        if (lane == 0) {
+            for (int i = (nk > KS ? nk - KS : 0); i < nk; ++i)
+                mbar_wait_sleep(&k_full[i % KS], uint32_t(i / KS) & 1, nullptr, 20000000ull);
+            for (int i = (nv > KS ? nv - KS : 0); i < nv; ++i)
+                mbar_wait_sleep(&v_full[i % KS], uint32_t(i / KS) & 1, nullptr, 20000000ull);
+        }
     } else if (warp == 1) {
         // ===================== MMA issue (one thread) =====================
         if (lane == 0) {
             constexpr uint32_t id_qk = idesc_bf16_f32(128, BN, false);
             constexpr uint32_t id_pv = idesc_bf16_f32(128, D, true);
-            const uint32_t qa = smem_u32(qs);
+            const uint64_t qd = sw128_desc(smem_u32(qs), 16, 1024);
             const uint32_t st0 = smem_u32(stages);
-            bool ok = mbar_wait(q_full, 0, abort);
-            for (int j = 0; ok && j <= nblk; ++j) {
-                if (j < nblk) {
-                    const int s = j % KS, bb = j & 1;
-                    ok = mbar_wait(&kv_full[s], uint32_t(j / KS) & 1, abort);
-                    if (ok && j >= 2) ok = mbar_wait(&pv_done[bb], uint32_t((j - 2) >> 1) & 1, abort);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t kb = st0 + s * Cfg::kStage;
+            bool ok = mbar_wait_sleep(q_full, 0, abort);
+            // S_i = Q K_i^T into buffer i % NS, once the P V that last read
+            // that buffer (block i - NS) has completed
+            auto issue_qk = [&](int i) -> bool {
+                const int s = i % KS, bb = i % NS;
+                if (!mbar_wait_sleep(&k_full[s], uint32_t(i / KS) & 1, abort)) return false;
+                if (i >= NS && !mbar_wait_sleep(&v_empty[(i - NS) % KS], uint32_t((i - NS) / KS) & 1, abort))
+                    return false;
+                tc_fence_after();
+                // descriptors advance by (byte offset >> 4) in their address field
+                const uint64_t kd = sw128_desc(st0 + s * Cfg::kStage, 16, 1024);
 #pragma unroll
-                    for (int c = 0; c < Cfg::kPanels; ++c)
+                for (int c = 0; c < Cfg::kPanels; ++c)
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma_ss(tmem + bb * BN, sw128_desc(qa + c * Cfg::kPanelQ + kk * 32, 16, 1024),
-                                    sw128_desc(kb + c * Cfg::kPanelKV + kk * 32, 16, 1024), id_qk,
-                                    uint32_t(c | kk));
-                    umma_commit(&s_full[bb]);
-                }
-                if (j >= 1) {
-                    const int jp = j - 1, sp = jp % KS, bp = jp & 1;
-                    ok = mbar_wait(&p_full[bp], uint32_t(jp >> 1) & 1, abort);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const int npg = pages - jp * Cfg::kPages < Cfg::kPages ? pages - jp * Cfg::kPages : Cfg::kPages;
-                    const uint32_t vb = st0 + sp * Cfg::kStage + Cfg::kKBytes;
-                    for (int pg = 0; pg < npg; ++pg)
-                        umma_ts(t_o, tmem + bp * BN + pg * 8, sw128_desc(vb + pg * 2048, Cfg::kPanelKV, 1024), id_pv,
-                                uint32_t(jp | pg));
-                    umma_commit(&kv_empty[sp]);
-                    umma_commit(&pv_done[bp]);
-                }
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_ss(tmem + bb * BN, qd + uint64_t((c * Cfg::kPanelQ + kk * 32) >> 4),
+                                kd + uint64_t((c * Cfg::kPanelKV + kk * 32) >> 4), id_qk, uint32_t(c | kk));
+                umma_commit(&s_full[bb]);
+                umma_commit(&k_empty[s]);
+                return true;
+            };
+            // S runs NS - 1 blocks ahead of P V.  With three or more buffers,
+            // block j's P V is issued as soon as P_j is in TMEM, then
+            // S_{j+NS-1} into the buffer P_{j-1} has released (its P V was
+            // issued one step earlier).  With two, S_{j+1} must wait for
+            // P_{j-1} V, so it is issued before waiting for P_j.
+            for (int i = 0; ok && i < NS - 1 && i < nblk; ++i) ok = issue_qk(i);
+            for (int j = 0; ok && j < nblk; ++j) {
+                if (NS == 2 && j + 1 < nblk && !(ok = issue_qk(j + 1))) break;
+                const int s = j % KS, bb = j % NS;
+                ok = mbar_wait_sleep(&p_full[bb], uint32_t(j / NS) & 1, abort) &&
+                     mbar_wait_sleep(&v_full[s], uint32_t(j / KS) & 1, abort);
+                if (!ok) break;
+                tc_fence_after();
+                const int npg = pages - j * Cfg::kPages < Cfg::kPages ? pages - j * Cfg::kPages : Cfg::kPages;
+                const uint64_t vd = sw128_desc(st0 + s * Cfg::kStage + Cfg::kKBytes, Cfg::kPanelKV, 1024);
+                const uint32_t pa = tmem + bb * BN;
+#pragma unroll
+                for (int pg = 0; pg < Cfg::kPages; ++pg)
+                    if (pg < npg) umma_ts(t_o, pa + pg * 8, vd + uint64_t(pg * (2048 >> 4)), id_pv, uint32_t(j | pg));
+                umma_commit(&v_empty[s]);
+                if (NS > 2 && j + NS - 1 < nblk) ok = issue_qk(j + NS - 1);
             }
             // no MMA may still run when TMEM and shared memory are released
             umma_commit(drain);
-            mbar_wait(drain, 0, nullptr, 20000000ull);
+            mbar_wait_sleep(drain, 0, nullptr, 20000000ull);
         }
         __syncwarp();
     } else {
-        // ========================= softmax warpgroup =========================
+        // ========================= softmax warpgroup ========================= =========================
         const int qw = warp & 3;                // TMEM lane quarter of this warp
         const int row = qw * 32 + lane;         // this thread's row of the tile
         const int gt = (warp - 2) * 32 + lane;  // 0..127 within the warpgroup
@@ -251,14 +296,13 @@ __global__ void __launch_bounds__(6 * 32, 1) prefill_tc_kernel(const __grid_cons
         float m = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < nblk; ++j) {
-            const int bb = j & 1;
-            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[bb], uint32_t(j >> 1) & 1, abort));
+            const int bb = j % NS;
+            ok = __all_sync(0xffffffffu, mbar_wait_sleep(&s_full[bb], uint32_t(j / NS) & 1, abort));
             if (!ok) break;
             tc_fence_after();
             float s[BN];
 #pragma unroll
-            for (int k = 0; k < BN / 32; ++k)
-                tmem_ld32(tmem + lanes + bb * BN + 32 * k, *reinterpret_cast<float(*)[32]>(&s[32 * k]));
+            for (int k = 0; k < BN / 64; ++k) tmem_ld64(tmem + lanes + bb * BN + 64 * k, &s[64 * k]);
             // scaled logits (log2 units); keys past the row's position -> -inf
             const int n0 = j * BN;
 #pragma unroll
@@ -268,15 +312,21 @@ __global__ void __launch_bounds__(6 * 32, 1) prefill_tc_kernel(const __grid_cons
                 for (int i = 0; i < BN; ++i)
                     if (n0 + i >= lim) s[i] = -INFINITY;
             }
-            float m_blk = s[0];
+            // row max and, below, row sum over 8 independent partials (no
+            // BN-long dependency chain)
+            float mp[8];
 #pragma unroll
-            for (int i = 1; i < BN; ++i) m_blk = fmaxf(m_blk, s[i]);
+            for (int u = 0; u < 8; ++u) mp[u] = s[u];
+#pragma unroll
+            for (int i = 8; i < BN; ++i) mp[i & 7] = fmaxf(mp[i & 7], s[i]);
+            const float m_blk = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                                      fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
             const float m_new = fmaxf(m, m_blk);
             if (__any_sync(0xffffffffu, m_new > m + 8.f)) {
                 const float alpha = ex2_approx(m - m_new);  // 0 while m = -inf
                 if (j > 0) {
                     ok = __all_sync(0xffffffffu,
-                                    mbar_wait(&pv_done[(j - 1) & 1], uint32_t((j - 1) >> 1) & 1, abort));
+                                    mbar_wait_sleep(&v_empty[(j - 1) % KS], uint32_t((j - 1) / KS) & 1, abort));
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll
@@ -293,7 +343,7 @@ __global__ void __launch_bounds__(6 * 32, 1) prefill_tc_kernel(const __grid_cons
                 m = m_new;
             }
             // P = 2^(s*c - m) as bf16 pairs over the first BN/2 columns of the buffer
-            float sum = 0.f;
+            float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int k = 0; k < BN / 64; ++k) {
                 uint32_t w[32];
@@ -301,15 +351,18 @@ __global__ void __launch_bounds__(6 * 32, 1) prefill_tc_kernel(const __grid_cons
                 for (int i = 0; i < 32; ++i) {
                     const float p0 = ex2_approx(s[64 * k + 2 * i] - m);
                     const float p1 = ex2_approx(s[64 * k + 2 * i + 1] - m);
-                    sum += p0 + p1;
+                    sp[(2 * i) & 7] += p0;
+                    sp[(2 * i + 1) & 7] += p1;
                     w[i] = float2_to_bf16x2(p0, p1);
                 }
                 tmem_st32(tmem + lanes + bb * BN + 32 * k, w);
             }
-            l += sum;
+            l += ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
             tmem_st_wait();
             if (j == zero_blk) {
                 // V rows rem .. 15 of the last page hold no token of the context
+                ok = __all_sync(0xffffffffu, mbar_wait_sleep(&v_full[j % KS], uint32_t(j / KS) & 1, abort));
+                if (!ok) break;
                 uint8_t* vz = stages + (j % KS) * Cfg::kStage + Cfg::kKBytes + (last_pg % Cfg::kPages) * 2048;
                 const int pieces = (16 - rem) * 8;  // 16-byte pieces per panel
                 for (int i = gt; i < pieces * Cfg::kPanels; i += 128) {
@@ -324,19 +377,21 @@ __global__ void __launch_bounds__(6 * 32, 1) prefill_tc_kernel(const __grid_cons
         }
 
         // ---- output: O / l as bf16 ----
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(nblk - 1) & 1], uint32_t((nblk - 1) >> 1) & 1, abort));
+        if (ok)
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait_sleep(&v_empty[(nblk - 1) % KS], uint32_t((nblk - 1) / KS) & 1, abort));
         if (ok) {
             tc_fence_after();
             const float inv = 1.f / l;
             uint4* dst = reinterpret_cast<uint4*>(p.out + orow);
 #pragma unroll
-            for (int k = 0; k < D / 32; ++k) {
-                float o[32];
-                tmem_ld32(t_o + lanes + 32 * k, o);
+            for (int k = 0; k < D / 64; ++k) {
+                float o[64];
+                tmem_ld64(t_o + lanes + 64 * k, o);
                 if (valid) {
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        dst[4 * k + q] = make_uint4(float2_to_bf16x2(o[8 * q] * inv, o[8 * q + 1] * inv),
+                    for (int q = 0; q < 8; ++q)
+                        dst[8 * k + q] = make_uint4(float2_to_bf16x2(o[8 * q] * inv, o[8 * q + 1] * inv),
                                                     float2_to_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
                                                     float2_to_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
                                                     float2_to_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
