@@ -303,6 +303,71 @@ pa_status dispatch_decode(int D, int G, const pa::DecodeParams& p, int grid, cud
                                          : dispatch_d_g<MathKind::kSimt, DUMP, APPEND>(D, G, p, grid, s, pdl);
 }
 
+// tcgen05 prefill configurations: BN keys per block, KS blocks in the ring,
+// CPS CTAs per SM.
+template <int D, int BN> constexpr int tc_stages() {
+    return BN == 128 ? (D == 64 ? 4 : 3) : (D == 64 ? 5 : 2);
+}
+
+template <int D, int BN>
+struct TcShape {
+    static constexpr int KS = tc_stages<D, BN>(), CPS = BN == 128 ? 1 : 2;
+    // S buffers: as many as TMEM holds next to O for CPS CTAs per SM
+    static constexpr int NS = (3 * BN + D) * CPS <= 512 ? 3 : 2;
+    using Cfg = pa::TcPrefillCfg<D, BN, KS, NS>;
+    static_assert(CPS * (Cfg::kSmemBytes + 1024) <= 233472, "CTAs per SM by shared memory");
+    static_assert(CPS * Cfg::kTmemCols <= 512, "CTAs per SM by TMEM columns");
+};
+
+template <int D, int G, int BN>
+pa_status launch_prefill_tc(const pa::PrefillParams& p, dim3 grid, cudaStream_t stream) {
+    using S = TcShape<D, BN>;
+    auto kern = pa::prefill_tc_kernel<D, G, BN, S::KS, S::CPS, S::NS>;
+    static unsigned attr_done[kMaxDevices];
+    if (!set_smem_once(kern, S::Cfg::kSmemBytes, attr_done)) return PA_ERR_CUDA;
+    kern<<<grid, S::Cfg::kThreads, S::Cfg::kSmemBytes, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <int D, int G, int BN>
+pa_status launch_prefix_tc(const pa::PrefixParams& p, dim3 grid, cudaStream_t stream) {
+    using S = TcShape<D, BN>;
+    auto kern = pa::prefix_tc_kernel<D, G, BN, S::KS, S::CPS, S::NS>;
+    static unsigned attr_done[kMaxDevices];
+    if (!set_smem_once(kern, S::Cfg::kSmemBytes, attr_done)) return PA_ERR_CUDA;
+    kern<<<grid, S::Cfg::kThreads, S::Cfg::kSmemBytes, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+// PA_PREFILL_BN=64|128 picks the block size (keys per softmax step).
+int prefill_bn() {
+    static const int v = [] {
+        const char* e = std::getenv("PA_PREFILL_BN");
+        return (e && std::atoi(e) == 128) ? 128 : 64;
+    }();
+    return v;
+}
+
+template <int D, int G>
+pa_status launch_prefill_tc(const pa::PrefillParams& p, dim3 grid, cudaStream_t s) {
+    return prefill_bn() == 128 ? launch_prefill_tc<D, G, 128>(p, grid, s) : launch_prefill_tc<D, G, 64>(p, grid, s);
+}
+
+template <int D, int G>
+pa_status launch_prefix_tc(const pa::PrefixParams& p, dim3 grid, cudaStream_t s) {
+    return prefill_bn() == 128 ? launch_prefix_tc<D, G, 128>(p, grid, s) : launch_prefix_tc<D, G, 64>(p, grid, s);
+}
+
+// PA_PREFILL_MMA=sync selects the warp-level mma.sync kernels (prefill and
+// shared-prefix pass; kept for comparison).
+bool prefill_use_mma_sync() {
+    static const bool v = [] {
+        const char* e = std::getenv("PA_PREFILL_MMA");
+        return e && std::strcmp(e, "sync") == 0;
+    }();
+    return v;
+}
+
 // ---- shared-prefix pass ----------------------------------------------------
 constexpr int kPrefixNW = 8;      // consumer warps: 128 query rows per CTA
 constexpr int kPrefixStages = 8;  // ring of K+V pages
@@ -346,7 +411,27 @@ pa_status launch_prefix(const pa::PrefixParams& p, dim3 grid, cudaStream_t strea
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+pa_status dispatch_prefix_tc(int D, int G, const pa::PrefixParams& p, dim3 grid, cudaStream_t s) {
+    if (D == 64) {
+        switch (G) {
+            case 1: return launch_prefix_tc<64, 1>(p, grid, s);
+            case 2: return launch_prefix_tc<64, 2>(p, grid, s);
+            case 4: return launch_prefix_tc<64, 4>(p, grid, s);
+            case 8: return launch_prefix_tc<64, 8>(p, grid, s);
+        }
+    } else if (D == 128) {
+        switch (G) {
+            case 1: return launch_prefix_tc<128, 1>(p, grid, s);
+            case 2: return launch_prefix_tc<128, 2>(p, grid, s);
+            case 4: return launch_prefix_tc<128, 4>(p, grid, s);
+            case 8: return launch_prefix_tc<128, 8>(p, grid, s);
+        }
+    }
+    return PA_ERR_UNSUPPORTED;
+}
+
 pa_status dispatch_prefix(int D, int G, const pa::PrefixParams& p, dim3 grid, cudaStream_t s) {
+    if (!prefill_use_mma_sync()) return dispatch_prefix_tc(D, G, p, grid, s);
     if (D == 64) {
         switch (G) {
             case 1: return launch_prefix<64, 1>(p, grid, s);
@@ -376,41 +461,6 @@ pa_status launch_prefill(const pa::PrefillParams& p, dim3 grid, cudaStream_t str
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-// tcgen05 prefill configurations: BN keys per block, KS blocks in the ring,
-// CPS CTAs per SM.
-template <int D, int BN> constexpr int tc_stages() {
-    return BN == 128 ? (D == 64 ? 4 : 3) : (D == 64 ? 5 : 2);
-}
-
-template <int D, int G, int BN>
-pa_status launch_prefill_tc(const pa::PrefillParams& p, dim3 grid, cudaStream_t stream) {
-    constexpr int KS = tc_stages<D, BN>(), CPS = BN == 128 ? 1 : 2;
-    // S buffers: as many as TMEM holds next to O for CPS CTAs per SM
-    constexpr int NS = (3 * BN + D) * CPS <= 512 ? 3 : 2;
-    using Cfg = pa::TcPrefillCfg<D, BN, KS, NS>;
-    static_assert(CPS * (Cfg::kSmemBytes + 1024) <= 233472, "CTAs per SM by shared memory");
-    static_assert(CPS * Cfg::kTmemCols <= 512, "CTAs per SM by TMEM columns");
-    auto kern = pa::prefill_tc_kernel<D, G, BN, KS, CPS, NS>;
-    static unsigned attr_done[kMaxDevices];
-    if (!set_smem_once(kern, Cfg::kSmemBytes, attr_done)) return PA_ERR_CUDA;
-    kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(p);
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
-}
-
-// PA_PREFILL_BN=64|128 picks the block size (keys per softmax step).
-int prefill_bn() {
-    static const int v = [] {
-        const char* e = std::getenv("PA_PREFILL_BN");
-        return (e && std::atoi(e) == 128) ? 128 : 64;
-    }();
-    return v;
-}
-
-template <int D, int G>
-pa_status launch_prefill_tc(const pa::PrefillParams& p, dim3 grid, cudaStream_t s) {
-    return prefill_bn() == 128 ? launch_prefill_tc<D, G, 128>(p, grid, s) : launch_prefill_tc<D, G, 64>(p, grid, s);
-}
-
 pa_status dispatch_prefill_tc(int D, int G, const pa::PrefillParams& p, dim3 grid, cudaStream_t s) {
     if (D == 64) {
         switch (G) {
@@ -428,15 +478,6 @@ pa_status dispatch_prefill_tc(int D, int G, const pa::PrefillParams& p, dim3 gri
         }
     }
     return PA_ERR_UNSUPPORTED;
-}
-
-// PA_PREFILL_MMA=sync selects the warp-level mma.sync kernel (kept for comparison).
-bool prefill_use_mma_sync() {
-    static const bool v = [] {
-        const char* e = std::getenv("PA_PREFILL_MMA");
-        return e && std::strcmp(e, "sync") == 0;
-    }();
-    return v;
 }
 
 pa_status dispatch_prefill(int D, int G, const pa::PrefillParams& p, dim3 grid, cudaStream_t s) {
@@ -707,8 +748,13 @@ pa_status pa_decode_shared_prefix(const void* k_new, const void* v_new, const in
         uint8_t* ws = static_cast<uint8_t*>(workspace);
         pa::PrefixParams pp;
         const int64_t cache_tiles = int64_t(d.num_blocks) * d.num_kv_heads;
-        if (!make_cache_map(&pp.tmap_k, k_cache, cache_tiles, d.head_dim, d.block_size, 1) ||
-            !make_cache_map(&pp.tmap_v, v_cache, cache_tiles, d.head_dim, d.block_size, 1))
+        const bool maps_ok =
+            prefill_use_mma_sync()
+                ? make_cache_map(&pp.tmap_k, k_cache, cache_tiles, d.head_dim, d.block_size, 1) &&
+                      make_cache_map(&pp.tmap_v, v_cache, cache_tiles, d.head_dim, d.block_size, 1)
+                : make_panel_map(&pp.tmap_k, k_cache, cache_tiles, d.head_dim, d.block_size) &&
+                      make_panel_map(&pp.tmap_v, v_cache, cache_tiles, d.head_dim, d.block_size);
+        if (!maps_ok)
             return PA_ERR_CUDA;
         pp.q = p.q;
         pp.block_tables = block_tables;

@@ -73,10 +73,14 @@ struct TcPrefillCfg {
     static_assert(kPanelKV % 1024 == 0 && kPanelQ % 1024 == 0, "swizzle atoms 1024-byte aligned");
 };
 
-template <int D, int G, int BN, int KS, int CPS, int NS>
-__global__ void __launch_bounds__(6 * 32, CPS) prefill_tc_kernel(const __grid_constant__ PrefillParams p) {
+// One CTA's 128-row tile.  PREFIX = false: rows of sequence b's query tokens
+// against its own pages, causal (PrefillParams, bf16 output).  PREFIX = true:
+// rows (member, query head) of a shared-prefix group against one key split
+// of the group's shared pages, all visible (PrefixParams, fp32 partials).
+template <bool PREFIX, int D, int G, int BN, int KS, int NS, class Params>
+__device__ __forceinline__ void tc_attention_tile(const Params& p) {
     using Cfg = TcPrefillCfg<D, BN, KS, NS>;
-    static_assert(Cfg::kBM % G == 0, "a tile holds whole tokens");
+    static_assert(Cfg::kBM % G == 0, "a tile holds whole tokens (members)");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* qs = smem;
@@ -95,31 +99,61 @@ __global__ void __launch_bounds__(6 * 32, CPS) prefill_tc_kernel(const __grid_co
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = blockIdx.y;
 
-    // ---- the sequence, its query rows and the tokens this tile needs ----
-    const int b = int(blockIdx.x) / p.tiles_per_seq;
-    const int tile = int(blockIdx.x) - b * p.tiles_per_seq;
-    if (b >= p.B) return;
-    const bool report = tile == 0 && g == 0 && threadIdx.x == 0;
-    int32_t L = __ldg(p.context_lens + b);
-    const int64_t cap = int64_t(p.M) * 16;
-    if (L < 0 || L > cap) {
-        if (report) raise_error(PA_DEVERR_CONTEXT);
-        L = L < 0 ? 0 : int32_t(cap);
+    // ---- this tile's rows and the key pages it attends ----
+    int nrows, row0, nkeys;  // rows of the task, the tile's first row, keys staged (0 .. nkeys-1)
+    const int32_t* bt;       // block-table entries of the staged pages
+    int L = 0, q0 = 0, first_pos = 0, first = 0, P = 0, pg0 = 0;
+    if constexpr (!PREFIX) {
+        const int b = int(blockIdx.x) / p.tiles_per_seq;
+        const int tile = int(blockIdx.x) - b * p.tiles_per_seq;
+        if (b >= p.B) return;
+        const bool report = tile == 0 && g == 0 && threadIdx.x == 0;
+        L = __ldg(p.context_lens + b);
+        const int64_t cap = int64_t(p.M) * 16;
+        if (L < 0 || L > cap) {
+            if (report) raise_error(PA_DEVERR_CONTEXT);
+            L = L < 0 ? 0 : int32_t(cap);
+        }
+        q0 = __ldg(p.cu_q_lens + b);
+        int32_t q_len = __ldg(p.cu_q_lens + b + 1) - q0;
+        if (q_len < 0 || q_len > L) {  // queries must be cached tokens of the sequence
+            if (report) raise_error(PA_DEVERR_CONTEXT);
+            q_len = q_len < 0 ? 0 : L;
+        }
+        nrows = q_len * G;
+        row0 = tile * Cfg::kBM;
+        if (row0 >= nrows) return;  // whole CTA, before any barrier or TMEM use
+        first_pos = L - q_len;      // position of query token 0
+        const int last_row = (row0 + Cfg::kBM < nrows ? row0 + Cfg::kBM : nrows) - 1;
+        nkeys = first_pos + last_row / G + 1;  // tokens 0 .. nkeys-1 are visible to some row
+        bt = p.block_tables + int64_t(b) * p.M;
+    } else {
+        const int gi = int(blockIdx.x) / p.tiles_per_group;
+        const int tile = int(blockIdx.x) - gi * p.tiles_per_group;
+        if (gi >= p.num_groups) return;
+        first = __ldg(p.group_offsets + gi);
+        int last = __ldg(p.group_offsets + gi + 1);
+        P = __ldg(p.group_prefix_pages + gi);
+        const bool report = tile == 0 && g == 0 && blockIdx.z == 0 && threadIdx.x == 0;
+        if (first < 0 || last > p.B || last < first || last - first > p.max_group_size || P > p.M) {
+            if (report) raise_error(PA_DEVERR_PREFIX);
+            first = first < 0 ? 0 : (first > p.B ? p.B : first);
+            last = last < first ? first : (last > p.B ? p.B : last);
+            if (last - first > p.max_group_size) last = first + p.max_group_size;
+            if (P > p.M) P = p.M;
+        }
+        nrows = (last - first) * G;
+        row0 = tile * Cfg::kBM;
+        if (P <= 0 || row0 >= nrows) return;
+        const int per = prefix_split_pages(P, gridDim.z);
+        pg0 = int(blockIdx.z) * per;
+        const int pg1 = pg0 + per < P ? pg0 + per : P;
+        if (pg0 >= pg1) return;
+        nkeys = (pg1 - pg0) * 16;  // shared pages are whole
+        bt = p.block_tables + int64_t(first) * p.M + pg0;  // the group leader's table
     }
-    const int32_t q0 = __ldg(p.cu_q_lens + b);
-    int32_t q_len = __ldg(p.cu_q_lens + b + 1) - q0;
-    if (q_len < 0 || q_len > L) {  // queries must be cached tokens of the sequence
-        if (report) raise_error(PA_DEVERR_CONTEXT);
-        q_len = q_len < 0 ? 0 : L;
-    }
-    const int nrows = q_len * G;
-    const int row0 = tile * Cfg::kBM;
-    if (row0 >= nrows) return;  // whole CTA, before any barrier or TMEM use
-    const int first_pos = L - q_len;  // position of query token 0
-    const int last_row = (row0 + Cfg::kBM < nrows ? row0 + Cfg::kBM : nrows) - 1;
-    const int n_need = first_pos + last_row / G + 1;  // tokens 0 .. n_need-1 are visible to some row
-    const int pages = (n_need + 15) / 16;
-    const int nblk = (n_need + BN - 1) / BN;
+    const int pages = (nkeys + 15) / 16;
+    const int nblk = (nkeys + BN - 1) / BN;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 128);
@@ -154,7 +188,6 @@ __global__ void __launch_bounds__(6 * 32, CPS) prefill_tc_kernel(const __grid_co
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_v)) : "memory");
         }
         const uint64_t pol = policy_evict_normal();  // the sequence's other row tiles read these pages too
-        const int32_t* bt = p.block_tables + int64_t(b) * p.M;
         // K of block j, or V: its stage half is free once the MMA that read
         // it (Q K^T, or P V) has completed
         auto load = [&](int j, bool v, int32_t blk) -> bool {
@@ -264,15 +297,17 @@ __global__ void __launch_bounds__(6 * 32, CPS) prefill_tc_kernel(const __grid_co
         }
         __syncwarp();
     } else {
-        // ========================= softmax warpgroup ========================= =========================
+        // ========================= softmax warpgroup =========================
         const int qw = warp & 3;                // TMEM lane quarter of this warp
         const int row = qw * 32 + lane;         // this thread's row of the tile
         const int gt = (warp - 2) * 32 + lane;  // 0..127 within the warpgroup
         const uint32_t lanes = uint32_t(qw * 32) << 16;
         const int r = row0 + row;
         const bool valid = r < nrows;
-        const int lim = valid ? first_pos + r / G + 1 : 1;  // keys 0 .. lim-1 are visible to this row
-        const int64_t orow = valid ? (int64_t(q0 + r / G) * p.Hq + g * G + r % G) * D : 0;
+        // keys 0 .. lim-1 are visible to this row; its query and output row
+        const int lim = PREFIX ? nkeys : (valid ? first_pos + r / G + 1 : 1);
+        const int64_t qrow = int64_t(PREFIX ? first : q0) + r / G;
+        const int64_t orow = valid ? (qrow * p.Hq + g * G + r % G) * D : 0;
 
         // Q row into shared memory (128-byte swizzle: 16-byte chunk c of row t at c ^ (t % 8))
         {
@@ -290,7 +325,7 @@ __global__ void __launch_bounds__(6 * 32, CPS) prefill_tc_kernel(const __grid_co
         // the sequence's last page, when it is staged and ends inside the context
         const int rem = L & 15;
         const int last_pg = (L - 1) >> 4;
-        const int zero_blk = (rem != 0 && last_pg < pages) ? last_pg / Cfg::kPages : -1;
+        const int zero_blk = (!PREFIX && rem != 0 && last_pg < pages) ? last_pg / Cfg::kPages : -1;
 
         const float c = p.qscale;
         float m = -INFINITY, l = 0.f;
@@ -383,18 +418,55 @@ __global__ void __launch_bounds__(6 * 32, CPS) prefill_tc_kernel(const __grid_co
         if (ok) {
             tc_fence_after();
             const float inv = 1.f / l;
-            uint4* dst = reinterpret_cast<uint4*>(p.out + orow);
+            if constexpr (!PREFIX) {
+                // bf16 output row
+                uint4* dst = reinterpret_cast<uint4*>(p.out + orow);
 #pragma unroll
-            for (int k = 0; k < D / 64; ++k) {
-                float o[64];
-                tmem_ld64(t_o + lanes + 64 * k, o);
-                if (valid) {
+                for (int k = 0; k < D / 64; ++k) {
+                    float o[64];
+                    tmem_ld64(t_o + lanes + 64 * k, o);
+                    if (valid) {
 #pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        dst[8 * k + q] = make_uint4(float2_to_bf16x2(o[8 * q] * inv, o[8 * q + 1] * inv),
-                                                    float2_to_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
-                                                    float2_to_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
-                                                    float2_to_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+                        for (int q = 0; q < 8; ++q)
+                            dst[8 * k + q] = make_uint4(float2_to_bf16x2(o[8 * q] * inv, o[8 * q + 1] * inv),
+                                                        float2_to_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
+                                                        float2_to_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
+                                                        float2_to_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+                    }
+                }
+            } else {
+                // this split's partial: normalised output, (max logit in base 2, exp-sum)
+                const int64_t idx = (int64_t(blockIdx.z) * p.B + qrow) * p.Hq + g * G + r % G;
+                float4* dst = reinterpret_cast<float4*>(p.prefix_o + idx * D);
+#pragma unroll
+                for (int k = 0; k < D / 64; ++k) {
+                    float o[64];
+                    tmem_ld64(t_o + lanes + 64 * k, o);
+                    if (valid) {
+#pragma unroll
+                        for (int q = 0; q < 16; ++q)
+                            dst[16 * k + q] = make_float4(o[4 * q] * inv, o[4 * q + 1] * inv, o[4 * q + 2] * inv,
+                                                          o[4 * q + 3] * inv);
+                    }
+                }
+                if (valid) p.prefix_ml[idx] = make_float2(m, l);
+            }
+        }
+        if constexpr (PREFIX) {
+            // checks of the caller's grouping (kv head 0 only): each member of
+            // the tile holds the split's prefix blocks in its own table and
+            // its context covers the whole prefix
+            if (g == 0) {
+                const int npg = nkeys / 16;
+                const int m_lo = row0 / G;
+                const int m_hi = ((row0 + Cfg::kBM < nrows ? row0 + Cfg::kBM : nrows) + G - 1) / G;
+                for (int x = gt; x < (m_hi - m_lo) * npg; x += 128) {
+                    const int mem = first + m_lo + x / npg;
+                    const int j = pg0 + x % npg;
+                    if (__ldg(p.block_tables + int64_t(mem) * p.M + j) != __ldg(bt + (j - pg0)))
+                        raise_error(PA_DEVERR_PREFIX);
+                    if (x % npg == 0 && int64_t(__ldg(p.context_lens + mem)) < int64_t(P) * 16)
+                        raise_error(PA_DEVERR_PREFIX);
                 }
             }
         }
@@ -407,6 +479,22 @@ __global__ void __launch_bounds__(6 * 32, CPS) prefill_tc_kernel(const __grid_co
         tc_fence_after();
         tmem_dealloc(tmem, Cfg::kTmemCols);
     }
+}
+
+template <int D, int G, int BN, int KS, int CPS, int NS>
+__global__ void __launch_bounds__(6 * 32, CPS) prefill_tc_kernel(const __grid_constant__ PrefillParams p) {
+    tc_attention_tile<false, D, G, BN, KS, NS>(p);
+}
+
+// The shared-prefix (cascade) pass on tcgen05: grid (group x row tile, kv
+// head, key split); each CTA also copies its slice of the step's append.
+template <int D, int G, int BN, int KS, int CPS, int NS>
+__global__ void __launch_bounds__(6 * 32, CPS) prefix_tc_kernel(const __grid_constant__ PrefixParams p) {
+    // the decode launched after this kernel may start its set-up now; it
+    // waits for this grid to complete before it reads anything written here
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    prefix_append_slice<D>(p, 6 * 32);
+    tc_attention_tile<true, D, G, BN, KS, NS>(p);
 }
 
 }  // namespace pa

@@ -189,6 +189,35 @@ struct PrefixParams {
     uint4* v_cache_w;
 };
 
+// This CTA's slice of the step's slot-mapped append (a bit copy of 16-byte
+// chunks; the rows land in the members' own blocks, never in the shared
+// ones), done by the shared-prefix pass so that the decode after it sees them.
+template <int D>
+__device__ __forceinline__ void prefix_append_slice(const PrefixParams& p, int nthreads) {
+    if (p.app_chunks <= 0) return;
+    const int64_t ncta = int64_t(gridDim.x) * gridDim.y * gridDim.z;
+    const int64_t lin = (int64_t(blockIdx.z) * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+    const int64_t per = (p.app_chunks + ncta - 1) / ncta;
+    const int64_t c0 = lin * per;
+    const int64_t c1 = c0 + per < p.app_chunks ? c0 + per : p.app_chunks;
+    constexpr int CPR = D / 8;  // 16-byte chunks per row
+    for (int64_t idx = c0 + threadIdx.x; idx < c1; idx += nthreads) {
+        const int64_t t = idx / (int64_t(p.Hkv) * CPR);
+        const int64_t rem = idx - t * p.Hkv * CPR;
+        const int32_t slot = __ldg(p.slot_mapping + t);
+        if (slot < 0) continue;
+        const int64_t block = slot / 16, offset = slot - (slot / 16) * 16;
+        if (block >= p.NB) {
+            if (rem == 0) raise_error(PA_DEVERR_SLOT);
+            continue;
+        }
+        const int64_t gg = rem / CPR, c = rem - gg * CPR;
+        const int64_t dst = ((block * p.Hkv + gg) * 16 + offset) * CPR + c;
+        p.k_cache_w[dst] = __ldg(p.k_new + idx);
+        p.v_cache_w[dst] = __ldg(p.v_new + idx);
+    }
+}
+
 template <int D, int NW, int RS>
 struct PrefixCfg {
     static constexpr int kRow = D * 2;
@@ -224,31 +253,7 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) prefix_kernel(const __grid_c
     // waits for this grid to complete before it reads anything written here.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-    if (p.app_chunks > 0) {
-        // this CTA's slice of the append (a bit copy of 16-byte chunks; the
-        // rows land in the members' own blocks, never in the shared ones)
-        const int64_t ncta = int64_t(gridDim.x) * gridDim.y * gridDim.z;
-        const int64_t lin = (int64_t(blockIdx.z) * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
-        const int64_t per = (p.app_chunks + ncta - 1) / ncta;
-        const int64_t c0 = lin * per;
-        const int64_t c1 = c0 + per < p.app_chunks ? c0 + per : p.app_chunks;
-        constexpr int CPR = D / 8;  // 16-byte chunks per row
-        for (int64_t idx = c0 + threadIdx.x; idx < c1; idx += Cfg::kThreads) {
-            const int64_t t = idx / (int64_t(p.Hkv) * CPR);
-            const int64_t rem = idx - t * p.Hkv * CPR;
-            const int32_t slot = __ldg(p.slot_mapping + t);
-            if (slot < 0) continue;
-            const int64_t block = slot / 16, offset = slot - (slot / 16) * 16;
-            if (block >= p.NB) {
-                if (rem == 0) raise_error(PA_DEVERR_SLOT);
-                continue;
-            }
-            const int64_t gg = rem / CPR, c = rem - gg * CPR;
-            const int64_t dst = ((block * p.Hkv + gg) * 16 + offset) * CPR + c;
-            p.k_cache_w[dst] = __ldg(p.k_new + idx);
-            p.v_cache_w[dst] = __ldg(p.v_new + idx);
-        }
-    }
+    prefix_append_slice<D>(p, Cfg::kThreads);
 
     // ---- the group, its members and this CTA's rows and pages ----
     const int gi = int(blockIdx.x) / p.tiles_per_group;
