@@ -218,7 +218,7 @@ PA_API pa_status pa_decode_static_ws(const void* q, const void* k_cache, const v
  * whose block_tables rows all begin with the same P_i = group_prefix_pages[i]
  * block ids (whole blocks: P_i*bs tokens).  First the queries of all members
  * attend to the P_i shared pages together, each page read once per group
- * (a dense [members*G x 16] x [16 x D] tensor-core product per page), giving
+ * (a dense [members*G x keys] x [keys x D] tcgen05 tensor-core tile), giving
  * split-KV partials; then the decode streams only each member's own pages
  * P_i .. ceil(L_b/bs)-1 and merges the prefix partials by log-sum-exp.
  *   - group_offsets [num_groups+1] and group_prefix_pages [num_groups] are
@@ -304,8 +304,12 @@ PA_API pa_status pa_decode_fp8(const void* q, const void* k_cache, const void* v
  *   - Shapes and alignment as for pa_decode (block_size 16, head_dim 64 or
  *     128, Hq/Hkv in {1, 2, 4, 8}); out [total][Hq][D].  No workspace.
  * One CTA per (sequence, 128-row tile, kv head) streams the sequence's
- * pages up to the tile's last position and computes the row tile against
- * each page on the tensor cores (mma.sync m16n8k16).
+ * pages up to the tile's last position in blocks of 64 keys and computes
+ * the tile on the tcgen05 tensor cores (S and O accumulated in tensor
+ * memory, P as bf16).  Environment, read at the first call:
+ * PA_PREFILL_BN=128 selects blocks of 128 keys (one CTA per SM);
+ * PA_PREFILL_MMA=sync selects the warp-level mma.sync kernels (this call
+ * and the prefix pass of pa_decode_shared_prefix).
  */
 PA_API pa_status pa_prefill(const void* q, const int32_t* cu_q_lens, int32_t max_q_len, const void* k_cache,
                             const void* v_cache, const int32_t* block_tables, const int32_t* context_lens,

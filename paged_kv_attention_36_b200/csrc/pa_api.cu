@@ -378,8 +378,14 @@ int prefix_tiles(const pa_dims& d, int max_group_size) {
     return int((rows + 16 * kPrefixNW - 1) / (16 * kPrefixNW));
 }
 
-// Key ranges per (group, row tile, kv head): enough CTAs for one wave.
+// Key ranges per (group, row tile, kv head): enough CTAs for one wave
+// (PA_PREFIX_SPLITS=n overrides, 1..16).
 int prefix_splits(const pa_dims& d, int num_groups, int max_group_size, int sms) {
+    static const int forced = [] {
+        const char* e = std::getenv("PA_PREFIX_SPLITS");
+        return e ? std::atoi(e) : 0;
+    }();
+    if (forced >= 1 && forced <= kMaxPrefixSplits) return forced;
     const int64_t base = int64_t(num_groups) * prefix_tiles(d, max_group_size) * d.num_kv_heads;
     int64_t s = base > 0 ? sms / base : 1;
     if (s < 1) s = 1;
