@@ -744,7 +744,8 @@ def run_prefill(args, ws, rank, local, reference: bool):
                      "kernel": ("pa::prefill_kernel (mma.sync m16n8k16; P.V as two bf16 products)"
                                 if os.environ.get("PA_PREFILL_MMA") == "sync" else
                                 "pa::prefill_tc_kernel (tcgen05.mma, S/P and O in TMEM, TMA-fed K/V)"),
-                     "traffic": None},
+                     "traffic": (None if os.environ.get("PA_PREFILL_MMA") or os.environ.get("PA_PREFILL_BN")
+                                 else _traffic(f"prefill-{wl}"))},
         "e2e": {"value": round(ws * flops / (e2e_ms / K * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / K, 5)},
         "gpu_launches": K,
