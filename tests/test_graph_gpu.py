@@ -7,10 +7,10 @@ so a whole step can be captured on a torch stream and replayed.  These
 tests capture (1) the fused append + decode (a cooperative launch with a
 grid barrier in the workspace), (2) the shared-prefix step (the prefix pass
 and the decode launched as its programmatic dependent) and (3) the two-call
-step (append, then decode), replay each several times with new inputs
-written into the captured buffers, and compare every replay with the fp64
-oracle.  Replays reuse the workspace, so they also prove that every call
-leaves its counters and barrier at zero.
+step (append, then decode), and (4) the multi-query prefill; they replay
+each several times with new inputs written into the captured buffers and
+compare every replay with the fp64 oracle.  Replays reuse the workspace,
+so they also prove that every call leaves its counters and barrier at zero.
 """
 import numpy as np
 import pytest
@@ -116,3 +116,42 @@ def test_graph_shared_prefix_step(pa, oracle_lib):
                                    k_new=t["k_new"], v_new=t["v_new"], slot_mapping=t["slot_mapping"],
                                    workspace=step.ws)
     _run(pa, oracle_lib, w, step)
+
+
+def test_graph_prefill(pa, oracle_lib):
+    """The multi-query prefill (tcgen05 kernel) captured once and replayed
+    with new query rows; each replay against the oracle's prefill."""
+    g0 = torch.Generator().manual_seed(88)
+    lens, q_lens, Hq, Hkv, D = [300, 47, 1000, 16], [64, 47, 200, 1], 16, 8, 128
+    ks = paging.random_seqs(g0, lens, Hkv, D)
+    vs = paging.random_seqs(g0, lens, Hkv, D)
+    nb = sum((L + 15) // 16 for L in lens) + 3
+    (kp, vp), bt = paging.page([ks, vs], lens, 16, nb, g0, poison=True)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(q_lens)]), dtype=torch.int32)
+    cl = torch.tensor(lens, dtype=torch.int32)
+    d = torch.device("cuda")
+    t = {"q": torch.zeros((sum(q_lens), Hq, D), dtype=torch.bfloat16, device=d), "cu": cu.to(d), "k": kp.to(d),
+         "v": vp.to(d), "bt": bt.to(d), "cl": cl.to(d)}
+    out = torch.empty_like(t["q"])
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+
+    def step():
+        pa.pa_prefill(t["q"], t["cu"], max(q_lens), t["k"], t["v"], t["bt"], t["cl"], D ** -0.5, out)
+    with torch.cuda.stream(stream):
+        step()  # warm-up outside capture
+    torch.cuda.current_stream().wait_stream(stream)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    for _ in range(3):
+        q = torch.randn(t["q"].shape, generator=g0).to(torch.bfloat16)
+        t["q"].copy_(q)
+        out.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        ref = oracle_lib.prefill(paging.bits(q), cu.numpy(), paging.bits(kp), paging.bits(vp), bt.numpy(),
+                                 cl.numpy(), D ** -0.5)
+        _close(out, ref)
+    assert pa.pa_device_errors(clear=True) == 0

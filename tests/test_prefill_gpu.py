@@ -82,3 +82,39 @@ def test_chunk_longer_than_context_is_reported(pa):
     out = torch.empty_like(q)
     pa.pa_prefill(q, cu, 12, kc, kc, bt, cl, 0.125, out)
     assert pa.pa_device_errors(clear=True) & pa.PA_DEVERR_CONTEXT
+
+
+@pytest.mark.parametrize("name", ["llama32", "qwen3"])
+def test_bench_batch_sampled_rows(pa, oracle_lib, name):
+    """The benchmark's own batch and launch (16 sequences, 512-token chunks
+    after prior contexts U[512,3584]) on the GPU; per sequence its first and
+    last query token and six seeded random ones are checked against the
+    oracle.  Query token i of sequence b is, by definition, the decode of
+    its q row over the first first_pos + i + 1 cached tokens (the oracle's
+    prefill equals its decode bit for bit there), so the pinned decode oracle
+    gives each sampled row without the whole O(chunk x context) reference."""
+    from paged_kv_attention_36_b200 import workloads
+    pb = workloads.make_prefill(name)
+    d = torch.device("cuda")
+    out = torch.full(pb.q.shape, float("nan"), dtype=torch.bfloat16, device=d)
+    pa.pa_prefill(pb.q.to(d), pb.cu_q_lens.to(d), pb.max_q_len, pb.k_cache.to(d), pb.v_cache.to(d),
+                  pb.block_tables.to(d), pb.context_lens.to(d), pb.scale, out)
+    torch.cuda.synchronize()
+    got = out.to(torch.float64).cpu().numpy()
+    assert not np.isnan(got).any(), "NaN in output"
+    rng = np.random.default_rng(36)
+    cu, cl = pb.cu_q_lens.numpy(), pb.context_lens.numpy()
+    rows, lens, seqs = [], [], []
+    for b in range(len(cl)):
+        ql = int(cu[b + 1] - cu[b])
+        first_pos = int(cl[b]) - ql
+        for i in sorted({0, ql - 1, *rng.integers(0, ql, 6).tolist()}):
+            rows.append(int(cu[b]) + i)
+            lens.append(first_pos + i + 1)
+            seqs.append(b)
+    ref = oracle_lib.decode(paging.bits(pb.q[rows]), paging.bits(pb.k_cache), paging.bits(pb.v_cache),
+                            pb.block_tables[seqs].numpy(), np.array(lens, dtype=np.int32), pb.scale)
+    err = np.abs(got[rows] - ref)
+    bad = err > ATOL + RTOL * np.abs(ref)
+    assert not bad.any(), f"{bad.sum()} of {bad.size} outside tolerance, max err {err.max():.3g}"
+    assert pa.pa_device_errors(clear=True) == 0
