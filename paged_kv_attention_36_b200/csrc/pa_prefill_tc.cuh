@@ -32,6 +32,12 @@
 // K and V halves of a ring stage are refilled separately (k_empty once Q K^T
 // has read it, v_empty once P V has), and K is loaded one block ahead of V,
 // so each has a full softmax step more of lead than a shared stage would give.
+// Parity waits are exact only if the barrier cannot complete again before
+// the wait: every wait here is on a phase whose next completion needs an
+// action the waiting thread takes later (a copy it has not issued, a P it
+// has not written, an MMA it has not issued).  Reusing s_full to release the
+// K ring breaks this when NS < KS (S_{j-KS+NS} can finish before K_j is
+// loaded) and deadlocks until the bounded wait gives up.
 //
 // The staged layout of a block is [D/64 panels][BN tokens][128 bytes] with the
 // 128-byte swizzle, for K and V alike: K is then the K-major B operand of
