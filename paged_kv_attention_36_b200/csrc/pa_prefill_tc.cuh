@@ -87,6 +87,7 @@ template <bool PREFIX, int D, int G, int BN, int KS, int NS, class Params>
 __device__ __forceinline__ void tc_attention_tile(const Params& p) {
     using Cfg = TcPrefillCfg<D, BN, KS, NS>;
     static_assert(Cfg::kBM % G == 0, "a tile holds whole tokens (members)");
+    constexpr bool kKOnV = KS >= 4;  // release K ring slots with the V ones (deep rings)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* qs = smem;
@@ -199,8 +200,11 @@ __device__ __forceinline__ void tc_attention_tile(const Params& p) {
         auto load = [&](int j, bool v, int32_t blk) -> bool {
             const int s = j % KS;
             uint64_t* full = v ? &v_full[s] : &k_full[s];
-            if (j >= KS &&
-                !__all_sync(0xffffffffu, mbar_wait_sleep(v ? &v_empty[s] : &k_empty[s], uint32_t(j / KS - 1) & 1, abort)))
+            // with a deep ring the K half is released with the V half (on
+            // v_empty: its next completion needs V_j, loaded after K_j), which
+            // saves the MMA thread a commit per block
+            if (j >= KS && !__all_sync(0xffffffffu, mbar_wait_sleep((v || kKOnV) ? &v_empty[s] : &k_empty[s],
+                                                                    uint32_t(j / KS - 1) & 1, abort)))
                 return false;
             const int npg = pages - j * Cfg::kPages < Cfg::kPages ? pages - j * Cfg::kPages : Cfg::kPages;
             if (lane == 0) mbar_arrive_expect_tx(full, uint32_t(npg * Cfg::kPageBytes));
@@ -272,7 +276,7 @@ __device__ __forceinline__ void tc_attention_tile(const Params& p) {
                         umma_ss(tmem + bb * BN, qd + uint64_t((c * Cfg::kPanelQ + kk * 32) >> 4),
                                 kd + uint64_t((c * Cfg::kPanelKV + kk * 32) >> 4), id_qk, uint32_t(c | kk));
                 umma_commit(&s_full[bb]);
-                umma_commit(&k_empty[s]);
+                if (!kKOnV) umma_commit(&k_empty[s]);
                 return true;
             };
             // S runs NS - 1 blocks ahead of P V.  With three or more buffers,
