@@ -348,24 +348,30 @@ __device__ __forceinline__ void tc_attention_tile(const Params& p) {
             float s[BN];
 #pragma unroll
             for (int k = 0; k < BN / 64; ++k) tmem_ld64(tmem + lanes + bb * BN + 64 * k, &s[64 * k]);
-            // scaled logits (log2 units); keys past the row's position -> -inf
+            // logits in log2 units are s * ce: with a positive scale the scale
+            // is applied inside the exponent's fma (the max commutes with it);
+            // otherwise s is scaled first and ce = 1.  Keys past the row's
+            // position -> -inf.
             const int n0 = j * BN;
+            float ce = c;
+            if (!(c > 0.f)) {
 #pragma unroll
-            for (int i = 0; i < BN; ++i) s[i] *= c;
+                for (int i = 0; i < BN; ++i) s[i] *= c;
+                ce = 1.f;
+            }
             if (n0 + BN > lim) {
 #pragma unroll
                 for (int i = 0; i < BN; ++i)
                     if (n0 + i >= lim) s[i] = -INFINITY;
             }
-            // row max and, below, row sum over 8 independent partials (no
-            // BN-long dependency chain)
+            // row max over 8 independent partials (no BN-long dependency chain)
             float mp[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) mp[u] = s[u];
 #pragma unroll
             for (int i = 8; i < BN; ++i) mp[i & 7] = fmaxf(mp[i & 7], s[i]);
             const float m_blk = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                                      fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+                                      fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * ce;
             const float m_new = fmaxf(m, m_blk);
             if (__any_sync(0xffffffffu, m_new > m + 8.f)) {
                 const float alpha = ex2_approx(m - m_new);  // 0 while m = -inf
@@ -387,22 +393,29 @@ __device__ __forceinline__ void tc_attention_tile(const Params& p) {
                 l *= alpha;
                 m = m_new;
             }
-            // P = 2^(s*c - m) as bf16 pairs over the first BN/2 columns of the buffer
-            float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            // P = 2^(s*ce - m) as bf16 pairs over the first BN/2 columns of the
+            // buffer; the exponent and the row sum in packed f32x2 arithmetic
+            const uint64_t ce2 = f2_pack(ce, ce), nm2 = f2_pack(-m, -m);
+            uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
             for (int k = 0; k < BN / 64; ++k) {
                 uint32_t w[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const float p0 = ex2_approx(s[64 * k + 2 * i] - m);
-                    const float p1 = ex2_approx(s[64 * k + 2 * i + 1] - m);
-                    sp[(2 * i) & 7] += p0;
-                    sp[(2 * i + 1) & 7] += p1;
+                    float t0, t1;
+                    f2_unpack(f2_fma(f2_pack(s[64 * k + 2 * i], s[64 * k + 2 * i + 1]), ce2, nm2), t0, t1);
+                    const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+                    acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
                     w[i] = float2_to_bf16x2(p0, p1);
                 }
                 tmem_st32(tmem + lanes + bb * BN + 32 * k, w);
             }
-            l += ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+            {
+                float a0, a1, b0, b1;
+                f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
+                f2_unpack(f2_add(acc[2], acc[3]), b0, b1);
+                l += (a0 + a1) + (b0 + b1);
+            }
             tmem_st_wait();
             if (j == zero_blk) {
                 // V rows rem .. 15 of the last page hold no token of the context
