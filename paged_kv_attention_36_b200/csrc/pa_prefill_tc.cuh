@@ -364,14 +364,15 @@ __device__ __forceinline__ void tc_attention_tile(const Params& p) {
                 for (int i = 0; i < BN; ++i)
                     if (n0 + i >= lim) s[i] = -INFINITY;
             }
-            // row max over 8 independent partials (no BN-long dependency chain)
+            // row max over 8 independent partials (no BN-long dependency
+            // chain), two logits per three-input max
             float mp[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) mp[u] = s[u];
 #pragma unroll
-            for (int i = 8; i < BN; ++i) mp[i & 7] = fmaxf(mp[i & 7], s[i]);
-            const float m_blk = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                                      fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * ce;
+            for (int i = 8; i < BN; i += 2) mp[(i >> 1) & 7] = fmax3(mp[(i >> 1) & 7], s[i], s[i + 1]);
+            const float m_blk =
+                fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7])) * ce;
             const float m_new = fmaxf(m, m_blk);
             if (__any_sync(0xffffffffu, m_new > m + 8.f)) {
                 const float alpha = ex2_approx(m - m_new);  // 0 while m = -inf
