@@ -435,45 +435,62 @@ __device__ __forceinline__ void tc_attention_tile(const Params& p) {
             mbar_arrive(&p_full[bb]);
         }
 
-        // ---- output: O / l as bf16 ----
+        // ---- output: O / l (bf16 rows, or the split's fp32 partial rows).
+        // Each thread writes its row into the Q and ring space, idle once the
+        // last P V has completed (rows padded by 16 bytes, so a warp's 16-byte
+        // writes fall in distinct banks); then every warp copies whole rows
+        // out with consecutive lanes on consecutive 16 bytes.
         if (ok)
             ok = __all_sync(0xffffffffu,
                             mbar_wait_sleep(&v_empty[(nblk - 1) % KS], uint32_t((nblk - 1) / KS) & 1, abort));
+        constexpr int kRowBytes = D * (PREFIX ? 4 : 2);
+        constexpr int kRowStride = kRowBytes + 16;
+        static_assert(Cfg::kBM * kRowStride <= Cfg::kBarOff, "output staging fits in the Q and ring space");
         if (ok) {
             tc_fence_after();
             const float inv = 1.f / l;
-            if constexpr (!PREFIX) {
-                // bf16 output row
-                uint4* dst = reinterpret_cast<uint4*>(p.out + orow);
+            uint8_t* mine = smem + row * kRowStride;
 #pragma unroll
-                for (int k = 0; k < D / 64; ++k) {
-                    float o[64];
-                    tmem_ld64(t_o + lanes + 64 * k, o);
-                    if (valid) {
+            for (int k = 0; k < D / 64; ++k) {
+                float o[64];
+                tmem_ld64(t_o + lanes + 64 * k, o);
+                if constexpr (!PREFIX) {
 #pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            dst[8 * k + q] = make_uint4(float2_to_bf16x2(o[8 * q] * inv, o[8 * q + 1] * inv),
-                                                        float2_to_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
-                                                        float2_to_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
-                                                        float2_to_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
-                    }
+                    for (int q = 0; q < 8; ++q)
+                        *reinterpret_cast<uint4*>(mine + (64 * k + 8 * q) * 2) =
+                            make_uint4(float2_to_bf16x2(o[8 * q] * inv, o[8 * q + 1] * inv),
+                                       float2_to_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
+                                       float2_to_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
+                                       float2_to_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q)
+                        *reinterpret_cast<float4*>(mine + (64 * k + 4 * q) * 4) =
+                            make_float4(o[4 * q] * inv, o[4 * q + 1] * inv, o[4 * q + 2] * inv, o[4 * q + 3] * inv);
                 }
-            } else {
-                // this split's partial: normalised output, (max logit in base 2, exp-sum)
-                const int64_t idx = (int64_t(blockIdx.z) * p.B + qrow) * p.Hq + g * G + r % G;
-                float4* dst = reinterpret_cast<float4*>(p.prefix_o + idx * D);
-#pragma unroll
-                for (int k = 0; k < D / 64; ++k) {
-                    float o[64];
-                    tmem_ld64(t_o + lanes + 64 * k, o);
-                    if (valid) {
-#pragma unroll
-                        for (int q = 0; q < 16; ++q)
-                            dst[16 * k + q] = make_float4(o[4 * q] * inv, o[4 * q + 1] * inv, o[4 * q + 2] * inv,
-                                                          o[4 * q + 3] * inv);
-                    }
-                }
-                if (valid) p.prefix_ml[idx] = make_float2(m, l);
+            }
+            if constexpr (PREFIX) {
+                // (max logit in base 2, exp-sum) of the row's partial
+                if (valid) p.prefix_ml[(int64_t(blockIdx.z) * p.B + qrow) * p.Hq + g * G + r % G] = make_float2(m, l);
+            }
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");  // the 4 softmax warps: rows staged
+        if (!*abort) {
+            constexpr int kChunks = kRowBytes / 16;       // 16-byte chunks per row
+            constexpr int kRowsPerPass = 32 / kChunks;    // rows per warp instruction
+            const int wq = warp - 2;
+            for (int rr = wq * kRowsPerPass + lane / kChunks; rr < Cfg::kBM; rr += 4 * kRowsPerPass) {
+                const int rg = row0 + rr;
+                if (rg >= nrows) break;  // rows only grow along the loop
+                const int ch = lane % kChunks;
+                const uint4 v = *reinterpret_cast<const uint4*>(smem + rr * kRowStride + ch * 16);
+                const int64_t qr = int64_t(PREFIX ? first : q0) + rg / G;
+                const int64_t grow = (PREFIX ? int64_t(blockIdx.z) * p.B * p.Hq : int64_t(0)) + qr * p.Hq +
+                                     g * G + rg % G;
+                if constexpr (PREFIX)
+                    reinterpret_cast<uint4*>(p.prefix_o + grow * D)[ch] = v;
+                else
+                    reinterpret_cast<uint4*>(p.out + grow * D)[ch] = v;
             }
         }
         if constexpr (PREFIX) {
