@@ -180,7 +180,7 @@ def _step_bytes(w):
 
 
 def cpu_baseline(w, dec_bytes: int, app_bytes: int, budget_s: float = 12.0):
-    """The oracle, as it stands, on the GPU machine's host cores: full append +
+    """The oracle, as it stands, on the host's cores: full append +
     decode steps of the same batch, repeated until about budget_s seconds."""
     import oracle
     from tests import paging  # bit-pattern views only
