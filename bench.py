@@ -475,7 +475,9 @@ def run_pa(args, ws, rank, local):
         "step_pct_of_8tbs_nominal": round(100 * achieved / 8000.0, 1),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                     "kernel": ("pa::prefix_kernel + pa::decode_kernel<..., APPEND> (pa_decode_shared_prefix)"
+                     "kernel": (("pa::prefix_kernel" if os.environ.get("PA_PREFILL_MMA") == "sync"
+                                 else "pa::prefix_tc_kernel (tcgen05; carries the append)")
+                                + " + pa::decode_kernel<...> (pa_decode_shared_prefix)"
                                 if grouped else "pa::decode_kernel<..., APPEND> (pa_append_decode)"),
                      "traffic": _traffic(args.workload),
                      "algorithmic_bytes_per_launch": step_bytes},
