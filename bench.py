@@ -294,6 +294,31 @@ def run_reference(args, ws, rank):
     print(json.dumps(line), flush=True)
 
 
+class Packed:
+    """A step's inputs as views into one device buffer (each at a 256-byte
+    aligned offset) with a pinned host twin, so that a caller refreshes all of
+    them with a single host-to-device copy."""
+
+    def __init__(self, tensors, dev):
+        offs, off = {}, 0
+        for n, t in tensors.items():
+            off = -(-off // 256) * 256
+            offs[n] = (off, t.numel() * t.element_size())
+            off += t.numel() * t.element_size()
+        self.nbytes = off
+        self.host = torch.empty(off, dtype=torch.uint8).pin_memory()
+        self.dev = torch.empty(off, dtype=torch.uint8, device=dev)
+        self.views = {}
+        for n, t in tensors.items():
+            o, nb = offs[n]
+            self.host[o:o + nb].view(t.dtype).view(t.shape).copy_(t)
+            self.views[n] = self.dev[o:o + nb].view(t.dtype).view(t.shape)
+        self.dev.copy_(self.host)
+
+    def h2d(self):
+        self.dev.copy_(self.host, non_blocking=True)
+
+
 def run_pa(args, ws, rank, local):
     from paged_kv_attention_36_b200 import binding as pa
     from paged_kv_attention_36_b200 import workloads
@@ -310,14 +335,18 @@ def run_pa(args, ws, rank, local):
     pool_bytes = 2 * w.k_cache.numel() * 2
     rotate = pool_bytes >= ROTATE_MIN_POOL
     ncopies = max(2, -(-ROTATE_BYTES // pool_bytes)) if rotate else 1
-    q, bt, cl = w.q.to(dev), w.block_tables.to(dev), w.context_lens.to(dev)
-    kn, vn, sm = w.k_new.to(dev), w.v_new.to(dev), w.slot_mapping.to(dev)
+    grouped = w.num_groups > 0
+    step_in = {"q": w.q, "bt": w.block_tables, "cl": w.context_lens, "kn": w.k_new, "vn": w.v_new,
+               "sm": w.slot_mapping}
+    if grouped:
+        step_in.update(go=w.group_offsets, gp=w.group_prefix_pages)
+    packed = Packed(step_in, dev)  # the per-step inputs, one host-to-device copy in the e2e step
+    q, bt, cl, kn, vn, sm = (packed.views[n] for n in ("q", "bt", "cl", "kn", "vn", "sm"))
     caches = [(w.k_cache.to(dev), w.v_cache.to(dev)) for _ in range(ncopies)]
     out = torch.empty_like(q)
     dims = pa.make_dims(q, caches[0][0], bt)
-    grouped = w.num_groups > 0
     if grouped:
-        go, gp, mgs = w.group_offsets.to(dev), w.group_prefix_pages.to(dev), w.max_group_size
+        go, gp, mgs = packed.views["go"], packed.views["gp"], w.max_group_size
         wsp = torch.zeros(pa.pa_decode_shared_prefix_workspace_bytes(dims, w.num_groups, mgs),
                           dtype=torch.uint8, device=dev)
     else:
@@ -403,22 +432,14 @@ def run_pa(args, ws, rank, local):
         torch.cuda.synchronize(dev)
         plain_avg = _max_over_ranks(sum(ev3[k][0].elapsed_time(ev3[k][1]) for k in range(K)) / K, ws)
 
-    # ---- end to end through the public API from pinned host buffers ----
-    host_src = [("q", w.q), ("bt", w.block_tables), ("cl", w.context_lens), ("kn", w.k_new), ("vn", w.v_new),
-                ("sm", w.slot_mapping)]
-    if grouped:
-        host_src += [("go", w.group_offsets), ("gp", w.group_prefix_pages)]
-    host = {n: t.pin_memory() for n, t in host_src}
+    # ---- end to end through the public API from pinned host memory: the
+    # step's inputs in one pinned buffer (one copy), the output read back ----
     out_h = torch.empty(w.q.shape, dtype=torch.bfloat16).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    h2d = packed.nbytes
     d2h = out_h.numel() * out_h.element_size()
-    dev_in = {"q": q, "bt": bt, "cl": cl, "kn": kn, "vn": vn, "sm": sm}
-    if grouped:
-        dev_in.update(go=go, gp=gp)
 
     def e2e_step(c):
-        for n, t in host.items():
-            dev_in[n].copy_(t, non_blocking=True)
+        packed.h2d()
         fused[c]()
         out_h.copy_(out, non_blocking=True)
 
@@ -518,8 +539,9 @@ def run_pa_fp8(args, ws, rank, local):
     ncopies = max(2, -(-ROTATE_BYTES // pool_bytes)) if rotate else 1
     caches = [(k8.clone(), v8.clone()) for _ in range(ncopies)]
     del k8, v8
-    q, bt, cl = w.q.to(dev), w.block_tables.to(dev), w.context_lens.to(dev)
-    kn, vn, sm = w.k_new.to(dev), w.v_new.to(dev), w.slot_mapping.to(dev)
+    packed = Packed({"q": w.q, "bt": w.block_tables, "cl": w.context_lens, "kn": w.k_new, "vn": w.v_new,
+                     "sm": w.slot_mapping}, dev)  # one host-to-device copy in the e2e step
+    q, bt, cl, kn, vn, sm = (packed.views[n] for n in ("q", "bt", "cl", "kn", "vn", "sm"))
     out = torch.empty_like(q)
     dims = pa.pa_dims(q.shape[0], q.shape[1], Hkv, D, 16, NB, bt.shape[1])
     wsp = pa.alloc_workspace(dims, device=dev)
@@ -560,16 +582,12 @@ def run_pa_fp8(args, ws, rank, local):
     app_avg = _max_over_ranks(sum(ev[k][0].elapsed_time(ev[k][1]) for k in range(K)) / K, ws)
     dec_avg = _max_over_ranks(sum(ev[k][1].elapsed_time(ev[k][2]) for k in range(K)) / K, ws)
 
-    host = {n: t.pin_memory() for n, t in (("q", w.q), ("bt", w.block_tables), ("cl", w.context_lens),
-                                            ("kn", w.k_new), ("vn", w.v_new), ("sm", w.slot_mapping))}
     out_h = torch.empty(w.q.shape, dtype=torch.bfloat16).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    h2d = packed.nbytes
     d2h = out_h.numel() * out_h.element_size()
-    dev_in = {"q": q, "bt": bt, "cl": cl, "kn": kn, "vn": vn, "sm": sm}
 
     def e2e_step(c):
-        for n, t in host.items():
-            dev_in[n].copy_(t, non_blocking=True)
+        packed.h2d()
         app[c]()
         dec[c]()
         out_h.copy_(out, non_blocking=True)
@@ -682,7 +700,8 @@ def run_prefill(args, ws, rank, local, reference: bool):
     from paged_kv_attention_36_b200 import binding as pa
     dev = torch.device("cuda", local if ws > 1 else torch.cuda.current_device())
     torch.cuda.set_device(dev)
-    t = {k: getattr(pb, k).to(dev) for k in ("q", "cu_q_lens", "k_cache", "v_cache", "block_tables", "context_lens")}
+    packed = Packed({k: getattr(pb, k) for k in ("q", "cu_q_lens", "block_tables", "context_lens")}, dev)
+    t = dict(packed.views, k_cache=pb.k_cache.to(dev), v_cache=pb.v_cache.to(dev))
     out = torch.empty_like(t["q"])
     stream = torch.cuda.current_stream(dev)
     call = pa.prepare_prefill(t["q"], t["cu_q_lens"], pb.max_q_len, t["k_cache"], t["v_cache"], t["block_tables"],
@@ -707,17 +726,16 @@ def run_prefill(args, ws, rank, local, reference: bool):
     if errs:
         raise RuntimeError(f"device error bits {errs:#x} during the benchmark")
     total_ms = _max_over_ranks(sum(ev[k][0].elapsed_time(ev[k][1]) for k in range(K)), ws)
-    # end to end: q and the batch metadata from pinned host memory, out back
-    host = {n: getattr(pb, n).pin_memory() for n in ("q", "cu_q_lens", "block_tables", "context_lens")}
+    # end to end: q and the batch metadata from pinned host memory (one
+    # packed copy), out back
     out_h = torch.empty(pb.q.shape, dtype=torch.bfloat16).pin_memory()
-    h2d = sum(x.numel() * x.element_size() for x in host.values())
+    h2d = packed.nbytes
     d2h = out_h.numel() * out_h.element_size()
     ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     torch.cuda.synchronize(dev)
     for k in range(K):
         ee[k][0].record(stream)
-        for n, x in host.items():
-            t[n].copy_(x, non_blocking=True)
+        packed.h2d()
         call()
         out_h.copy_(out, non_blocking=True)
         ee[k][1].record(stream)
