@@ -130,7 +130,10 @@ PA_API int32_t pa_decode_default_ctas(void);
  * aligned.  The per-page math runs on the tensor cores (mma.sync, fp32
  * accumulation); setting the environment variable PA_DECODE_MATH=simt
  * before the first call selects the fp32 CUDA core variant instead
- * (head_dim*Hq/Hkv <= 256 only).
+ * (head_dim*Hq/Hkv <= 256 only).  PA_SEG_WEIGHT_BYTES (read at the first
+ * call; default 65536) is the fixed cost of finishing a (sequence, head
+ * group) segment, in K+V bytes, that the equal-share split charges: larger
+ * values cut short contexts into fewer split pieces.
  */
 PA_API pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
                     const int32_t* block_tables, const int32_t* context_lens, float scale,
@@ -243,6 +246,9 @@ PA_API pa_status pa_decode_static_ws(const void* q, const void* k_cache, const v
  *     be at least pa_decode_shared_prefix_workspace_bytes(dims, num_groups,
  *     max_group_size) bytes, zero-filled before its first use, and is left
  *     ready for the next call; calls that share it must not overlap.
+ *   - The prefix pass splits each group's shared pages into key ranges
+ *     (enough CTAs for one wave; PA_PREFIX_SPLITS=n, 1..16, read at the
+ *     first call, overrides); the decode folds one partial per range.
  *   - num_groups = 0 is pa_decode / pa_append_decode with this workspace.
  */
 PA_API size_t pa_decode_shared_prefix_workspace_bytes(const pa_dims* dims, int32_t num_groups,
