@@ -106,3 +106,26 @@ def test_binding_rejects_host_tensors(binding):
         binding.pa_decode(q, kc, kc, bt, cl, 0.125, q.clone(), workspace=torch.zeros(8, dtype=torch.uint8))
     with pytest.raises(TypeError):
         binding.pa_decode(q.float(), kc, kc, bt, cl, 0.125, q.clone())
+
+
+def test_prefill_host_validation(binding):
+    # fake, never-dereferenced addresses: every case is decided before any CUDA call
+    vp = ctypes.c_void_p
+
+    def call(dims, q=16, cu=16, mq=8, k=16, v=16, bt=16, cl=16, out=16):
+        return binding.lib.pa_prefill(vp(q), vp(cu), mq, vp(k), vp(v), vp(bt), vp(cl), 0.125, vp(out),
+                                      ctypes.byref(dims) if dims is not None else None, vp(0))
+    assert call(None) == -1                                                   # NULL dims
+    assert call(_dims(binding), mq=-1) == -2                                  # negative max_q_len
+    assert call(_dims(binding, num_q_heads=6, num_kv_heads=4)) == -2
+    assert call(_dims(binding, head_dim=96)) == -3
+    assert call(_dims(binding, block_size=32)) == -3
+    assert call(_dims(binding, num_q_heads=16, num_kv_heads=1)) == -3         # G = 16
+    assert call(_dims(binding), mq=0) == 0                                    # nothing to do
+    assert call(_dims(binding, num_seqs=0)) == 0
+    assert call(_dims(binding, num_blocks=0)) == -2
+    assert call(_dims(binding), cu=0) == -1
+    assert call(_dims(binding), out=0) == -1
+    assert call(_dims(binding), q=8) == -4                                    # misaligned
+    assert call(_dims(binding), cu=2) == -4
+    assert call(_dims(binding, num_blocks=1 << 27)) == -2                     # 2^32 cache rows
