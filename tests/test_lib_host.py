@@ -129,3 +129,52 @@ def test_prefill_host_validation(binding):
     assert call(_dims(binding), q=8) == -4                                    # misaligned
     assert call(_dims(binding), cu=2) == -4
     assert call(_dims(binding, num_blocks=1 << 27)) == -2                     # 2^32 cache rows
+
+
+def test_fp8_host_validation(binding):
+    vp = ctypes.c_void_p
+    d = _dims(binding)
+    app = binding.lib.pa_cache_append_fp8
+
+    def a(dims, n=3, kn=16, vn=16, sm=16, kc=16, vc=16, ks=16, vs=16):
+        return app(vp(kn), vp(vn), vp(sm), n, vp(kc), vp(vc), vp(ks), vp(vs),
+                   ctypes.byref(dims) if dims is not None else None, vp(0))
+    assert a(None) == -1
+    assert a(d, n=-1) == -2
+    assert a(_dims(binding, head_dim=12)) == -3
+    assert a(_dims(binding, block_size=32)) == -3
+    assert a(d, n=0) == 0
+    assert a(d, ks=0) == -1
+    assert a(d, kn=24) == -4
+    assert a(d, vs=2) == -4
+
+    dec = binding.lib.pa_decode_fp8
+
+    def dd(dims, q=16, out=16):
+        return dec(vp(q), vp(16), vp(16), vp(16), vp(16), vp(16), vp(16), 0.125, vp(out),
+                   ctypes.byref(dims) if dims is not None else None, vp(16), 1 << 30, vp(0))
+    assert dd(None) == -1
+    assert dd(_dims(binding, num_q_heads=6, num_kv_heads=4)) == -2
+    assert dd(_dims(binding, head_dim=96)) == -3
+    assert dd(_dims(binding, num_seqs=0)) == 0
+    assert dd(d, q=0) == -1
+    assert dd(d, out=8) == -4
+
+
+def test_shared_prefix_host_validation(binding):
+    vp = ctypes.c_void_p
+    f = binding.lib.pa_decode_shared_prefix
+
+    def call(dims, n=0, groups=1, mgs=4, kn=16, q=16, out=16, go=16, gp=16):
+        return f(vp(kn), vp(16), vp(16), n, vp(q), vp(16), vp(16), vp(16), vp(16), 0.125, vp(go), vp(gp), groups,
+                 mgs, vp(out), ctypes.byref(dims) if dims is not None else None, vp(16), 1 << 30, vp(0))
+    d = _dims(binding)
+    assert call(None) == -1
+    assert call(d, n=-1) == -2
+    assert call(d, groups=-1) == -2
+    assert call(d, mgs=0) == -2                                   # groups need a group size
+    assert call(_dims(binding, num_q_heads=6, num_kv_heads=4)) == -2
+    assert call(_dims(binding, head_dim=96)) == -3
+    assert call(d, q=0) == -1
+    assert call(d, out=8) == -4
+    assert call(_dims(binding, num_seqs=0)) == 0                  # nothing to attend over, nothing to append
