@@ -6,7 +6,7 @@ merge included).  Prints ONE JSON line on rank 0.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama32]
     python bench.py --impl reference ...   # the fp64 CPU oracle, timed on host cores
-    python bench.py --kv fp8 ...           # fp8 (E4M3) caches: append_fp8 + decode_fp8
+    python bench.py --kv fp8 ...           # fp8 (E4M3) caches: the fused append_fp8 + decode_fp8
 
 Metric: effective GB/s = algorithmic bytes / device time, where the
 algorithmic bytes of a step are the distinct K/V rows the decode must read
@@ -60,6 +60,8 @@ def _args():
                     help="cache format: bf16, or fp8 E4M3 codes with per-kv-head scales")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="with the default llama32 batch, skip timing the long/skewed batch beside it")
     return ap.parse_args()
 
 
@@ -125,15 +127,25 @@ def _traffic(workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle samples every 100 ms during the timed regions."""
+    """nvidia-smi clock / throttle samples every 100 ms, kept only inside the
+    windows opened with begin() and closed with end() (end() also takes one
+    synchronous sample, so every window has at least one).  The sampler is
+    started before the warm-up; each window brackets a timed region and the
+    untimed runs of the same step around it, so the samples see the step's
+    load even when the timed region itself lasts a few milliseconds."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int, enabled: bool):
+        import threading
         self.proc = None
         self.idx = device_index
+        self.samples = []      # (time, line)
+        self.windows = []
+        self.t_open = None
+        self.enabled = enabled
         if enabled:
             try:
                 self.proc = subprocess.Popen(
@@ -142,19 +154,44 @@ class ClockSampler:
                     stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             except (OSError, FileNotFoundError):
                 self.proc = None
+        if self.proc is not None:
+            threading.Thread(target=self._read, daemon=True).start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line))
+
+    def begin(self):
+        self.t_open = time.time()
+
+    def end(self):
+        if not self.enabled or self.t_open is None:
+            return
+        try:
+            r = subprocess.run(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                                "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=10)
+            now = time.time()
+            self.samples += [(now, ln) for ln in r.stdout.splitlines()]
+        except (OSError, subprocess.TimeoutExpired):
+            now = time.time()
+        self.windows.append((self.t_open, now + 0.01))
+        self.t_open = None
 
     def stop(self):
-        if self.proc is None:
+        if not self.enabled:
             return None
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.proc.wait()
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
+        for t, line in list(self.samples):
+            if not any(a <= t <= b for a, b in self.windows):
+                continue
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -170,6 +207,19 @@ class ClockSampler:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def hold_load(call, seconds: float, dev, between=None):
+    """Runs `call` back to back, untimed, for about `seconds` of wall time
+    (in bursts of 50, synchronised), so that the clock samples taken around
+    a short timed region see the same load."""
+    t0 = time.time()
+    while time.time() - t0 < seconds:
+        for _ in range(50):
+            call()
+            if between is not None:
+                between()
+        torch.cuda.synchronize(dev)
 
 
 def _step_bytes(w):
@@ -319,6 +369,65 @@ class Packed:
         self.dev.copy_(self.host, non_blocking=True)
 
 
+def time_fused_step(pa, name, args, dev, ws, clocks):
+    """The fused append + decode step of batch `name` (larger than L2),
+    timed like the headline step: the same --steps / --warmup, cache copies
+    rotated, CUDA events on the launching stream, max over ranks.  Returns
+    its own record (value, step time and roofline)."""
+    from paged_kv_attention_36_b200 import workloads
+    w = workloads.make(name)
+    dec_bytes, app_bytes = _step_bytes(w)
+    step_bytes = dec_bytes + app_bytes
+    pool_bytes = 2 * w.k_cache.numel() * 2
+    assert pool_bytes >= ROTATE_MIN_POOL
+    ncopies = max(2, -(-ROTATE_BYTES // pool_bytes))
+    q, bt, cl, kn, vn, sm = (t.to(dev) for t in (w.q, w.block_tables, w.context_lens, w.k_new, w.v_new,
+                                                 w.slot_mapping))
+    caches = [(w.k_cache.to(dev), w.v_cache.to(dev)) for _ in range(ncopies)]
+    out = torch.empty_like(q)
+    wsp = pa.alloc_workspace(pa.make_dims(q, caches[0][0], bt), device=dev)
+    stream = torch.cuda.current_stream(dev)
+    fused = [pa.prepare_append_decode(kn, vn, sm, q, kc, vc, bt, cl, w.scale, out, wsp, stream=stream)
+             for kc, vc in caches]
+    W_ = max(3, args.warmup)
+    for k in range(W_):
+        fused[k % ncopies]()
+    torch.cuda.synchronize(dev)
+    rot = iter(range(W_, 1 << 62))
+    clocks.begin()
+    hold_load(lambda: fused[next(rot) % ncopies](), 0.3, dev)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    _barrier(ws)
+    torch.cuda.synchronize(dev)
+    for k in range(K):
+        ev[k][0].record(stream)
+        fused[k % ncopies]()
+        ev[k][1].record(stream)
+    torch.cuda.synchronize(dev)
+    _barrier(ws)
+    hold_load(lambda: fused[next(rot) % ncopies](), 0.2, dev)
+    clocks.end()
+    errs = pa.pa_device_errors(clear=True)
+    if errs:
+        raise RuntimeError(f"device error bits {errs:#x} during the {name} benchmark")
+    total_ms = _max_over_ranks(sum(ev[k][0].elapsed_time(ev[k][1]) for k in range(K)), ws)
+    peak, peak_kind = _peaks()
+    step_avg = total_ms / K
+    achieved = step_bytes / (step_avg * 1e-3) / 1e9
+    return {
+        "workload": name, "description": w.spec.description,
+        "value": round(ws * K * step_bytes / (total_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+        "steps": K, "warmup": W_, "step_us": round(step_avg * 1e3, 2),
+        "l2": f"inputs larger than L2: {ncopies} copies of the {pool_bytes / 1e6:.0f} MB paged cache rotated, no flush",
+        "step_pct_of_8tbs_nominal": round(100 * achieved / 8000.0, 1),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                     "kernel": "pa::decode_kernel<..., APPEND> (pa_append_decode)",
+                     "traffic": _traffic(name), "algorithmic_bytes_per_launch": step_bytes},
+    }
+
+
 def run_pa(args, ws, rank, local):
     from paged_kv_attention_36_b200 import binding as pa
     from paged_kv_attention_36_b200 import workloads
@@ -372,16 +481,19 @@ def run_pa(args, ws, rank, local):
         if flush is not None:
             flush.zero_()
 
+    clocks = ClockSampler(dev.index, enabled=not args.no_clocks)
     W_ = max(3, args.warmup)
     for k in range(W_):
         fused[k % ncopies]()
         between()
     torch.cuda.synchronize(dev)
+    rot = iter(range(1 << 62))
+    clocks.begin()
+    hold_load(lambda: fused[next(rot) % ncopies](), 0.3, dev, between)  # untimed: the clock samples see the load
 
     # ---- timed region: K steps, each one launch of the fused append + decode ----
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
-    clocks = ClockSampler(dev.index, enabled=not args.no_clocks)
     _barrier(ws)
     torch.cuda.synchronize(dev)
     for k in range(K):
@@ -391,6 +503,8 @@ def run_pa(args, ws, rank, local):
         between()
     torch.cuda.synchronize(dev)
     _barrier(ws)
+    hold_load(lambda: fused[next(rot) % ncopies](), 0.2, dev, between)
+    clocks.end()
     errs = pa.pa_device_errors(clear=True)
     if errs:
         raise RuntimeError(f"device error bits {errs:#x} during the benchmark")
@@ -457,8 +571,13 @@ def run_pa(args, ws, rank, local):
         between()
     torch.cuda.synchronize(dev)
     _barrier(ws)
-    clk = clocks.stop()
     e2e_total = _max_over_ranks(sum(ee[k][0].elapsed_time(ee[k][1]) for k in range(K)), ws)
+
+    # the other batch the 70 %-of-HBM target names, timed the same way
+    extra = None
+    if args.workload == "llama32" and not args.no_extra:
+        extra = time_fused_step(pa, "longskew", args, dev, ws, clocks)
+    clk = clocks.stop()
 
     if rank != 0:
         return
@@ -511,13 +630,17 @@ def run_pa(args, ws, rank, local):
     if grouped:
         line["config"]["shared_prefix_groups"] = w.num_groups
         line["plain_path_step_us"] = round(plain_avg * 1e3, 2)
+    if extra is not None:
+        line["longskew_step"] = extra
     if ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, dec_bytes, app_bytes)
     print(json.dumps(line), flush=True)
 
 
 def run_pa_fp8(args, ws, rank, local):
-    """The fp8 step: pa_cache_append_fp8 then pa_decode_fp8 (two launches)."""
+    """The fp8 step: pa_append_decode_fp8 (the E4M3 append and the decode in
+    one launch); the same steps as two launches (pa_cache_append_fp8, then
+    pa_decode_fp8) are timed beside it for the split."""
     from paged_kv_attention_36_b200 import binding as pa
     from paged_kv_attention_36_b200 import workloads
 
@@ -547,6 +670,8 @@ def run_pa_fp8(args, ws, rank, local):
     wsp = pa.alloc_workspace(dims, device=dev)
     flush = None if rotate else torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    fused = [pa.prepare_append_decode_fp8(kn, vn, sm, q, kc, vc, ks, vs, bt, cl, w.scale, out, wsp, stream=stream)
+             for kc, vc in caches]
     app = [pa.prepare_append_fp8(kn, vn, sm, kc, vc, ks, vs, stream=stream) for kc, vc in caches]
     dec = [pa.prepare_decode_fp8(q, kc, vc, ks, vs, bt, cl, w.scale, out, wsp, stream=stream) for kc, vc in caches]
 
@@ -554,33 +679,51 @@ def run_pa_fp8(args, ws, rank, local):
         if flush is not None:
             flush.zero_()
 
+    clocks = ClockSampler(dev.index, enabled=not args.no_clocks)
     W_ = max(3, args.warmup)
+    for k in range(W_):
+        fused[k % ncopies]()
+        between()
+    torch.cuda.synchronize(dev)
+    rot = iter(range(1 << 62))
+    clocks.begin()
+    hold_load(lambda: fused[next(rot) % ncopies](), 0.3, dev, between)  # untimed: the clock samples see the load
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    _barrier(ws)
+    torch.cuda.synchronize(dev)
+    for k in range(K):
+        ev[k][0].record(stream)
+        fused[k % ncopies]()
+        ev[k][1].record(stream)
+        between()
+    torch.cuda.synchronize(dev)
+    _barrier(ws)
+    hold_load(lambda: fused[next(rot) % ncopies](), 0.2, dev, between)
+    clocks.end()
+    errs = pa.pa_device_errors(clear=True)
+    if errs:
+        raise RuntimeError(f"device error bits {errs:#x} during the benchmark")
+    total_ms = _max_over_ranks(sum(ev[k][0].elapsed_time(ev[k][1]) for k in range(K)), ws)
+
+    # ---- the same steps as two launches, for the split ----
     for k in range(W_):
         app[k % ncopies]()
         dec[k % ncopies]()
         between()
-    torch.cuda.synchronize(dev)
-    K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    clocks = ClockSampler(dev.index, enabled=not args.no_clocks)
-    _barrier(ws)
+    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     torch.cuda.synchronize(dev)
     for k in range(K):
         c = k % ncopies
-        ev[k][0].record(stream)
+        ev2[k][0].record(stream)
         app[c]()
-        ev[k][1].record(stream)
+        ev2[k][1].record(stream)
         dec[c]()
-        ev[k][2].record(stream)
+        ev2[k][2].record(stream)
         between()
     torch.cuda.synchronize(dev)
-    _barrier(ws)
-    errs = pa.pa_device_errors(clear=True)
-    if errs:
-        raise RuntimeError(f"device error bits {errs:#x} during the benchmark")
-    total_ms = _max_over_ranks(sum(ev[k][0].elapsed_time(ev[k][2]) for k in range(K)), ws)
-    app_avg = _max_over_ranks(sum(ev[k][0].elapsed_time(ev[k][1]) for k in range(K)) / K, ws)
-    dec_avg = _max_over_ranks(sum(ev[k][1].elapsed_time(ev[k][2]) for k in range(K)) / K, ws)
+    app_avg = _max_over_ranks(sum(ev2[k][0].elapsed_time(ev2[k][1]) for k in range(K)) / K, ws)
+    dec_avg = _max_over_ranks(sum(ev2[k][1].elapsed_time(ev2[k][2]) for k in range(K)) / K, ws)
 
     out_h = torch.empty(w.q.shape, dtype=torch.bfloat16).pin_memory()
     h2d = packed.nbytes
@@ -588,8 +731,7 @@ def run_pa_fp8(args, ws, rank, local):
 
     def e2e_step(c):
         packed.h2d()
-        app[c]()
-        dec[c]()
+        fused[c]()
         out_h.copy_(out, non_blocking=True)
 
     for k in range(3):
@@ -612,7 +754,7 @@ def run_pa_fp8(args, ws, rank, local):
         return
     peak, peak_kind = _peaks()
     step_avg = total_ms / K
-    achieved = dec_bytes / (dec_avg * 1e-3) / 1e9
+    achieved = step_bytes / (step_avg * 1e-3) / 1e9
     value = ws * K * step_bytes / (total_ms * 1e-3) / 1e9
     l2 = (f"inputs larger than L2: {ncopies} copies of the {pool_bytes / 1e6:.0f} MB fp8 cache rotated, "
           f"no flush" if rotate else "flushed between steps (256 MB write, outside the timed events)")
@@ -626,17 +768,19 @@ def run_pa_fp8(args, ws, rank, local):
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU", "l2": l2,
                    "unique_kv_bytes": workloads.unique_kv_bytes(w) // 2},
         "step_us": round(step_avg * 1e3, 2),
+        "two_launch_step_us": round((app_avg + dec_avg) * 1e3, 2),
         "decode_us": round(dec_avg * 1e3, 2),
         "append_us": round(app_avg * 1e3, 2),
-        "decode_only_gbs": round(achieved, 1),
+        "decode_only_gbs": round(dec_bytes / (dec_avg * 1e-3) / 1e9, 1),
+        "step_pct_of_hbm_peak": round(100 * achieved / peak, 1),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                     "kernel": "pa::decode_kernel<..., Fp8MmaMath> (pa_decode_fp8)",
+                     "kernel": "pa::decode_kernel<..., APPEND, Fp8MmaMath> (pa_append_decode_fp8)",
                      "traffic": _traffic(args.workload + ":fp8"),
-                     "algorithmic_bytes_per_launch": dec_bytes},
+                     "algorithmic_bytes_per_launch": step_bytes},
         "e2e": {"value": round(ws * K * step_bytes / (e2e_total * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_total / K, 5)},
-        "gpu_launches": 2 * K,
+        "gpu_launches": K,
         "clocks": clk,
     }
     if ws == 1 and not args.no_cpu_baseline:
@@ -706,13 +850,15 @@ def run_prefill(args, ws, rank, local, reference: bool):
     stream = torch.cuda.current_stream(dev)
     call = pa.prepare_prefill(t["q"], t["cu_q_lens"], pb.max_q_len, t["k_cache"], t["v_cache"], t["block_tables"],
                               t["context_lens"], pb.scale, out, stream=stream)
+    clocks = ClockSampler(dev.index, enabled=not args.no_clocks)
     W_ = max(3, args.warmup)
     for _ in range(W_):
         call()
     torch.cuda.synchronize(dev)
+    clocks.begin()
+    hold_load(call, 0.3, dev)  # untimed: the clock samples see the load
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
-    clocks = ClockSampler(dev.index, enabled=not args.no_clocks)
     _barrier(ws)
     torch.cuda.synchronize(dev)
     for k in range(K):
@@ -721,6 +867,8 @@ def run_prefill(args, ws, rank, local, reference: bool):
         ev[k][1].record(stream)
     torch.cuda.synchronize(dev)
     _barrier(ws)
+    hold_load(call, 0.2, dev)
+    clocks.end()
     clk = clocks.stop()
     errs = pa.pa_device_errors(clear=True)
     if errs:

@@ -130,7 +130,9 @@ PA_API int32_t pa_decode_default_ctas(void);
  * aligned.  The per-page math runs on the tensor cores (mma.sync, fp32
  * accumulation); setting the environment variable PA_DECODE_MATH=simt
  * before the first call selects the fp32 CUDA core variant instead
- * (head_dim*Hq/Hkv <= 256 only).  PA_SEG_WEIGHT_BYTES (read at the first
+ * (head_dim*Hq/Hkv <= 256 only).  Split pieces are merged in a fixed
+ * order, whatever order they finish in, so repeated calls on the same
+ * inputs give bit-identical outputs.  PA_SEG_WEIGHT_BYTES (read at the first
  * call; default 65536) is the fixed cost of finishing a (sequence, head
  * group) segment, in K+V bytes, that the equal-share split charges: larger
  * values cut short contexts into fewer split pieces.
@@ -144,9 +146,11 @@ PA_API pa_status pa_decode(const void* q, const void* k_cache, const void* v_cac
  * One decode step in one launch: the slot-mapped append of the step's new
  * K/V rows (pa_cache_append) and then paged decode attention over the
  * caches including those rows (pa_decode), fused.  Each CTA writes a slice
- * of the rows, then all CTAs meet at a grid barrier (a cooperative launch,
- * so all are resident) before any K/V page is read; the barrier wait
- * overlaps the kernel's own set-up.  Arguments as for the two calls; the
+ * of the rows and arrives at a grid barrier (a cooperative launch, so all
+ * CTAs are resident); a CTA waits there only before it reads a block that
+ * the step's rows go to (blocks marked in a hashed bitmap of the slots), so
+ * for a decode step, whose new rows sit in each sequence's last page, the
+ * wait is off the critical path.  Arguments as for the two calls; the
  * workspace as for pa_decode.  Compared with the two calls it saves the
  * append's launch and its latency (miniVLLM docs index, "What is
  * miniVLLM?": low-latency decode; the append and the decode of one step).
@@ -193,7 +197,12 @@ PA_API pa_status pa_decode_partials(const void* q, const void* k_cache, const vo
  *   - Nothing is allocated: no cudaMalloc/cudaFree, no allocating library call.
  *   - A problem whose scratch (pa_decode_workspace_bytes(dims, 0)) exceeds
  *     PA_STATIC_SCRATCH_BYTES is rejected with PA_ERR_SCRATCH_LIMIT before
- *     anything is launched.
+ *     anything is launched.  The scratch is two partial slots per CTA (one
+ *     CTA per SM) of min(Hkv, 8) * Hq/Hkv * head_dim fp32 values, plus 4
+ *     bytes per (sequence, kv head): on a 148-SM B200 the largest head shape
+ *     built (8 kv heads x a GQA group of 8, head_dim 128) takes 9.9 MB, so
+ *     every supported head shape fits with up to 1.7 million (sequence, kv
+ *     head) pairs (e.g. 200,000 sequences of 8 kv heads).
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.
@@ -203,7 +212,7 @@ PA_API pa_status pa_decode_partials(const void* q, const void* k_cache, const vo
  *     overlap on the GPU (different streams without ordering) race on the
  *     array and give undefined results: order them.
  */
-#define PA_STATIC_SCRATCH_BYTES (4u << 20)
+#define PA_STATIC_SCRATCH_BYTES (16u << 20)
 PA_API pa_status pa_decode_static_ws(const void* q, const void* k_cache, const void* v_cache,
                                      const int32_t* block_tables, const int32_t* context_lens,
                                      float scale, void* out, const pa_dims* dims, void* stream);
@@ -292,6 +301,22 @@ PA_API pa_status pa_decode_fp8(const void* q, const void* k_cache, const void* v
                                size_t workspace_bytes, void* stream);
 
 /*
+ * One fp8 decode step in one launch: pa_cache_append_fp8 of the step's new
+ * bf16 rows into the fp8 caches, then pa_decode_fp8 over the caches
+ * including them, fused as pa_append_decode fuses the bf16 calls (a
+ * cooperative launch; a CTA waits at the grid barrier only before reading a
+ * block the new rows go to).  Arguments, codes and results as for the two
+ * calls; the workspace as for pa_decode.  Graph-capturable like every call
+ * here (no allocation, no synchronisation).  After a call that set
+ * PA_DEVERR_TIMEOUT the workspace must be zero-filled again.
+ */
+PA_API pa_status pa_append_decode_fp8(const void* k_new, const void* v_new, const int32_t* slot_mapping,
+                                      int32_t num_tokens, const void* q, void* k_cache, void* v_cache,
+                                      const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                                      const int32_t* context_lens, float scale, void* out, const pa_dims* dims,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Multi-query (chunked prefill) attention over the paged cache, the step
  * beside decode in the pages' engines (miniVLLM docs index, "What is
  * miniVLLM?": flash attention for prefill; Mini-SGLang write-up, "Key
@@ -320,6 +345,20 @@ PA_API pa_status pa_decode_fp8(const void* q, const void* k_cache, const void* v
 PA_API pa_status pa_prefill(const void* q, const int32_t* cu_q_lens, int32_t max_q_len, const void* k_cache,
                             const void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
                             float scale, void* out, const pa_dims* dims, void* stream);
+
+/*
+ * Test hook for the bounded waits (no counterpart in the pages).  Every wait
+ * of the kernels above gives up after a time limit instead of spinning for
+ * ever, sets PA_DEVERR_TIMEOUT and lets the kernel return, so that a broken
+ * pipeline leaves the GPU usable.  This call makes such waits run out on
+ * purpose: one CTA on `stream` waits, with the bounded polling wait of the
+ * decode pipeline and then with the sleeping wait of the prefill pipeline,
+ * on a shared-memory mbarrier that nothing arrives on, each for `limit_ns`
+ * nanoseconds, and returns.  limit_ns must lie in [1000, 1000000000]
+ * (else PA_ERR_SHAPE).  Afterwards pa_device_errors() reports
+ * PA_DEVERR_TIMEOUT and the device stays usable.
+ */
+PA_API pa_status pa_test_wait_timeout(int64_t limit_ns, void* stream);
 
 /*
  * Reads (and, if `clear` != 0, resets) the device error word of the

@@ -69,10 +69,14 @@ def _load(path: str = LIB_PATH):
     lib.pa_cache_append_fp8.restype = i32
     lib.pa_decode_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, f32, vp, dp, vp, sz, vp]
     lib.pa_decode_fp8.restype = i32
+    lib.pa_append_decode_fp8.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, f32, vp, dp, vp, sz, vp]
+    lib.pa_append_decode_fp8.restype = i32
     lib.pa_prefill.argtypes = [vp, vp, i32, vp, vp, vp, vp, f32, vp, dp, vp]
     lib.pa_prefill.restype = i32
     lib.pa_decode_static_ws.argtypes = [vp, vp, vp, vp, vp, f32, vp, dp, vp]
     lib.pa_decode_static_ws.restype = i32
+    lib.pa_test_wait_timeout.argtypes = [ctypes.c_int64, vp]
+    lib.pa_test_wait_timeout.restype = i32
     lib.pa_device_errors.argtypes = [ctypes.POINTER(i32), i32]
     lib.pa_device_errors.restype = i32
     lib.pa_status_string.argtypes = [i32]
@@ -86,10 +90,10 @@ lib = _load()
 EXPORTS = ("pa_cache_append", "pa_decode_workspace_bytes", "pa_decode_default_ctas", "pa_decode",
            "pa_append_decode", "pa_decode_partials", "pa_decode_static_ws",
            "pa_decode_shared_prefix_workspace_bytes", "pa_decode_shared_prefix", "pa_cache_append_fp8",
-           "pa_decode_fp8", "pa_prefill", "pa_device_errors", "pa_status_string")
+           "pa_decode_fp8", "pa_append_decode_fp8", "pa_prefill", "pa_test_wait_timeout", "pa_device_errors", "pa_status_string")
 
 PA_ERR_SCRATCH_LIMIT = -7
-PA_STATIC_SCRATCH_BYTES = 4 << 20  # include/pa.h
+PA_STATIC_SCRATCH_BYTES = 16 << 20  # include/pa.h
 
 
 def pa_status_string(code: int) -> str:
@@ -388,6 +392,46 @@ def pa_decode_fp8(q, k_cache8, v_cache8, k_scale, v_scale, block_tables, context
                              _ptr(workspace), workspace.numel(), _stream(stream)), "pa_decode_fp8")
 
 
+def _append_decode_fp8_args(k_new, v_new, slot_mapping, q, k_cache8, v_cache8, k_scale, v_scale, block_tables,
+                            context_lens, out):
+    dims = _decode_fp8_args(q, k_cache8, v_cache8, k_scale, v_scale, block_tables, context_lens, out)
+    for t, n in ((k_new, "k_new"), (v_new, "v_new")):
+        _need(t, torch.bfloat16, n, 3)
+    _need(slot_mapping, torch.int32, "slot_mapping", 1)
+    T = slot_mapping.shape[0]
+    if k_new.shape != v_new.shape or k_new.shape[0] != T or k_new.shape[1:] != (dims.num_kv_heads, dims.head_dim):
+        raise ValueError("k_new/v_new must be [T][Hkv][D] of the cache")
+    return dims, T
+
+
+def pa_append_decode_fp8(k_new, v_new, slot_mapping, q, k_cache8, v_cache8, k_scale, v_scale, block_tables,
+                         context_lens, scale: float, out, workspace=None, stream=None) -> None:
+    """pa_cache_append_fp8 then pa_decode_fp8, fused into one launch."""
+    dims, T = _append_decode_fp8_args(k_new, v_new, slot_mapping, q, k_cache8, v_cache8, k_scale, v_scale,
+                                      block_tables, context_lens, out)
+    if workspace is None:
+        workspace = alloc_workspace(dims, device=q.device)
+    _need(workspace, torch.uint8, "workspace", 1)
+    _check(lib.pa_append_decode_fp8(_ptr(k_new), _ptr(v_new), _ptr(slot_mapping), T, _ptr(q), _ptr(k_cache8),
+                                    _ptr(v_cache8), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+                                    _ptr(context_lens), float(scale), _ptr(out), ctypes.byref(dims), _ptr(workspace),
+                                    workspace.numel(), _stream(stream)), "pa_append_decode_fp8")
+
+
+def prepare_append_decode_fp8(k_new, v_new, slot_mapping, q, k_cache8, v_cache8, k_scale, v_scale, block_tables,
+                              context_lens, scale: float, out, workspace, stream=None) -> "Prepared":
+    dims, T = _append_decode_fp8_args(k_new, v_new, slot_mapping, q, k_cache8, v_cache8, k_scale, v_scale,
+                                      block_tables, context_lens, out)
+    _need(workspace, torch.uint8, "workspace", 1)
+    p = Prepared(lib.pa_append_decode_fp8,
+                 (_ptr(k_new), _ptr(v_new), _ptr(slot_mapping), T, _ptr(q), _ptr(k_cache8), _ptr(v_cache8),
+                  _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), _ptr(context_lens), float(scale), _ptr(out),
+                  ctypes.byref(dims), _ptr(workspace), workspace.numel(), _stream(stream)), "pa_append_decode_fp8")
+    p._keep = (dims, k_new, v_new, slot_mapping, q, k_cache8, v_cache8, k_scale, v_scale, block_tables,
+               context_lens, out, workspace)
+    return p
+
+
 def prepare_append_fp8(k_new, v_new, slot_mapping, k_cache8, v_cache8, k_scale, v_scale, stream=None) -> "Prepared":
     NB, Hkv, D = _fp8_cache_args(k_cache8, v_cache8, k_scale, v_scale)
     dims = pa_dims(0, Hkv, Hkv, D, 16, NB, 0)
@@ -446,6 +490,12 @@ def prepare_prefill(q, cu_q_lens, max_q_len: int, k_cache, v_cache, block_tables
                   _ptr(context_lens), float(scale), _ptr(out), ctypes.byref(dims), _stream(stream)), "pa_prefill")
     p._keep = (dims, q, cu_q_lens, k_cache, v_cache, block_tables, context_lens, out)
     return p
+
+
+def pa_test_wait_timeout(limit_ns: int, stream=None) -> None:
+    """Test hook: one CTA whose bounded waits run out after limit_ns each
+    (they set PA_DEVERR_TIMEOUT and return); see include/pa.h."""
+    _check(lib.pa_test_wait_timeout(int(limit_ns), _stream(stream)), "pa_test_wait_timeout")
 
 
 def pa_device_errors(clear: bool = False) -> int:

@@ -269,8 +269,8 @@ pa_status launch_decode(const pa::DecodeParams& p, int grid, cudaStream_t stream
 // The SIMT policy is built only for G*D <= 256 (its per-lane state grows with G*D).
 template <MathKind MK, int D, int G, bool DUMP, bool APPEND>
 pa_status launch_built(const pa::DecodeParams& p, int grid, cudaStream_t s, bool pdl) {
-    if constexpr (MK == MathKind::kFp8 && (DUMP || APPEND))
-        return PA_ERR_UNSUPPORTED;  // fp8: the plain decode only
+    if constexpr (MK == MathKind::kFp8 && DUMP)
+        return PA_ERR_UNSUPPORTED;  // fp8: no partials test hook
     else if constexpr (MK != MathKind::kSimt || G * D <= 256)
         return launch_decode<MK, D, G, DUMP, APPEND>(p, grid, s, pdl);
     else
@@ -703,6 +703,7 @@ pa_status pa_append_decode(const void* k_new, const void* v_new, const int32_t* 
     p.v_new = static_cast<const uint4*>(v_new);
     p.slot_mapping = slot_mapping;
     p.app_chunks = int64_t(num_tokens) * dims->num_kv_heads * (dims->head_dim / 8);
+    p.app_tokens = num_tokens;
     p.k_cache_w = static_cast<uint4*>(k_cache);
     p.v_cache_w = static_cast<uint4*>(v_cache);
     return dispatch_decode<false, true>(dims->head_dim, dims->num_q_heads / dims->num_kv_heads, p, grid,
@@ -802,6 +803,7 @@ pa_status pa_decode_shared_prefix(const void* k_new, const void* v_new, const in
     p.v_new = static_cast<const uint4*>(v_new);
     p.slot_mapping = slot_mapping;
     p.app_chunks = int64_t(num_tokens) * d.num_kv_heads * (d.head_dim / 8);
+    p.app_tokens = num_tokens;
     p.k_cache_w = static_cast<uint4*>(k_cache);
     p.v_cache_w = static_cast<uint4*>(v_cache);
     return dispatch_decode<false, true>(d.head_dim, G, p, grid, s);
@@ -880,6 +882,39 @@ pa_status pa_decode_fp8(const void* q, const void* k_cache, const void* v_cache,
                                                       grid, static_cast<cudaStream_t>(stream), false);
 }
 
+pa_status pa_append_decode_fp8(const void* k_new, const void* v_new, const int32_t* slot_mapping, int32_t num_tokens,
+                               const void* q, void* k_cache, void* v_cache, const float* k_scale, const float* v_scale,
+                               const int32_t* block_tables, const int32_t* context_lens, float scale, void* out,
+                               const pa_dims* dims, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!dims) return PA_ERR_NULL;
+    if (num_tokens < 0) return PA_ERR_SHAPE;
+    pa::DecodeParams p;
+    const int grid = sm_count();
+    const pa_status st = prepare_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, dims, grid,
+                                        workspace, workspace_bytes, p, /*eb=*/1);
+    if (st != PA_OK) return st;
+    if (!k_scale || !v_scale) return PA_ERR_NULL;
+    if (!aligned4(k_scale) || !aligned4(v_scale)) return PA_ERR_ALIGN;
+    if (num_tokens > 0) {
+        if (!k_new || !v_new || !slot_mapping) return PA_ERR_NULL;
+        if (!aligned16(k_new) || !aligned16(v_new) || !aligned4(slot_mapping)) return PA_ERR_ALIGN;
+    }
+    if (dims->num_seqs == 0)  // nothing to attend over: the append alone
+        return pa_cache_append_fp8(k_new, v_new, slot_mapping, num_tokens, k_cache, v_cache, k_scale, v_scale, dims,
+                                   stream);
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.k_new = static_cast<const uint4*>(k_new);
+    p.v_new = static_cast<const uint4*>(v_new);
+    p.slot_mapping = slot_mapping;
+    p.app_chunks = int64_t(num_tokens) * dims->num_kv_heads * (dims->head_dim / 8);
+    p.app_tokens = num_tokens;
+    p.k_cache_w = static_cast<uint4*>(k_cache);
+    p.v_cache_w = static_cast<uint4*>(v_cache);
+    return dispatch_d_g<MathKind::kFp8, false, true>(dims->head_dim, dims->num_q_heads / dims->num_kv_heads, p, grid,
+                                                     static_cast<cudaStream_t>(stream), false);
+}
+
 pa_status pa_prefill(const void* q, const int32_t* cu_q_lens, int32_t max_q_len, const void* k_cache,
                      const void* v_cache, const int32_t* block_tables, const int32_t* context_lens, float scale,
                      void* out, const pa_dims* dims, void* stream) {
@@ -922,6 +957,12 @@ pa_status pa_prefill(const void* q, const int32_t* cu_q_lens, int32_t max_q_len,
     const dim3 grid(unsigned(d.num_seqs * tiles), unsigned(d.num_kv_heads));
     return sync_mma ? dispatch_prefill(d.head_dim, G, p, grid, static_cast<cudaStream_t>(stream))
                     : dispatch_prefill_tc(d.head_dim, G, p, grid, static_cast<cudaStream_t>(stream));
+}
+
+pa_status pa_test_wait_timeout(int64_t limit_ns, void* stream) {
+    if (limit_ns < 1000 || limit_ns > 1000000000LL) return PA_ERR_SHAPE;
+    pa::wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(uint64_t(limit_ns));
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 pa_status pa_device_errors(int32_t* errors_out, int32_t clear) {

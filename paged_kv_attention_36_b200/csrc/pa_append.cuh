@@ -73,26 +73,30 @@ struct AppendFp8Params {
 
 __device__ __forceinline__ int vt_position(int t) { return 4 * ((t & 7) >> 1) + 2 * (t >> 3) + (t & 1); }
 
-__global__ void __launch_bounds__(kAppendThreads) append_fp8_kernel(AppendFp8Params p) {
-    const int64_t idx = int64_t(blockIdx.x) * kAppendThreads + threadIdx.x;
-    if (idx >= p.num_chunks) return;
-    const int64_t per_token = int64_t(p.kv_heads) * p.chunks_per_row;
+// Encodes and stores chunk idx (8 values of one (token, kv head) row of K
+// and of V) of the step's new rows; the body of append_fp8_kernel, also run
+// by the fused fp8 append + decode.
+__device__ __forceinline__ void append_fp8_chunk(const uint4* k_new, const uint4* v_new, const int32_t* slot_mapping,
+                                                 uint8_t* k_cache, uint8_t* v_cache, const float* k_scale,
+                                                 const float* v_scale, int kv_heads, int chunks_per_row,
+                                                 int num_blocks, int64_t idx) {
+    const int64_t per_token = int64_t(kv_heads) * chunks_per_row;
     const int64_t t = idx / per_token;
     const int64_t rem = idx - t * per_token;
-    const int32_t slot = __ldg(p.slot_mapping + t);
+    const int32_t slot = __ldg(slot_mapping + t);
     if (slot < 0) return;
     const int64_t block = slot >> 4;
     const int offset = slot & 15;
-    if (block >= p.num_blocks) {
+    if (block >= num_blocks) {
         if (rem == 0) raise_error(PA_DEVERR_SLOT);
         return;
     }
-    const int g = int(rem / p.chunks_per_row);
-    const int c = int(rem - int64_t(g) * p.chunks_per_row);
-    const int D = p.chunks_per_row * 8;
-    const int64_t tile = block * p.kv_heads + g;
-    const float ks = __ldg(p.k_scale + g), vs = __ldg(p.v_scale + g);
-    const uint4 kv = __ldg(p.k_new + idx), vv = __ldg(p.v_new + idx);
+    const int g = int(rem / chunks_per_row);
+    const int c = int(rem - int64_t(g) * chunks_per_row);
+    const int D = chunks_per_row * 8;
+    const int64_t tile = block * kv_heads + g;
+    const float ks = __ldg(k_scale + g), vs = __ldg(v_scale + g);
+    const uint4 kv = __ldg(k_new + idx), vv = __ldg(v_new + idx);
     const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w}, vw[4] = {vv.x, vv.y, vv.z, vv.w};
     uint16_t k8[4], v8[4];
 #pragma unroll
@@ -102,15 +106,22 @@ __global__ void __launch_bounds__(kAppendThreads) append_fp8_kernel(AppendFp8Par
         v8[j] = f32x2_to_e4m3x2(__fdiv_rn(vf.x, vs), __fdiv_rn(vf.y, vs));
     }
     // K: 8 consecutive codes of row `offset`
-    *reinterpret_cast<uint2*>(p.k_cache + (tile * 16 + offset) * D + c * 8) =
+    *reinterpret_cast<uint2*>(k_cache + (tile * 16 + offset) * D + c * 8) =
         make_uint2(uint32_t(k8[0]) | (uint32_t(k8[1]) << 16), uint32_t(k8[2]) | (uint32_t(k8[3]) << 16));
     // V: one code in each of the rows c*8 .. c*8+7 of the transposed tile
-    uint8_t* vrow = p.v_cache + (tile * D + c * 8) * 16 + vt_position(offset);
+    uint8_t* vrow = v_cache + (tile * D + c * 8) * 16 + vt_position(offset);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         vrow[(2 * j) * 16] = uint8_t(v8[j] & 0xff);
         vrow[(2 * j + 1) * 16] = uint8_t(v8[j] >> 8);
     }
+}
+
+__global__ void __launch_bounds__(kAppendThreads) append_fp8_kernel(AppendFp8Params p) {
+    const int64_t idx = int64_t(blockIdx.x) * kAppendThreads + threadIdx.x;
+    if (idx >= p.num_chunks) return;
+    append_fp8_chunk(p.k_new, p.v_new, p.slot_mapping, p.k_cache, p.v_cache, p.k_scale, p.v_scale, p.kv_heads,
+                     p.chunks_per_row, p.num_blocks, idx);
 }
 
 }  // namespace pa

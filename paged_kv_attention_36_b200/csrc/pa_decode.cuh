@@ -15,11 +15,14 @@
 // log-sum-exp (flash-decoding), so long or skewed contexts are split exactly
 // where the balance needs it and nowhere else.  A (b, kv head) in two
 // pieces takes its merge ticket first: the first piece to finish publishes
-// its partial with a ready flag and the other folds it into its own
+// its partial with a ready flag and the other merges it with its own
 // registers, so the merge adds two memory round trips to that CTA.  More
 // pieces publish first and the last merges from memory, in two levels
 // beyond 16 pieces: the last piece to finish in each run of 16 merges that
 // run, and the last run merges the runs, so no CTA reads more than 16.
+// Every merge combines normalised partials in a fixed (leaf) order, so the
+// output does not depend on the order in which pieces finish: repeated
+// calls give bit-identical results.
 //
 // Inside a CTA.  Warp 8 (the producer) walks the share, reads one block id
 // per page from the block table and copies the page into a ring of R
@@ -54,6 +57,7 @@
 //     mantissa bits; the softmax bookkeeping stays in fp32 registers.
 #pragma once
 
+#include "pa_append.cuh"
 #include "pa_device.cuh"
 #include "pa_prefix.cuh"
 
@@ -97,6 +101,7 @@ struct DecodeParams {
     const uint4* v_new;
     const int32_t* slot_mapping;  // [T]
     int64_t app_chunks;           // T * Hkv * D / 8
+    int32_t app_tokens;           // T
     uint4* k_cache_w;             // the caches, writable
     uint4* v_cache_w;
     unsigned int* grid_bar;       // {arrivals, departures}: zero between calls
@@ -138,6 +143,7 @@ struct Split {
 // Shared scalars.
 struct Misc {
     int abort;
+    int all_dirty;       // fused append: every page counts as written this step
     int b0;              // sequence where the share starts
     long long pre0;      // weighted position of b0's first unit
     long long red[16];  // block reductions, one slot per warp (<= 16 warps)
@@ -348,6 +354,47 @@ struct SimtMath {
             }
         }
     }
+    // After finish(): out[h][:] (bf16) = the log-sum-exp merge of this
+    // state with the finished partial pc of the same (b, kv head), both
+    // taken as normalised partials (this state as store_partial would write
+    // it) and combined in leaf order (this one first iff mine_first): the
+    // result does not depend on which of the two pieces finished last.
+    __device__ __forceinline__ void store_merged2(const Piece& pc, bool mine_first, __nv_bfloat16* out,
+                                                  int lane) const {
+        const int tg = lane >> 3, c = lane & 7;
+        if (tg != 0) return;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float2 oml = __ldcg(pc.ml + h);
+            const float inv = 1.f / l[h];
+            const float ma = mine_first ? m[h] : oml.x, la = mine_first ? l[h] : oml.y;
+            const float mb = mine_first ? oml.x : m[h], lb = mine_first ? oml.y : l[h];
+            const float M = fmaxf(ma, mb);
+            const float wa = la * exp2f(ma - M), wb = lb * exp2f(mb - M);
+            const float r = oscale / (wa + wb);
+#pragma unroll
+            for (int i = 0; i < NCH; ++i) {
+                const float4* src = reinterpret_cast<const float4*>(pc.o + h * D + (c + 8 * i) * 8);
+                const float4 q0 = __ldcg(src), q1 = __ldcg(src + 1);
+                const float other[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+                float res[8];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float own0 = acc[h][i][j].x * inv, own1 = acc[h][i][j].y * inv;
+                    const float a0 = mine_first ? own0 : other[2 * j], b0 = mine_first ? other[2 * j] : own0;
+                    const float a1 = mine_first ? own1 : other[2 * j + 1], b1 = mine_first ? other[2 * j + 1] : own1;
+                    res[2 * j] = (wa * a0 + wb * b0) * r;
+                    res[2 * j + 1] = (wa * a1 + wb * b1) * r;
+                }
+                uint4 v;
+                v.x = float2_to_bf16x2(res[0], res[1]);
+                v.y = float2_to_bf16x2(res[2], res[3]);
+                v.z = float2_to_bf16x2(res[4], res[5]);
+                v.w = float2_to_bf16x2(res[6], res[7]);
+                *reinterpret_cast<uint4*>(out + h * D + (c + 8 * i) * 8) = v;
+            }
+        }
+    }
     // After finish(): o[h][:] = acc / l (fp32) and the (max logit base 2,
     // exp-sum) pair of each head: to ml[h] if ml, else m (natural log units)
     // to mo[h] and l to lo[h].
@@ -551,6 +598,35 @@ struct MmaMath {
             for (int mt = 0; mt < KS; ++mt) {
                 out[h * D + 16 * mt + d0] = __float2bfloat16_rn(acc[mt][e] * inv);
                 out[h * D + 16 * mt + d0 + 8] = __float2bfloat16_rn(acc[mt][2 + e] * inv);
+            }
+        }
+    }
+    // After finish(): out[h][:] (bf16) = the log-sum-exp merge of this
+    // state with the finished partial pc of the same (b, kv head), both
+    // taken as normalised partials (this state as store_partial would write
+    // it) and combined in leaf order (this one first iff mine_first): the
+    // result does not depend on which of the two pieces finished last.
+    __device__ __forceinline__ void store_merged2(const Piece& pc, bool mine_first, __nv_bfloat16* out,
+                                                  int lane) const {
+        const int h0 = (lane & 3) * 2, d0 = lane >> 2;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int h = h0 + e;
+            if (h >= G) continue;
+            const float inv = 1.f / l[e];
+            const float ma = mine_first ? m[e] : pc.ml[e].x, la = mine_first ? l[e] : pc.ml[e].y;
+            const float mb = mine_first ? pc.ml[e].x : m[e], lb = mine_first ? pc.ml[e].y : l[e];
+            const float M = fmaxf(ma, mb);
+            const float wa = la * exp2f(ma - M), wb = lb * exp2f(mb - M);
+            const float r = oscale / (wa + wb);
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const float own = acc[mt][2 * k + e] * inv, other = pc.o[mt][2 * k + e];
+                    const float a = mine_first ? own : other, b = mine_first ? other : own;
+                    out[h * D + 16 * mt + d0 + 8 * k] = __float2bfloat16_rn((wa * a + wb * b) * r);
+                }
             }
         }
     }
@@ -819,7 +895,11 @@ struct DecodeCfg {
     static constexpr int kNumBars = 2 * R + 2 * kSegSlots;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kMiscBytes = 256;
-    static constexpr int kSmemBytes = kMiscOff + kMiscBytes + 1024;  // + alignment slack
+    // fused append: a bitmap of the blocks the step's append writes, hashed
+    // by block id (bit blk % kDirtyBits)
+    static constexpr int kDirtyOff = kMiscOff + kMiscBytes;
+    static constexpr int kDirtyBytes = 1024;
+    static constexpr int kSmemBytes = kDirtyOff + kDirtyBytes + 1024;  // + alignment slack
     static_assert(kTile % 1024 == 0 && kStage % 1024 == 0, "TMA tile alignment (128-byte swizzle)");
     static_assert(kBarOff % 8 == 0, "mbarrier alignment");
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
@@ -1016,6 +1096,54 @@ __device__ __noinline__ void merge_pieces(const DecodeParams& p, int k0, int off
     }
 }
 
+// Fused append.  Every CTA writes a slice of the step's new rows and
+// arrives at a grid barrier (grid_bar[0] counts arrivals).  A CTA must not
+// read a block those rows go to before every CTA has arrived, but most pages
+// are not written this step: each CTA marks the written blocks in a hashed
+// bitmap, and its producer waits at the barrier only before the first page
+// whose block is marked (a hash collision only makes it wait earlier).
+constexpr int kDirtyMaxTokens = 2048;  // more appended tokens: every page counts as written
+
+__device__ __forceinline__ bool block_marked(const uint32_t* map, int words, int32_t blk) {
+    const uint32_t bit = uint32_t(blk) % uint32_t(words * 32);
+    return (map[bit >> 5] >> (bit & 31)) & 1u;
+}
+
+// Waits, in every lane of the calling warp, until all CTAs have arrived
+// (bounded in time); then orders the lane's later TMA (async-proxy) reads
+// after the rows they wrote.  False if it gave up or *abort was set.
+__device__ __forceinline__ bool wait_rows_written(const DecodeParams& p, volatile int* abort) {
+    const uint64_t t0 = globaltimer_ns();
+    bool ok = true;
+    for (uint32_t it = 0; ld_acquire_gpu(&p.grid_bar[0]) < gridDim.x; ++it) {
+        __nanosleep(32);
+        if ((it & 63u) == 63u) {
+            if (*abort) {
+                ok = false;
+                break;
+            }
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                raise_error(PA_DEVERR_TIMEOUT);
+                *abort = 1;
+                ok = false;
+                break;
+            }
+        }
+    }
+    ok = __all_sync(0xffffffffu, ok);
+    fence_proxy_async_global();
+    return ok;
+}
+
+// Each CTA departs once, after its last read of the arrival count; the last
+// one to depart (when no CTA can still be waiting) resets the barrier.
+__device__ __forceinline__ void depart_grid(const DecodeParams& p) {
+    if (atomicAdd(&p.grid_bar[1], 1u) == gridDim.x - 1) {
+        p.grid_bar[0] = 0;
+        p.grid_bar[1] = 0;
+    }
+}
+
 template <int D, int G, int BS, int R, bool DUMP, bool APPEND, template <int, int, int> class Math>
 __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
     using Cfg = DecodeCfg<D, BS, R, Math<D, G, BS>::kElemBytes>;
@@ -1034,6 +1162,8 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
     uint64_t* segempty = segfull + S;
     Misc* misc = reinterpret_cast<Misc*>(smem + Cfg::kMiscOff);
     volatile int* abort = &misc->abort;
+    uint32_t* dirty_map = reinterpret_cast<uint32_t*>(smem + Cfg::kDirtyOff);
+    constexpr int kDirtyWords = Cfg::kDirtyBytes / 4;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int HG = p.HG, HS = p.HS, SPL = p.SPL;
@@ -1052,14 +1182,33 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
     }
 
     if (APPEND) {
+        // The blocks this step's rows go to, marked in the hashed bitmap.
+        for (int i = threadIdx.x; i < kDirtyWords; i += NT) dirty_map[i] = 0u;
+        if (threadIdx.x == 0) misc->all_dirty = p.app_tokens > kDirtyMaxTokens;
+        __syncthreads();
+        if (p.app_tokens <= kDirtyMaxTokens) {
+            for (int t = threadIdx.x; t < p.app_tokens; t += NT) {
+                const int32_t slot = __ldg(p.slot_mapping + t);
+                if (slot < 0) continue;
+                const uint32_t bit = uint32_t(slot / BS) % uint32_t(kDirtyWords * 32);
+                atomicOr(&dirty_map[bit >> 5], 1u << (bit & 31));
+            }
+        }
         // This CTA's slice of the slot-mapped append (the bit copy of
-        // pa::append_kernel), then arrival at the grid barrier; the rows must
-        // be visible to the TMA loads of every CTA before any page is read.
+        // pa::append_kernel, or the E4M3 encoding of pa::append_fp8_kernel
+        // for fp8 caches), then arrival at the grid barrier; a written row
+        // must be visible to the TMA loads of every CTA that reads its block.
         const int64_t per = (p.app_chunks + gridDim.x - 1) / gridDim.x;
         const int64_t c0 = int64_t(blockIdx.x) * per;
         const int64_t c1 = c0 + per < p.app_chunks ? c0 + per : p.app_chunks;
         constexpr int CPR = D / 8;  // 16-byte chunks per row
         for (int64_t idx = c0 + threadIdx.x; idx < c1; idx += NT) {
+            if constexpr (Math<D, G, BS>::kElemBytes == 1) {  // fp8 caches: encode (pa::append_fp8_kernel)
+                append_fp8_chunk(p.k_new, p.v_new, p.slot_mapping, reinterpret_cast<uint8_t*>(p.k_cache_w),
+                                 reinterpret_cast<uint8_t*>(p.v_cache_w), p.k_scale, p.v_scale, p.Hkv, CPR, p.NB,
+                                 idx);
+                continue;
+            }
             const int64_t t = idx / (int64_t(p.Hkv) * CPR);
             const int64_t rem = idx - t * p.Hkv * CPR;
             const int32_t slot = __ldg(p.slot_mapping + t);
@@ -1102,28 +1251,6 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
         v_mine = v;
         incl_mine = incl;
     }
-    if (APPEND) {
-        // wait for every CTA's rows (all CTAs are resident: a cooperative
-        // launch); the last CTA through resets the barrier for the next call
-        if (threadIdx.x == 0) {
-            const uint64_t t0 = globaltimer_ns();
-            for (uint32_t it = 0; ld_acquire_gpu(&p.grid_bar[0]) < gridDim.x; ++it) {
-                __nanosleep(32);
-                if ((it & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) {
-                    raise_error(PA_DEVERR_TIMEOUT);
-                    misc->abort = 1;
-                    break;
-                }
-            }
-            if (atomicAdd(&p.grid_bar[1], 1u) == gridDim.x - 1) {
-                p.grid_bar[0] = 0;
-                p.grid_bar[1] = 0;
-            }
-        }
-        __syncthreads();
-        fence_proxy_async_global();
-        if (misc->abort) return;
-    }
     // A decode launched right after prefix_kernel (programmatic dependent
     // launch) has done the set-up above meanwhile; the prefix partials and
     // the rows that kernel appended are read only after this wait (a no-op
@@ -1153,10 +1280,12 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
             }
         }
     }
-    if (Wt == 0) return;
     const int64_t want = (Wt + p.min_pages - 1) / p.min_pages;
     const int64_t grid_eff = want < int64_t(gridDim.x) ? want : int64_t(gridDim.x);
-    if (int64_t(blockIdx.x) >= grid_eff) return;
+    if (Wt == 0 || int64_t(blockIdx.x) >= grid_eff) {  // no share: read no page
+        if (APPEND && threadIdx.x == 0) depart_grid(p);
+        return;
+    }
     const Split split{Wt / grid_eff, Wt % grid_eff};
     const int64_t p_start = split.start(blockIdx.x);
     const int64_t p_end = split.start(int64_t(blockIdx.x) + 1);
@@ -1197,6 +1326,7 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
         uint32_t stage_i = 0, seg_i = 0;
         constexpr int C = R < 32 ? R : 32;
         bool ok = true;
+        bool rows_ready = !APPEND;  // fused append: every CTA's rows are visible
         const uint64_t pol = PA_EVICT_FIRST ? policy_evict_first() : policy_evict_normal();
         const uint32_t stage_tx = uint32_t(2 * HS * Cfg::kTile);
 
@@ -1237,14 +1367,28 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
                 for (int c0 = 0; ok && c0 < nst; c0 += C) {
                     const int n = (nst - c0) < C ? (nst - c0) : C;
                     bool lane_ok = true;
+                    int32_t blk = 0;
                     if (lane < n) {
-                        const int x = c0 + lane;
-                        const int pg = x >> p.SPL_LOG, sub = x & (SPL - 1);
-                        int32_t blk = __ldg(bt + pg);
+                        blk = __ldg(bt + ((c0 + lane) >> p.SPL_LOG));
                         if (blk < 0 || blk >= p.NB) {
                             raise_error(PA_DEVERR_BLOCK_ID);
                             blk = 0;
                         }
+                    }
+                    if (APPEND && !rows_ready) {
+                        const bool marked =
+                            lane < n && (misc->all_dirty || block_marked(dirty_map, kDirtyWords, blk));
+                        if (__any_sync(0xffffffffu, marked)) {
+                            rows_ready = true;
+                            if (!wait_rows_written(p, abort)) {
+                                ok = false;
+                                break;
+                            }
+                        }
+                    }
+                    if (lane < n) {
+                        const int x = c0 + lane;
+                        const int sub = x & (SPL - 1);
                         const uint32_t i = stage_i + x;
                         const int slot = int(i % R);
                         const uint32_t use = i / R;
@@ -1292,6 +1436,7 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
             for (uint32_t i = (last > R ? last - R : 0); i < last; ++i)
                 mbar_wait(&full[i % R], (i / R) & 1, nullptr, 20000000ull);
         }
+        if (APPEND && lane == 0) depart_grid(p);
         return;
     }
     if (warp >= HG) return;
@@ -1389,8 +1534,8 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
         const int leaf = int(blockIdx.x) - d.k0;
         int32_t* top = p.counters + int64_t(d.b) * p.Hkv + g;
         if (!DUMP && !whole && nk <= kFastMergePieces) {
-            // ticket first; the second piece to finish folds the first one's
-            // published partial into its registers
+            // ticket first; the second piece to finish merges the first one's
+            // published partial with its own registers, in leaf order
             if (ticket(top, nk, lane)) {
                 const int64_t sl = leaf_slot(d.k0, 1 - leaf);
                 const int* flag = p.slot_sync + sl * HG + warp;
@@ -1404,9 +1549,10 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
                 }
                 __syncwarp();
                 const int64_t ps = sl * hgG + int64_t(warp) * G;
-                st.absorb(p.part_o + ps * D, p.part_ml + ps, lane);
+                typename MathT::Piece other;
+                st.piece_load(other, p.part_o + ps * D, p.part_ml + ps, lane);
                 st.finish();
-                st.store_out(p.out + row * D, lane);
+                st.store_merged2(other, leaf == 0, p.out + row * D, lane);
                 __syncwarp();
                 if (lane == 0) {
                     p.slot_sync[sl * HG + warp] = 0;

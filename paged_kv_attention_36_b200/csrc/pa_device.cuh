@@ -135,6 +135,26 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, 
     }
 }
 
+// Makes both bounded waits above run out: thread 0 waits on a barrier that
+// nothing arrives on, first polling (mbar_wait), then sleeping
+// (mbar_wait_sleep), each for limit_ns; each sets PA_DEVERR_TIMEOUT when it
+// gives up.  Used only by the test hook pa_test_wait_timeout.
+__global__ void wait_timeout_kernel(uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_poll, abort_sleep;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_poll = 0;
+        abort_sleep = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        mbar_wait(&bar, 0, &abort_poll, limit_ns);
+        mbar_wait_sleep(&bar, 0, &abort_sleep, limit_ns);
+    }
+}
+
 // ---- 1-D bulk copy global -> shared, completing on an mbarrier ------------
 // Both addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {

@@ -40,3 +40,33 @@ def test_packed_inputs_views(monkeypatch):
     p.host.zero_()
     p.h2d()
     assert all(int(v.abs().sum()) == 0 for v in (p.views["bt"], p.views["cl"]))
+
+
+def test_clock_sampler_keeps_only_samples_inside_windows(monkeypatch):
+    # the sampler process is replaced by injected lines; end() takes one
+    # synchronous query (faked here) so every window has a sample
+    import subprocess
+    import types
+
+    import bench
+
+    def no_popen(*a, **k):
+        raise OSError("no nvidia-smi here")
+
+    monkeypatch.setattr(subprocess, "Popen", no_popen)
+    line = "0, {sm}, 1965, 700.0, 0x0, Not Active, Not Active, Not Active, {cap}\n"
+    monkeypatch.setattr(subprocess, "run", lambda *a, **k: types.SimpleNamespace(
+        stdout=line.format(sm=1900, cap="Active")))
+    c = bench.ClockSampler(0, enabled=True)
+    c.samples = [(1.0, line.format(sm=500, cap="Not Active")),    # before the window: idle, dropped
+                 (2.5, line.format(sm=1965, cap="Not Active"))]
+    monkeypatch.setattr(bench.time, "time", lambda: 2.0)
+    c.begin()
+    monkeypatch.setattr(bench.time, "time", lambda: 3.0)
+    c.end()
+    c.samples.append((9.0, line.format(sm=300, cap="Not Active")))  # after: dropped
+    rec = c.stop()
+    assert rec["samples"] == 2
+    assert rec["sm_mhz"] == (1965 + 1900) / 2 and rec["sm_max_mhz"] == 1965
+    assert rec["reasons"] == ["sw_power_cap"]
+    assert bench.ClockSampler(0, enabled=False).stop() is None

@@ -70,7 +70,7 @@ def _close(out, ref):
 @pytest.mark.parametrize("name", ["tiny", "qwen3", "llama32", "longskew", "prefix"])
 def test_fp8_append_and_decode_match_oracle(pa, oracle_lib, name):
     from paged_kv_attention_36_b200 import workloads
-    w = workloads.make(name, poison=name in ("tiny", "qwen3", "prefix"))
+    w = workloads.make(name, poison=True)
     ks, vs = _scales(w.k_cache.shape[1])
     k8, v8, gk8, gv8, tks, tvs = _quantize_both(pa, oracle_lib, w.k_cache, w.v_cache, ks, vs)
     ref = oracle_lib.decode_fp8(paging.bits(w.q), k8, v8, ks, vs, w.block_tables.numpy(),
@@ -80,6 +80,52 @@ def test_fp8_append_and_decode_match_oracle(pa, oracle_lib, name):
     out = torch.full_like(q, float("nan"))
     pa.pa_decode_fp8(q, gk8, gv8, tks, tvs, w.block_tables.to(d), w.context_lens.to(d), w.scale, out)
     torch.cuda.synchronize()
+    _close(out, ref)
+    assert pa.pa_device_errors(clear=True) == 0
+
+
+@pytest.mark.parametrize("name", ["tiny", "qwen3", "llama32", "longskew", "prefix"])
+def test_fp8_fused_append_decode_matches_oracle(pa, oracle_lib, name):
+    # one launch (pa_append_decode_fp8): every CTA encodes a slice of the
+    # step's new rows, then the decode reads the caches including them
+    from paged_kv_attention_36_b200 import workloads
+    w = workloads.make(name, poison=True)
+    ks, vs = _scales(w.k_cache.shape[1])
+    k8, v8, gk8, gv8, tks, tvs = _quantize_both(pa, oracle_lib, w.k_cache, w.v_cache, ks, vs)
+    oracle_lib.append_fp8(paging.bits(w.k_new), paging.bits(w.v_new), w.slot_mapping.numpy(), k8, v8, ks, vs)
+    ref = oracle_lib.decode_fp8(paging.bits(w.q), k8, v8, ks, vs, w.block_tables.numpy(),
+                                w.context_lens.numpy(), w.scale)
+    d = torch.device("cuda")
+    q = w.q.to(d)
+    out = torch.full_like(q, float("nan"))
+    pa.pa_append_decode_fp8(w.k_new.to(d), w.v_new.to(d), w.slot_mapping.to(d), q, gk8, gv8, tks, tvs,
+                            w.block_tables.to(d), w.context_lens.to(d), w.scale, out)
+    torch.cuda.synchronize()
+    assert np.array_equal(gk8.cpu().numpy(), k8), "k codes differ from the oracle append"
+    assert np.array_equal(gv8.cpu().numpy(), v8), "v codes differ from the oracle append"
+    _close(out, ref)
+    assert pa.pa_device_errors(clear=True) == 0
+
+
+def test_fp8_fused_reads_rows_written_by_other_ctas(pa, oracle_lib):
+    # every new row goes to another sequence's last page (reversed slot
+    # mapping), so the CTA that reads it is not the one that wrote it
+    from paged_kv_attention_36_b200 import workloads
+    w = workloads.make("llama32", poison=True)
+    perm = torch.arange(w.q.shape[0] - 1, -1, -1)
+    kn, vn, sm = w.k_new[perm].contiguous(), w.v_new[perm].contiguous(), w.slot_mapping[perm].contiguous()
+    ks, vs = _scales(w.k_cache.shape[1])
+    k8, v8, gk8, gv8, tks, tvs = _quantize_both(pa, oracle_lib, w.k_cache, w.v_cache, ks, vs)
+    oracle_lib.append_fp8(paging.bits(kn), paging.bits(vn), sm.numpy(), k8, v8, ks, vs)
+    ref = oracle_lib.decode_fp8(paging.bits(w.q), k8, v8, ks, vs, w.block_tables.numpy(),
+                                w.context_lens.numpy(), w.scale)
+    d = torch.device("cuda")
+    q = w.q.to(d)
+    out = torch.full_like(q, float("nan"))
+    pa.pa_append_decode_fp8(kn.to(d), vn.to(d), sm.to(d), q, gk8, gv8, tks, tvs, w.block_tables.to(d),
+                            w.context_lens.to(d), w.scale, out)
+    torch.cuda.synchronize()
+    assert np.array_equal(gk8.cpu().numpy(), k8) and np.array_equal(gv8.cpu().numpy(), v8)
     _close(out, ref)
     assert pa.pa_device_errors(clear=True) == 0
 

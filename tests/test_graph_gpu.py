@@ -6,8 +6,9 @@ Every C-ABI call is asynchronous, allocates nothing and never synchronises,
 so a whole step can be captured on a torch stream and replayed.  These
 tests capture (1) the fused append + decode (a cooperative launch with a
 grid barrier in the workspace), (2) the shared-prefix step (the prefix pass
-and the decode launched as its programmatic dependent) and (3) the two-call
-step (append, then decode), and (4) the multi-query prefill; they replay
+and the decode launched as its programmatic dependent), (3) the two-call
+step (append, then decode), (4) the fused fp8 append + decode and (5) the
+multi-query prefill; they replay
 each several times with new inputs written into the captured buffers and
 compare every replay with the fp64 oracle.  Replays reuse the workspace,
 so they also prove that every call leaves its counters and barrier at zero.
@@ -90,7 +91,7 @@ def test_graph_fused_append_decode(pa, oracle_lib):
 
 def test_graph_two_call_step(pa, oracle_lib):
     from paged_kv_attention_36_b200 import workloads
-    w = workloads.make("longskew")
+    w = workloads.make("longskew", poison=True)
 
     def step(t, out):
         dims = pa.make_dims(t["q"], t["k_cache"], t["block_tables"])
@@ -116,6 +117,61 @@ def test_graph_shared_prefix_step(pa, oracle_lib):
                                    k_new=t["k_new"], v_new=t["v_new"], slot_mapping=t["slot_mapping"],
                                    workspace=step.ws)
     _run(pa, oracle_lib, w, step)
+
+
+def test_graph_fused_fp8_step(pa, oracle_lib):
+    """The fused fp8 step (pa_append_decode_fp8) captured once and replayed
+    with new q and new rows; each replay against the oracle's fp8 append and
+    decode of the same rows."""
+    from paged_kv_attention_36_b200 import workloads
+    w = workloads.make("llama32", poison=True)
+    NB, Hkv, bs, D = w.k_cache.shape
+    gsc = np.arange(Hkv, dtype=np.float32)
+    ks, vs = (gsc + 4) / 32, (gsc + 3) / 24
+    rows_k = w.k_cache.permute(0, 2, 1, 3).reshape(NB * bs, Hkv, D).contiguous()
+    rows_v = w.v_cache.permute(0, 2, 1, 3).reshape(NB * bs, Hkv, D).contiguous()
+    slots = torch.arange(NB * bs, dtype=torch.int32)
+    k8 = np.zeros((NB, Hkv, 16, D), np.uint8)
+    v8 = np.zeros((NB, Hkv, D, 16), np.uint8)
+    oracle_lib.append_fp8(paging.bits(rows_k), paging.bits(rows_v), slots.numpy(), k8, v8, ks, vs)
+    d = torch.device("cuda")
+    t = {"q": w.q.to(d), "kn": w.k_new.to(d), "vn": w.v_new.to(d), "sm": w.slot_mapping.to(d),
+         "k8": torch.from_numpy(k8).to(d), "v8": torch.from_numpy(v8).to(d), "ks": torch.from_numpy(ks).to(d),
+         "vs": torch.from_numpy(vs).to(d), "bt": w.block_tables.to(d), "cl": w.context_lens.to(d)}
+    out = torch.empty_like(t["q"])
+    dims = pa.pa_dims(w.q.shape[0], w.q.shape[1], Hkv, D, 16, NB, w.block_tables.shape[1])
+    ws = pa.alloc_workspace(dims)
+
+    def step():
+        pa.pa_append_decode_fp8(t["kn"], t["vn"], t["sm"], t["q"], t["k8"], t["v8"], t["ks"], t["vs"], t["bt"],
+                                t["cl"], w.scale, out, workspace=ws)
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        step()  # warm-up outside capture
+    torch.cuda.current_stream().wait_stream(stream)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    gen = torch.Generator().manual_seed(78)
+    for _ in range(3):
+        q = torch.randn(w.q.shape, generator=gen).to(torch.bfloat16)
+        kn = torch.randn(w.k_new.shape, generator=gen).to(torch.bfloat16)
+        vn = torch.randn(w.v_new.shape, generator=gen).to(torch.bfloat16)
+        t["q"].copy_(q)
+        t["kn"].copy_(kn)
+        t["vn"].copy_(vn)
+        out.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        rk, rv = k8.copy(), v8.copy()
+        oracle_lib.append_fp8(paging.bits(kn), paging.bits(vn), w.slot_mapping.numpy(), rk, rv, ks, vs)
+        assert np.array_equal(t["k8"].cpu().numpy(), rk) and np.array_equal(t["v8"].cpu().numpy(), rv)
+        ref = oracle_lib.decode_fp8(paging.bits(q), rk, rv, ks, vs, w.block_tables.numpy(), w.context_lens.numpy(),
+                                    w.scale)
+        _close(out, ref)
+    assert pa.pa_device_errors(clear=True) == 0
 
 
 def test_graph_prefill(pa, oracle_lib):

@@ -6,7 +6,10 @@ environment at its first call (so each needs a process of its own):
   * PA_PREFILL_MMA=sync — the warp-level mma.sync prefill and prefix pass;
   * PA_PREFIX_SPLITS=1 / 16 — the fewest and the most key ranges of the
                          shared-prefix pass (the decode folds one or sixteen
-                         range partials per member).
+                         range partials per member);
+  * PA_DECODE_MATH=simt — the decode's per-page math in fp32 on the CUDA
+                         cores instead of mma.sync (head_dim * Hq/Hkv <= 256;
+                         the suites skip the shapes it is not built for).
 
 Each runs the parity suites it affects against the oracle in a child pytest
 process with the variable set.
@@ -21,7 +24,7 @@ import torch
 pytestmark = pytest.mark.gpu
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-_VARS = ("PA_PREFILL_BN", "PA_PREFILL_MMA", "PA_PREFIX_SPLITS")
+_VARS = ("PA_PREFILL_BN", "PA_PREFILL_MMA", "PA_PREFIX_SPLITS", "PA_DECODE_MATH")
 
 
 @pytest.mark.parametrize("var,value,suites", [
@@ -29,6 +32,7 @@ _VARS = ("PA_PREFILL_BN", "PA_PREFILL_MMA", "PA_PREFIX_SPLITS")
     ("PA_PREFILL_MMA", "sync", ("test_prefill_gpu.py", "test_prefix_gpu.py")),
     ("PA_PREFIX_SPLITS", "1", ("test_prefix_gpu.py",)),
     ("PA_PREFIX_SPLITS", "16", ("test_prefix_gpu.py",)),
+    ("PA_DECODE_MATH", "simt", ("test_parity_gpu.py", "test_prefix_gpu.py")),
 ])
 def test_configuration_matches_oracle(var, value, suites):
     if not torch.cuda.is_available():

@@ -178,3 +178,13 @@ def test_shared_prefix_host_validation(binding):
     assert call(d, q=0) == -1
     assert call(d, out=8) == -4
     assert call(_dims(binding, num_seqs=0)) == 0                  # nothing to attend over, nothing to append
+
+
+def test_binding_constants_match_the_header(binding):
+    # the ctypes binding restates the header's #define values; they must agree
+    src = open(os.path.join(ROOT, "include", "pa.h")).read()
+    defs = dict(re.findall(r"#define\s+(PA_(?:DEVERR_\w+|STATIC_SCRATCH_BYTES))\s+(\S.*?)\s*(?:/\*|$)", src,
+                           re.M))
+    assert "PA_STATIC_SCRATCH_BYTES" in defs and "PA_DEVERR_TIMEOUT" in defs
+    for name, val in defs.items():
+        assert getattr(binding, name) == eval(val.replace("u", "")), name

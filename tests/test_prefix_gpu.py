@@ -13,6 +13,8 @@ breaches that fall back to a plain decode of the member (a context shorter
 than the prefix, a group larger than max_group_size) or are only reported
 (a member whose table does not hold the prefix blocks).
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -22,6 +24,10 @@ from tests import paging
 pytestmark = pytest.mark.gpu
 
 ATOL, RTOL = 1e-2, 1e-2
+
+# PA_DECODE_MATH=simt (set for a child process by test_kernel_variants_gpu.py)
+# selects the fp32 CUDA-core decode policy, built for head_dim * Hq/Hkv <= 256.
+SIMT = os.environ.get("PA_DECODE_MATH") == "simt"
 
 
 @pytest.fixture(scope="module")
@@ -111,6 +117,8 @@ def test_group_shapes(pa, oracle_lib, heads):
     # groups of 5 (ragged suffixes), 1, 17 (crosses a 128-row tile at G = 8),
     # a group sharing nothing, ungrouped tails including an empty context
     from paged_kv_attention_36_b200 import workloads
+    if SIMT and (heads[0] // heads[1]) * heads[2] > 256:
+        pytest.skip("the fp32 CUDA-core policy is built for head_dim * Hq/Hkv <= 256")
     g = torch.Generator().manual_seed(sum(heads))
     groups = [(5, 6), (1, 3), (17, 2), (3, 0)]
     n = sum(m for m, _ in groups)
@@ -145,7 +153,7 @@ def test_long_member_split_over_ctas(pa, oracle_lib):
     # a member with 40000 own tokens is split over many CTAs: only the piece
     # that starts at its first own page may carry the prefix
     from paged_kv_attention_36_b200 import workloads
-    w = workloads.make_grouped("qwen3", [(3, 40)], [40000, 9, 300], tail_lens=[5000])
+    w = workloads.make_grouped("qwen3", [(3, 40)], [40000, 9, 300], tail_lens=[5000], poison=True)
     ref = _ref(oracle_lib, w)
     _assert_close(_decode(pa, _dev(w), w), ref)
     assert pa.pa_device_errors(clear=True) == 0
@@ -153,7 +161,7 @@ def test_long_member_split_over_ctas(pa, oracle_lib):
 
 def test_context_shorter_than_prefix_falls_back(pa, oracle_lib):
     from paged_kv_attention_36_b200 import workloads
-    w = workloads.make_grouped("qwen3", [(4, 6)], [10, 20, 30, 40])
+    w = workloads.make_grouped("qwen3", [(4, 6)], [10, 20, 30, 40], poison=True)
     w.context_lens[2] = 6 * 16 - 5    # inside the shared blocks: decoded over its own table
     ref = _ref(oracle_lib, w)
     _assert_close(_decode(pa, _dev(w), w), ref)
@@ -162,7 +170,7 @@ def test_context_shorter_than_prefix_falls_back(pa, oracle_lib):
 
 def test_group_larger_than_max_group_size_falls_back(pa, oracle_lib):
     from paged_kv_attention_36_b200 import workloads
-    w = workloads.make_grouped("qwen3", [(6, 4), (2, 3)], [5, 6, 7, 8, 9, 10, 11, 12])
+    w = workloads.make_grouped("qwen3", [(6, 4), (2, 3)], [5, 6, 7, 8, 9, 10, 11, 12], poison=True)
     ref = _ref(oracle_lib, w)
     _assert_close(_decode(pa, _dev(w), w, max_group_size=4), ref)
     assert pa.pa_device_errors(clear=True) & pa.PA_DEVERR_PREFIX
