@@ -42,7 +42,7 @@ template <int D, int EB = 2>
 constexpr int ring_fit() {
     using C1 = pa::DecodeCfg<D, kBlockSize, 1, EB>;
     int r = PA_MAX_RING;
-    while (r > 1 && C1::kSmemBytes + (r - 1) * (C1::kStage + 16) > 232448) --r;
+    while (r > 1 && C1::kBaseBytes + (r - 1) * (C1::kStage + 16) > 232448) --r;
     r -= r % C1::kMaxSpl;
     return r;
 }
@@ -235,12 +235,14 @@ pa_status launch_decode(const pa::DecodeParams& p, int grid, cudaStream_t stream
     }();
     static unsigned attr_done[kMaxDevices];
     if (!set_smem_once(kern, Cfg::kSmemBytes, attr_done)) return PA_ERR_CUDA;
-    if (APPEND) {
+    // the rest of shared memory is needed only to stage prefix partials
+    const int smem = p.num_groups > 0 ? Cfg::kSmemBytes : Cfg::kBaseBytes;
+    if (APPEND && !p.app_local) {
         // the CTAs meet at a grid barrier: a cooperative launch guarantees they are all resident
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(grid);
         cfg.blockDim = dim3(Cfg::kThreads);
-        cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+        cfg.dynamicSmemBytes = smem;
         cfg.stream = stream;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeCooperative;
@@ -252,7 +254,7 @@ pa_status launch_decode(const pa::DecodeParams& p, int grid, cudaStream_t stream
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(grid);
         cfg.blockDim = dim3(Cfg::kThreads);
-        cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+        cfg.dynamicSmemBytes = smem;
         cfg.stream = stream;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -261,7 +263,7 @@ pa_status launch_decode(const pa::DecodeParams& p, int grid, cudaStream_t stream
         cfg.numAttrs = 1;
         if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return PA_ERR_CUDA;
     } else {
-        kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(p);
+        kern<<<grid, Cfg::kThreads, smem, stream>>>(p);
     }
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
@@ -704,6 +706,7 @@ pa_status pa_append_decode(const void* k_new, const void* v_new, const int32_t* 
     p.slot_mapping = slot_mapping;
     p.app_chunks = int64_t(num_tokens) * dims->num_kv_heads * (dims->head_dim / 8);
     p.app_tokens = num_tokens;
+    p.app_local = num_tokens <= pa::kLocalMaxTokens;
     p.k_cache_w = static_cast<uint4*>(k_cache);
     p.v_cache_w = static_cast<uint4*>(v_cache);
     return dispatch_decode<false, true>(dims->head_dim, dims->num_q_heads / dims->num_kv_heads, p, grid,
@@ -779,11 +782,16 @@ pa_status pa_decode_shared_prefix(const void* k_new, const void* v_new, const in
         pp.qscale = p.qscale;
         pp.prefix_o = reinterpret_cast<float*>(ws + w.o);
         pp.prefix_ml = reinterpret_cast<float2*>(ws + w.ml);
-        // the append rides on the prefix launch; the decode follows it
+        // Up to kLocalMaxTokens new rows are appended by the decode itself
+        // (each CTA writes the rows of the blocks it reads), so the decode
+        // streams its pages while the prefix pass runs and waits for the pass
+        // only before reading its partials; more rows ride on the prefix
+        // launch and the decode waits for the pass before reading anything.
+        const bool local = num_tokens <= pa::kLocalMaxTokens;
         pp.k_new = static_cast<const uint4*>(k_new);
         pp.v_new = static_cast<const uint4*>(v_new);
         pp.slot_mapping = slot_mapping;
-        pp.app_chunks = int64_t(num_tokens) * d.num_kv_heads * (d.head_dim / 8);
+        pp.app_chunks = local ? 0 : int64_t(num_tokens) * d.num_kv_heads * (d.head_dim / 8);
         pp.k_cache_w = static_cast<uint4*>(k_cache);
         pp.v_cache_w = static_cast<uint4*>(v_cache);
         const pa_status ps = dispatch_prefix(d.head_dim, G, pp, dim3(unsigned(num_groups * tiles),
@@ -796,7 +804,17 @@ pa_status pa_decode_shared_prefix(const void* k_new, const void* v_new, const in
         p.prefix_splits = splits;
         p.prefix_o = pp.prefix_o;
         p.prefix_ml = pp.prefix_ml;
-        return dispatch_decode<false>(d.head_dim, G, p, grid, s, /*pdl=*/true);
+        p.defer_dep = local ? 1 : 0;
+        if (!local || num_tokens == 0) return dispatch_decode<false>(d.head_dim, G, p, grid, s, /*pdl=*/true);
+        p.k_new = static_cast<const uint4*>(k_new);
+        p.v_new = static_cast<const uint4*>(v_new);
+        p.slot_mapping = slot_mapping;
+        p.app_chunks = int64_t(num_tokens) * d.num_kv_heads * (d.head_dim / 8);
+        p.app_tokens = num_tokens;
+        p.app_local = 1;
+        p.k_cache_w = static_cast<uint4*>(k_cache);
+        p.v_cache_w = static_cast<uint4*>(v_cache);
+        return dispatch_decode<false, true>(d.head_dim, G, p, grid, s, /*pdl=*/true);
     }
     if (num_tokens == 0) return dispatch_decode<false>(d.head_dim, G, p, grid, s);
     p.k_new = static_cast<const uint4*>(k_new);
@@ -804,6 +822,7 @@ pa_status pa_decode_shared_prefix(const void* k_new, const void* v_new, const in
     p.slot_mapping = slot_mapping;
     p.app_chunks = int64_t(num_tokens) * d.num_kv_heads * (d.head_dim / 8);
     p.app_tokens = num_tokens;
+    p.app_local = num_tokens <= pa::kLocalMaxTokens;
     p.k_cache_w = static_cast<uint4*>(k_cache);
     p.v_cache_w = static_cast<uint4*>(v_cache);
     return dispatch_decode<false, true>(d.head_dim, G, p, grid, s);
@@ -909,6 +928,7 @@ pa_status pa_append_decode_fp8(const void* k_new, const void* v_new, const int32
     p.slot_mapping = slot_mapping;
     p.app_chunks = int64_t(num_tokens) * dims->num_kv_heads * (dims->head_dim / 8);
     p.app_tokens = num_tokens;
+    p.app_local = num_tokens <= pa::kLocalMaxTokens;
     p.k_cache_w = static_cast<uint4*>(k_cache);
     p.v_cache_w = static_cast<uint4*>(v_cache);
     return dispatch_d_g<MathKind::kFp8, false, true>(dims->head_dim, dims->num_q_heads / dims->num_kv_heads, p, grid,

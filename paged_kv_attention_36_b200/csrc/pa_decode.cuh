@@ -102,6 +102,8 @@ struct DecodeParams {
     const int32_t* slot_mapping;  // [T]
     int64_t app_chunks;           // T * Hkv * D / 8
     int32_t app_tokens;           // T
+    int32_t app_local;            // 1: readers write the rows of the blocks they read (T <= kLocalMaxTokens),
+                                  // 0: a grid barrier (a cooperative launch)
     uint4* k_cache_w;             // the caches, writable
     uint4* v_cache_w;
     unsigned int* grid_bar;       // {arrivals, departures}: zero between calls
@@ -111,6 +113,9 @@ struct DecodeParams {
     const int32_t* group_prefix_pages;  // [num_groups]
     int32_t num_groups, max_group_size;
     int32_t prefix_splits;              // key ranges of the prefix partials
+    int32_t defer_dep;                  // 1: the decode owns the step's append, so it waits for the
+                                        // prefix pass (griddepcontrol.wait) only before reading its
+                                        // partials; 0: before reading anything (the pass appended)
     const float* prefix_o;              // [splits][B][Hq][D]
     const float2* prefix_ml;            // [splits][B][Hq] (max logit base 2, exp-sum)
     // fp8 caches: value = e4m3 code * scale[kv head] (null for bf16 caches)
@@ -150,6 +155,17 @@ struct Misc {
 };
 static_assert(sizeof(Misc) <= 256, "misc area");
 
+
+// A finished partial is read from global memory (written by other CTAs or
+// by the shared-prefix pass: L2, not L1) or from this warp's shared-memory
+// staging.
+template <bool SMEM, class T>
+__device__ __forceinline__ T ld_part(const T* p) {
+    if constexpr (SMEM)
+        return *p;
+    else
+        return __ldcg(p);
+}
 
 // ===========================================================================
 // SIMT math policy.
@@ -297,11 +313,12 @@ struct SimtMath {
     // Folds a finished partial (normalised output o[G][D], (max logit base
     // 2, exp-sum) per head) into the state, as if its tokens had been paged
     // here.  The sums live in token group 0; every lane keeps the same m.
+    template <bool SMEM = false>
     __device__ __forceinline__ void absorb(const float* o, const float2* ml, int lane) {
         const int tg = lane >> 3, c = lane & 7;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-            const float2 pml = __ldcg(ml + h);
+            const float2 pml = ld_part<SMEM>(ml + h);
             const float M = fmaxf(m[h], pml.x);
             const float a_old = exp2f(m[h] - M), a_new = pml.y * exp2f(pml.x - M);
             m[h] = M;
@@ -311,7 +328,7 @@ struct SimtMath {
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     float2 v = make_float2(0.f, 0.f);
-                    if (tg == 0) v = __ldcg(reinterpret_cast<const float2*>(o + h * D + (c + 8 * i) * 8 + 2 * j));
+                    if (tg == 0) v = ld_part<SMEM>(reinterpret_cast<const float2*>(o + h * D + (c + 8 * i) * 8 + 2 * j));
                     acc[h][i][j] = make_float2(acc[h][i][j].x * a_old + a_new * v.x,
                                                acc[h][i][j].y * a_old + a_new * v.y);
                 }
@@ -540,16 +557,17 @@ struct MmaMath {
         float o[KS][4];
         float2 ml[2];
     };
+    template <bool SMEM = false>
     __device__ __forceinline__ void piece_load(Piece& pc, const float* o, const float2* ml, int lane) const {
         const int h0 = (lane & 3) * 2, d0 = lane >> 2;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const int h = h0 + e < G ? h0 + e : 0;  // heads past G: loaded, never folded
-            pc.ml[e] = __ldcg(ml + h);
+            pc.ml[e] = ld_part<SMEM>(ml + h);
 #pragma unroll
             for (int mt = 0; mt < KS; ++mt) {
-                pc.o[mt][e] = __ldcg(o + h * D + 16 * mt + d0);
-                pc.o[mt][2 + e] = __ldcg(o + h * D + 16 * mt + d0 + 8);
+                pc.o[mt][e] = ld_part<SMEM>(o + h * D + 16 * mt + d0);
+                pc.o[mt][2 + e] = ld_part<SMEM>(o + h * D + 16 * mt + d0 + 8);
             }
         }
     }
@@ -571,9 +589,10 @@ struct MmaMath {
             }
         }
     }
+    template <bool SMEM = false>
     __device__ __forceinline__ void absorb(const float* o, const float2* ml, int lane) {
         Piece pc;
-        piece_load(pc, o, ml, lane);
+        piece_load<SMEM>(pc, o, ml, lane);
         piece_absorb(pc, lane);
     }
 
@@ -895,11 +914,17 @@ struct DecodeCfg {
     static constexpr int kNumBars = 2 * R + 2 * kSegSlots;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kMiscBytes = 256;
-    // fused append: a bitmap of the blocks the step's append writes, hashed
-    // by block id (bit blk % kDirtyBits)
+    // The rest of shared memory (at least 1 KB) is one area: the fused
+    // append's bitmap of the blocks it writes (hashed by block id; kDirtyBytes,
+    // or the first half of it in a shared-prefix decode) and, in a
+    // shared-prefix decode, from byte kDirtyBytes / 2 on, per-warp staging of
+    // the prefix range partials.
     static constexpr int kDirtyOff = kMiscOff + kMiscBytes;
     static constexpr int kDirtyBytes = 1024;
-    static constexpr int kSmemBytes = kDirtyOff + kDirtyBytes + 1024;  // + alignment slack
+    static constexpr int kBaseBytes = kDirtyOff + kDirtyBytes + 1024;  // with the smallest area; + alignment slack
+    static constexpr int kAreaBytes = ((232448 - kDirtyOff - 1024) / (NW * 16)) * (NW * 16);
+    static constexpr int kSmemBytes = kDirtyOff + kAreaBytes + 1024;
+    static_assert(kAreaBytes >= kDirtyBytes, "the area holds the bitmap");
     static_assert(kTile % 1024 == 0 && kStage % 1024 == 0, "TMA tile alignment (128-byte swizzle)");
     static_assert(kBarOff % 8 == 0, "mbarrier alignment");
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
@@ -1096,16 +1121,26 @@ __device__ __noinline__ void merge_pieces(const DecodeParams& p, int k0, int off
     }
 }
 
-// Fused append.  Every CTA writes a slice of the step's new rows and
-// arrives at a grid barrier (grid_bar[0] counts arrivals).  A CTA must not
-// read a block those rows go to before every CTA has arrived, but most pages
-// are not written this step: each CTA marks the written blocks in a hashed
-// bitmap, and its producer waits at the barrier only before the first page
-// whose block is marked (a hash collision only makes it wait earlier).
+// Fused append.  Every CTA writes a slice of the step's new rows, so that
+// every row lands, and marks the blocks the rows go to in a hashed bitmap.
+// A CTA must not read a marked block before the rows that go to it are
+// there.  Two ways:
+//   * local (T <= kLocalMaxTokens, the decode step's one token per
+//     sequence): before loading a marked block, the producer finds the
+//     tokens whose slots lie in it and writes their rows of its head group
+//     itself (the same bytes the slice owner writes, so the duplicate
+//     writes are harmless); no CTA waits for another, and the launch needs
+//     no co-residency;
+//   * barrier (more tokens): the CTAs arrive at a grid barrier (grid_bar[0]
+//     counts arrivals; a cooperative launch) and a producer waits there
+//     before its first marked block (a hash collision only makes it wait
+//     earlier).
 constexpr int kDirtyMaxTokens = 2048;  // more appended tokens: every page counts as written
+constexpr int kLocalMaxTokens = 256;   // the producer warp keeps the step's slots in registers
 
+// words * 32 is a power of two
 __device__ __forceinline__ bool block_marked(const uint32_t* map, int words, int32_t blk) {
-    const uint32_t bit = uint32_t(blk) % uint32_t(words * 32);
+    const uint32_t bit = uint32_t(blk) & uint32_t(words * 32 - 1);
     return (map[bit >> 5] >> (bit & 31)) & 1u;
 }
 
@@ -1144,6 +1179,68 @@ __device__ __forceinline__ void depart_grid(const DecodeParams& p) {
     }
 }
 
+// Sequences whose whole context is their group's shared prefix take no
+// units: their output is the merge of the prefix partials alone.  The
+// calling threads (tid of nthreads) share CTA blockIdx.x's such sequences;
+// they must have waited for the prefix pass.
+template <int D>
+__device__ __forceinline__ void prefix_only_outputs(const DecodeParams& p, int tid, int nthreads) {
+    for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
+        const SeqPages sp = seq_pages<16>(p, b, false);
+        if (sp.P == 0 || sp.np != 0) continue;
+        const int per = prefix_split_pages(sp.P, p.prefix_splits);
+        const int nz = (sp.P + per - 1) / per;
+        for (int o = tid; o < p.Hq * D; o += nthreads) {
+            const int h = o / D;
+            float M = -INFINITY;
+            for (int z = 0; z < nz; ++z) M = fmaxf(M, __ldcg(&p.prefix_ml[(int64_t(z) * p.B + b) * p.Hq + h]).x);
+            float lsum = 0.f, a = 0.f;
+            for (int z = 0; z < nz; ++z) {
+                const int64_t idx = (int64_t(z) * p.B + b) * p.Hq + h;
+                const float2 ml = __ldcg(&p.prefix_ml[idx]);
+                const float w = ml.y * exp2f(ml.x - M);
+                lsum += w;
+                a += w * __ldcg(&p.prefix_o[idx * D + (o - h * D)]);
+            }
+            p.out[int64_t(b) * p.Hq * D + o] = __float2bfloat16_rn(a / lsum);
+        }
+    }
+}
+
+// Local fused append: the calling warp writes the rows of every appended
+// token whose slot lies in block bk, for the kv heads g0 .. g0+ng-1, into
+// the cache (a bit copy, or the E4M3 encoding for fp8 caches), in token
+// order.  slots: lane l holds the slots of tokens l, l+32, ...
+template <int D, int BS, int EB>
+__device__ __forceinline__ void write_block_rows(const DecodeParams& p, const int32_t (&slots)[kLocalMaxTokens / 32],
+                                                 int32_t bk, int g0, int ng, int lane) {
+    constexpr int CPR = D / 8;  // 16-byte chunks of bf16 per row
+#pragma unroll
+    for (int k = 0; k < kLocalMaxTokens / 32; ++k) {
+        if (32 * k >= p.app_tokens) break;
+        unsigned hit = __ballot_sync(0xffffffffu, slots[k] >= 0 && slots[k] / BS == bk);
+        while (hit) {
+            const int tl = __ffs(hit) - 1;
+            hit &= hit - 1;
+            const int64_t t = 32 * k + tl;
+            const int32_t off = __shfl_sync(0xffffffffu, slots[k], tl) - bk * BS;
+            for (int c = lane; c < ng * CPR; c += 32) {
+                const int g = g0 + c / CPR, ch = c % CPR;
+                const int64_t src = (t * p.Hkv + g) * CPR + ch;
+                if constexpr (EB == 1) {
+                    append_fp8_chunk(p.k_new, p.v_new, p.slot_mapping, reinterpret_cast<uint8_t*>(p.k_cache_w),
+                                     reinterpret_cast<uint8_t*>(p.v_cache_w), p.k_scale, p.v_scale, p.Hkv, CPR, p.NB,
+                                     src);
+                } else {
+                    const int64_t dst = ((int64_t(bk) * p.Hkv + g) * BS + off) * CPR + ch;
+                    p.k_cache_w[dst] = __ldg(p.k_new + src);
+                    p.v_cache_w[dst] = __ldg(p.v_new + src);
+                }
+            }
+        }
+    }
+}
+
 template <int D, int G, int BS, int R, bool DUMP, bool APPEND, template <int, int, int> class Math>
 __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
     using Cfg = DecodeCfg<D, BS, R, Math<D, G, BS>::kElemBytes>;
@@ -1163,7 +1260,8 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
     Misc* misc = reinterpret_cast<Misc*>(smem + Cfg::kMiscOff);
     volatile int* abort = &misc->abort;
     uint32_t* dirty_map = reinterpret_cast<uint32_t*>(smem + Cfg::kDirtyOff);
-    constexpr int kDirtyWords = Cfg::kDirtyBytes / 4;
+    // a shared-prefix decode keeps half the bitmap: the rest of the area stages partials
+    const int kDirtyWords = (p.num_groups > 0 ? Cfg::kDirtyBytes / 2 : Cfg::kDirtyBytes) / 4;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int HG = p.HG, HS = p.HS, SPL = p.SPL;
@@ -1190,7 +1288,7 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
             for (int t = threadIdx.x; t < p.app_tokens; t += NT) {
                 const int32_t slot = __ldg(p.slot_mapping + t);
                 if (slot < 0) continue;
-                const uint32_t bit = uint32_t(slot / BS) % uint32_t(kDirtyWords * 32);
+                const uint32_t bit = uint32_t(slot / BS) & uint32_t(kDirtyWords * 32 - 1);
                 atomicOr(&dirty_map[bit >> 5], 1u << (bit & 31));
             }
         }
@@ -1223,10 +1321,12 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
             p.k_cache_w[dst] = __ldg(p.k_new + idx);
             p.v_cache_w[dst] = __ldg(p.v_new + idx);
         }
-        fence_proxy_async_global();
-        __threadfence();
-        __syncthreads();
-        if (threadIdx.x == 0) atomicAdd(&p.grid_bar[0], 1u);
+        if (!p.app_local) {  // barrier: arrive once the slice is visible to every CTA's TMA loads
+            fence_proxy_async_global();
+            __threadfence();
+            __syncthreads();
+            if (threadIdx.x == 0) atomicAdd(&p.grid_bar[0], 1u);
+        }
     }
 
     // ---- the CTA's share: a scan of v_b = NG * (pages(b) + seg_weight) over
@@ -1255,35 +1355,15 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
     // launch) has done the set-up above meanwhile; the prefix partials and
     // the rows that kernel appended are read only after this wait (a no-op
     // for an ordinary launch).
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (p.num_groups > 0) {
-        // Sequences whose whole context is their group's shared prefix take no
-        // units: their output is the merge of the prefix partials alone.
-        for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
-            const SeqPages sp = seq_pages<BS>(p, b, false);
-            if (sp.P == 0 || sp.np != 0) continue;
-            const int per = prefix_split_pages(sp.P, p.prefix_splits);
-            const int nz = (sp.P + per - 1) / per;
-            for (int o = threadIdx.x; o < p.Hq * D; o += NT) {
-                const int h = o / D;
-                float M = -INFINITY;
-                for (int z = 0; z < nz; ++z) M = fmaxf(M, __ldcg(&p.prefix_ml[(int64_t(z) * p.B + b) * p.Hq + h]).x);
-                float lsum = 0.f, a = 0.f;
-                for (int z = 0; z < nz; ++z) {
-                    const int64_t idx = (int64_t(z) * p.B + b) * p.Hq + h;
-                    const float2 ml = __ldcg(&p.prefix_ml[idx]);
-                    const float w = ml.y * exp2f(ml.x - M);
-                    lsum += w;
-                    a += w * __ldcg(&p.prefix_o[idx * D + (o - h * D)]);
-                }
-                p.out[int64_t(b) * p.Hq * D + o] = __float2bfloat16_rn(a / lsum);
-            }
-        }
-    }
+    if (!p.defer_dep) asm volatile("griddepcontrol.wait;" ::: "memory");
     const int64_t want = (Wt + p.min_pages - 1) / p.min_pages;
     const int64_t grid_eff = want < int64_t(gridDim.x) ? want : int64_t(gridDim.x);
     if (Wt == 0 || int64_t(blockIdx.x) >= grid_eff) {  // no share: read no page
-        if (APPEND && threadIdx.x == 0) depart_grid(p);
+        if (APPEND && !p.app_local && threadIdx.x == 0) depart_grid(p);
+        if (p.num_groups > 0) {
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            prefix_only_outputs<D>(p, threadIdx.x, NT);
+        }
         return;
     }
     const Split split{Wt / grid_eff, Wt % grid_eff};
@@ -1326,7 +1406,15 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
         uint32_t stage_i = 0, seg_i = 0;
         constexpr int C = R < 32 ? R : 32;
         bool ok = true;
-        bool rows_ready = !APPEND;  // fused append: every CTA's rows are visible
+        bool rows_ready = !APPEND;  // fused append, barrier: every CTA's rows are visible
+        // fused append, local: the step's slots, lane l holding tokens l, l+32, ...
+        constexpr int kSlotRegs = kLocalMaxTokens / 32;
+        int32_t my_slots[kSlotRegs];
+#pragma unroll
+        for (int k = 0; k < kSlotRegs; ++k) {
+            const int t = 32 * k + lane;
+            my_slots[k] = (APPEND && p.app_local && t < p.app_tokens) ? __ldg(p.slot_mapping + t) : -1;
+        }
         const uint64_t pol = PA_EVICT_FIRST ? policy_evict_first() : policy_evict_normal();
         const uint32_t stage_tx = uint32_t(2 * HS * Cfg::kTile);
 
@@ -1375,7 +1463,25 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
                             blk = 0;
                         }
                     }
-                    if (APPEND && !rows_ready) {
+                    if (APPEND && p.app_local) {
+                        // the new rows of each marked page of the batch (its first
+                        // stage's lane stands for it), this head group's heads
+                        const bool marked = lane < n && ((c0 + lane) & (SPL - 1)) == 0 &&
+                                            block_marked(dirty_map, kDirtyWords, blk);
+                        unsigned pages_hit = __ballot_sync(0xffffffffu, marked);
+                        if (pages_hit) {
+                            while (pages_hit) {
+                                const int src = __ffs(pages_hit) - 1;
+                                pages_hit &= pages_hit - 1;
+                                const int32_t bk = __shfl_sync(0xffffffffu, blk, src);
+                                write_block_rows<D, BS, Math<D, G, BS>::kElemBytes>(p, my_slots, bk, tile0, HG,
+                                                                                     lane);
+                            }
+                            fence_proxy_async_global();
+                            __syncwarp();
+                            fence_proxy_async_global();
+                        }
+                    } else if (APPEND && !rows_ready) {
                         const bool marked =
                             lane < n && (misc->all_dirty || block_marked(dirty_map, kDirtyWords, blk));
                         if (__any_sync(0xffffffffu, marked)) {
@@ -1436,7 +1542,11 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
             for (uint32_t i = (last > R ? last - R : 0); i < last; ++i)
                 mbar_wait(&full[i % R], (i / R) & 1, nullptr, 20000000ull);
         }
-        if (APPEND && lane == 0) depart_grid(p);
+        if (APPEND && !p.app_local && lane == 0) depart_grid(p);
+        if (p.num_groups > 0) {  // after this warp's last copy: the prefix-only sequences
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            prefix_only_outputs<D>(p, lane, 32);
+        }
         return;
     }
     if (warp >= HG) return;
@@ -1444,6 +1554,13 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
     // ========================= consumer warps =========================
     using MathT = Math<D, G, BS>;
     MathT st;
+    // this warp's staging of prefix range partials: per range G*D floats of
+    // output, then G (max, sum) pairs; 16-byte copies of whole pairs need G even
+    constexpr int kRangeBytes = G * D * 4 + ((G * 8 + 15) / 16) * 16;
+    constexpr int kStageWarpBytes = ((Cfg::kAreaBytes - Cfg::kDirtyBytes / 2) / NW) / 16 * 16;
+    constexpr int kStagedRanges = (G % 2 == 0) ? kStageWarpBytes / kRangeBytes : 0;
+    uint8_t* stage_area = smem + Cfg::kDirtyOff + Cfg::kDirtyBytes / 2 + warp * kStageWarpBytes;
+    bool dep_done = !p.defer_dep;  // this warp has waited for the prefix pass
     uint32_t stage_base = 0, seg_i = 0;
     const int64_t hgG = int64_t(HG) * G;  // query heads of one partial slot
     const int sub = warp / HS;              // this warp's stage within a page
@@ -1462,14 +1579,33 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
         st.oscale = p.v_scale ? __ldg(p.v_scale + g) : 1.f;
         st.reset();
         // The piece that starts at b's first own page carries the shared
-        // prefix: the partial of prefix key range 0 is loaded now and folded
-        // in after the pages (the loads overlap them), the others after it.
+        // prefix: the partials of its nz prefix key ranges are folded in after
+        // the pages.  When they fit, all of them are copied now (cp.async)
+        // into this warp's staging area and folded from shared memory, so the
+        // copies overlap the pages; otherwise range 0 is loaded into
+        // registers now and the others are read after the pages.
         const int nz = (d.P > 0 && d.j0 == d.P)
                            ? (d.P + prefix_split_pages(d.P, p.prefix_splits) - 1) /
                                  prefix_split_pages(d.P, p.prefix_splits)
                            : 0;
+        const bool staged = nz > 0 && nz <= kStagedRanges;
         typename MathT::Piece piece;
-        if (nz > 0) st.piece_load(piece, p.prefix_o + row * D, p.prefix_ml + row, lane);
+        auto stage_ranges = [&]() {
+            for (int z = 0; z < nz; ++z) {
+                const int64_t idx = int64_t(z) * p.B * p.Hq + row;
+                uint8_t* dst = stage_area + z * kRangeBytes;
+                const uint8_t* so = reinterpret_cast<const uint8_t*>(p.prefix_o + idx * D);
+                for (int c = lane; c < G * D / 4; c += 32) cp_async16(dst + 16 * c, so + 16 * c);
+                const uint8_t* sml = reinterpret_cast<const uint8_t*>(p.prefix_ml + idx);
+                if (lane < G / 2) cp_async16(dst + G * D * 4 + 16 * lane, sml + 16 * lane);
+            }
+            cp_async_commit();
+        };
+        // the partials exist once the prefix pass is complete: a warp that has
+        // waited for it once fetches them now, otherwise after the pages
+        const bool early = nz > 0 && dep_done;
+        if (early && staged) stage_ranges();
+        else if (early) st.piece_load(piece, p.prefix_o + row * D, p.prefix_ml + row, lane);
 
         // (R is a multiple of SPL, so the stages of each warp recur in the
         // same slots and every parity wait is exact)
@@ -1520,7 +1656,22 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
             if (lane == 0) mbar_arrive(&empty[slot]);
         }
         stage_base += uint32_t(d.npg * SPL);
-        if (nz > 0) {
+        if (nz > 0 && !early) {
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            dep_done = true;
+            if (staged) stage_ranges();
+            else st.piece_load(piece, p.prefix_o + row * D, p.prefix_ml + row, lane);
+        }
+        if (staged) {
+            cp_async_wait_all();
+            __syncwarp();
+            for (int z = 0; z < nz; ++z) {
+                const uint8_t* src = stage_area + z * kRangeBytes;
+                st.template absorb<true>(reinterpret_cast<const float*>(src),
+                                         reinterpret_cast<const float2*>(src + G * D * 4), lane);
+            }
+            __syncwarp();  // read before the next segment's copies land
+        } else if (nz > 0) {
             st.piece_absorb(piece, lane);
             for (int z = 1; z < nz; ++z) {
                 const int64_t idx = int64_t(z) * p.B * p.Hq + row;

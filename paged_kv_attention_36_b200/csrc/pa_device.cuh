@@ -155,6 +155,16 @@ __global__ void wait_timeout_kernel(uint64_t limit_ns) {
     }
 }
 
+// ---- per-thread asynchronous copies global -> shared (cp.async) ------------
+// 16 bytes, both addresses 16-byte aligned, through L2 only (not L1).
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Waits for all of this thread's cp.async copies (then a warp or CTA barrier
+// makes them visible to the other threads).
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // ---- 1-D bulk copy global -> shared, completing on an mbarrier ------------
 // Both addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {

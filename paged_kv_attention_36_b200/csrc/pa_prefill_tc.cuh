@@ -279,14 +279,14 @@ __device__ __forceinline__ void tc_attention_tile(const Params& p) {
                 if (!kKOnV) umma_commit(&k_empty[s]);
                 return true;
             };
-            // S runs NS - 1 blocks ahead of P V.  With three or more buffers,
-            // block j's P V is issued as soon as P_j is in TMEM, then
-            // S_{j+NS-1} into the buffer P_{j-1} has released (its P V was
-            // issued one step earlier).  With two, S_{j+1} must wait for
-            // P_{j-1} V, so it is issued before waiting for P_j.
+            // S runs NS - 1 blocks ahead of P V.  Each step first issues the
+            // next S (S_{j+NS-1} with three or more buffers, into the buffer
+            // P_{j-1} V releases; S_{j+1} with two, after P_{j-1} V), then
+            // waits for P_j and issues P_j V, so an S never waits behind the
+            // softmax of the block before it.
             for (int i = 0; ok && i < NS - 1 && i < nblk; ++i) ok = issue_qk(i);
             for (int j = 0; ok && j < nblk; ++j) {
-                if (NS == 2 && j + 1 < nblk && !(ok = issue_qk(j + 1))) break;
+                if (j + NS - 1 < nblk && !(ok = issue_qk(j + NS - 1))) break;
                 const int s = j % KS, bb = j % NS;
                 ok = mbar_wait_sleep(&p_full[bb], uint32_t(j / NS) & 1, abort) &&
                      mbar_wait_sleep(&v_full[s], uint32_t(j / KS) & 1, abort);
@@ -299,7 +299,6 @@ __device__ __forceinline__ void tc_attention_tile(const Params& p) {
                 for (int pg = 0; pg < Cfg::kPages; ++pg)
                     if (pg < npg) umma_ts(t_o, pa + pg * 8, vd + uint64_t(pg * (2048 >> 4)), id_pv, uint32_t(j | pg));
                 umma_commit(&v_empty[s]);
-                if (NS > 2 && j + NS - 1 < nblk) ok = issue_qk(j + NS - 1);
             }
             // no MMA may still run when TMEM and shared memory are released
             umma_commit(drain);

@@ -130,6 +130,35 @@ def test_fp8_fused_reads_rows_written_by_other_ctas(pa, oracle_lib):
     assert pa.pa_device_errors(clear=True) == 0
 
 
+@pytest.mark.parametrize("name", ["qwen3", "llama32"])
+def test_fp8_fused_multi_token_append(pa, oracle_lib, name):
+    # the last 3 positions of every sequence appended in one step: 180 tokens
+    # (qwen3; each CTA writes the rows of the blocks it reads) or 384
+    # (llama32; the grid barrier of a cooperative launch)
+    from paged_kv_attention_36_b200 import workloads
+    w = workloads.make(name, poison=True)
+    B, Hkv, D = w.q.shape[0], w.k_cache.shape[1], w.q.shape[2]
+    seq = torch.arange(B).repeat(3)
+    pos = w.context_lens.to(torch.int64)[seq] - 1 - torch.arange(3).repeat_interleave(B)
+    sm = workloads.slots_for_positions(w.block_tables[seq], pos, 16)
+    g = torch.Generator().manual_seed(62)
+    kn = torch.randn((3 * B, Hkv, D), generator=g).to(torch.bfloat16)
+    vn = torch.randn((3 * B, Hkv, D), generator=g).to(torch.bfloat16)
+    ks, vs = _scales(Hkv)
+    k8, v8, gk8, gv8, tks, tvs = _quantize_both(pa, oracle_lib, w.k_cache, w.v_cache, ks, vs)
+    oracle_lib.append_fp8(paging.bits(kn), paging.bits(vn), sm.numpy(), k8, v8, ks, vs)
+    ref = oracle_lib.decode_fp8(paging.bits(w.q), k8, v8, ks, vs, w.block_tables.numpy(),
+                                w.context_lens.numpy(), w.scale)
+    d = torch.device("cuda")
+    out = torch.full_like(w.q.to(d), float("nan"))
+    pa.pa_append_decode_fp8(kn.to(d), vn.to(d), sm.to(d), w.q.to(d), gk8, gv8, tks, tvs, w.block_tables.to(d),
+                            w.context_lens.to(d), w.scale, out)
+    torch.cuda.synchronize()
+    assert np.array_equal(gk8.cpu().numpy(), k8) and np.array_equal(gv8.cpu().numpy(), v8)
+    _close(out, ref)
+    assert pa.pa_device_errors(clear=True) == 0
+
+
 @pytest.mark.parametrize("D,Hq,Hkv", [(64, 8, 2), (64, 32, 8), (128, 16, 8), (128, 8, 8), (64, 16, 2),
                                       (128, 64, 8)])
 def test_fp8_ragged_shapes(pa, oracle_lib, D, Hq, Hkv):

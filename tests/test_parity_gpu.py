@@ -361,6 +361,40 @@ def test_fused_append_reads_rows_written_by_other_ctas(pa, oracle_lib):
     _assert_close(out, ref)
 
 
+def _multi_token_step(w, per_seq, seed):
+    """The last per_seq positions of every sequence appended this step, in
+    position-major order, with fresh rows: T = per_seq * B tokens."""
+    from paged_kv_attention_36_b200 import workloads
+    B, Hkv, D = w.q.shape[0], w.k_cache.shape[1], w.q.shape[2]
+    seq = torch.arange(B).repeat(per_seq)
+    pos = w.context_lens.to(torch.int64)[seq] - 1 - torch.arange(per_seq).repeat_interleave(B)
+    slots = workloads.slots_for_positions(w.block_tables[seq], pos, 16)
+    g = torch.Generator().manual_seed(seed)
+    w.k_new = torch.randn((per_seq * B, Hkv, D), generator=g).to(torch.bfloat16)
+    w.v_new = torch.randn((per_seq * B, Hkv, D), generator=g).to(torch.bfloat16)
+    w.slot_mapping = slots
+    return w
+
+
+@pytest.mark.parametrize("name,per_seq", [("qwen3", 3), ("llama32", 3)])
+def test_fused_multi_token_append(pa, oracle_lib, name, per_seq):
+    # several new tokens per sequence: qwen3 gives 180 (at most 256: every CTA
+    # writes the rows of the blocks it reads itself), llama32 384 (the grid
+    # barrier of a cooperative launch)
+    from paged_kv_attention_36_b200 import workloads
+    _skip_unbuilt_workload(name)
+    w = _multi_token_step(workloads.make(name, poison=True), per_seq, seed=61)
+    kb, vb, ref = _oracle_step(oracle_lib, w)
+    t = _to_dev(w)
+    out = torch.full_like(t["q"], float("nan"))
+    pa.pa_append_decode(t["k_new"], t["v_new"], t["slot_mapping"], t["q"], t["k_cache"], t["v_cache"],
+                        t["block_tables"], t["context_lens"], w.scale, out)
+    torch.cuda.synchronize()
+    _assert_caches_equal(t, kb, vb)
+    _assert_close(out, ref)
+    assert pa.pa_device_errors(clear=True) == 0
+
+
 def test_fused_reports_bad_slot(pa):
     d = torch.device("cuda")
     q = torch.randn((2, 8, 64), device=d).to(torch.bfloat16)
