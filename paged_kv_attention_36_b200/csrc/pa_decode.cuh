@@ -152,7 +152,9 @@ struct Misc {
     int b0;              // sequence where the share starts
     long long pre0;      // weighted position of b0's first unit
     long long red[16];  // block reductions, one slot per warp (<= 16 warps)
+    unsigned char patch[32];  // fused append, local: per ring stage, the consumers write the new row
 };
+constexpr int kMaxRing = 32;  // ring stages a decode CTA may have (Misc::patch)
 static_assert(sizeof(Misc) <= 256, "misc area");
 
 
@@ -1207,6 +1209,41 @@ __device__ __forceinline__ void prefix_only_outputs(const DecodeParams& p, int t
     }
 }
 
+// Local fused append, consumer side.  In a decode step token b's new row
+// goes to the last page of sequence b; the CTA that reads that page does
+// not need it in global memory first: the consumer warp of each kv head
+// loads its head's new K and V values (bf16 caches) when the segment starts
+// (lane l: values E*l .. E*l+E-1, E = D/32) and writes them over the row in
+// the staged tiles (the swizzled panel layout).  The slice owner still
+// writes the row to the cache.
+template <int D>
+struct NewRow {
+    static constexpr int E = D / 32;  // values per lane
+    uint32_t k[E / 2], v[E / 2];      // bf16 pairs
+
+    __device__ __forceinline__ void load(const DecodeParams& p, int b, int g, int lane) {
+        const uint32_t* kr = reinterpret_cast<const uint32_t*>(p.k_new) + ((int64_t(b) * p.Hkv + g) * D + E * lane) / 2;
+        const uint32_t* vr = reinterpret_cast<const uint32_t*>(p.v_new) + ((int64_t(b) * p.Hkv + g) * D + E * lane) / 2;
+#pragma unroll
+        for (int i = 0; i < E / 2; ++i) {
+            k[i] = __ldg(kr + i);
+            v[i] = __ldg(vr + i);
+        }
+    }
+    // Writes the row over row `off` of the staged K tile kt and V tile vt.
+    __device__ __forceinline__ void patch(uint8_t* kt, uint8_t* vt, int off, int lane) const {
+        const int e0 = E * lane;
+        const int o = tile_off(off, e0 / 8) + (e0 % 8) * 2;
+        if constexpr (E == 4) {
+            *reinterpret_cast<uint2*>(kt + o) = make_uint2(k[0], k[1]);
+            *reinterpret_cast<uint2*>(vt + o) = make_uint2(v[0], v[1]);
+        } else {
+            *reinterpret_cast<uint32_t*>(kt + o) = k[0];
+            *reinterpret_cast<uint32_t*>(vt + o) = v[0];
+        }
+    }
+};
+
 // Local fused append: the calling warp writes the rows of every appended
 // token whose slot lies in block bk, for the kv heads g0 .. g0+ng-1, into
 // the cache (a bit copy, or the E4M3 encoding for fp8 caches), in token
@@ -1249,6 +1286,7 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
     constexpr int NT = Cfg::kThreads;
     static_assert(NW + 1 <= 16, "block reductions hold 16 warps");
     static_assert(R % Cfg::kMaxSpl == 0, "the stages of a page recur in the same slots");
+    static_assert(R <= kMaxRing, "one patch flag per stage");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* ring = smem + Cfg::kRingOff;
@@ -1265,6 +1303,10 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int HG = p.HG, HS = p.HS, SPL = p.SPL;
+    // fused append, local: consumers write token b's new row into the staged
+    // tiles of bf16 caches (for fp8 caches the encoding in the consumers cost
+    // more than it saved: the producer writes the row to the cache first)
+    constexpr bool kConsumerPatch = APPEND && Math<D, G, BS>::kElemBytes == 2;
 
     if (threadIdx.x == 0) {
         for (int r = 0; r < R; ++r) {
@@ -1279,29 +1321,19 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
         fence_mbar_init();
     }
 
-    if (APPEND) {
-        // The blocks this step's rows go to, marked in the hashed bitmap.
-        for (int i = threadIdx.x; i < kDirtyWords; i += NT) dirty_map[i] = 0u;
-        if (threadIdx.x == 0) misc->all_dirty = p.app_tokens > kDirtyMaxTokens;
-        __syncthreads();
-        if (p.app_tokens <= kDirtyMaxTokens) {
-            for (int t = threadIdx.x; t < p.app_tokens; t += NT) {
-                const int32_t slot = __ldg(p.slot_mapping + t);
-                if (slot < 0) continue;
-                const uint32_t bit = uint32_t(slot / BS) & uint32_t(kDirtyWords * 32 - 1);
-                atomicOr(&dirty_map[bit >> 5], 1u << (bit & 31));
-            }
-        }
-        // This CTA's slice of the slot-mapped append (the bit copy of
-        // pa::append_kernel, or the E4M3 encoding of pa::append_fp8_kernel
-        // for fp8 caches), then arrival at the grid barrier; a written row
-        // must be visible to the TMA loads of every CTA that reads its block.
+    // Fused append: this CTA's slice of the step's new rows (the bit copy of
+    // pa::append_kernel, or the E4M3 encoding of pa::append_fp8_kernel for
+    // fp8 caches).  Barrier mode: written now, then arrival at the grid
+    // barrier (a written row must be visible to the TMA loads of every CTA
+    // that reads its block).  Local mode: nobody waits for these writes, so
+    // the consumer warps make them while the first pages are in flight.
+    auto append_slice = [&](int tid, int nthreads) {
         const int64_t per = (p.app_chunks + gridDim.x - 1) / gridDim.x;
         const int64_t c0 = int64_t(blockIdx.x) * per;
         const int64_t c1 = c0 + per < p.app_chunks ? c0 + per : p.app_chunks;
         constexpr int CPR = D / 8;  // 16-byte chunks per row
-        for (int64_t idx = c0 + threadIdx.x; idx < c1; idx += NT) {
-            if constexpr (Math<D, G, BS>::kElemBytes == 1) {  // fp8 caches: encode (pa::append_fp8_kernel)
+        for (int64_t idx = c0 + tid; idx < c1; idx += nthreads) {
+            if constexpr (Math<D, G, BS>::kElemBytes == 1) {
                 append_fp8_chunk(p.k_new, p.v_new, p.slot_mapping, reinterpret_cast<uint8_t*>(p.k_cache_w),
                                  reinterpret_cast<uint8_t*>(p.v_cache_w), p.k_scale, p.v_scale, p.Hkv, CPR, p.NB,
                                  idx);
@@ -1321,7 +1353,18 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
             p.k_cache_w[dst] = __ldg(p.k_new + idx);
             p.v_cache_w[dst] = __ldg(p.v_new + idx);
         }
-        if (!p.app_local) {  // barrier: arrive once the slice is visible to every CTA's TMA loads
+    };
+    // The blocks the rows go to are marked in the hashed bitmap: cleared now,
+    // marked after the share scan (whose barriers order the two), read by the
+    // producer after the barrier that ends the set-up.  A thread's first slot
+    // is loaded now so that its latency overlaps the scan.
+    int32_t first_slot = -1;
+    if (APPEND) {
+        for (int i = threadIdx.x; i < kDirtyWords; i += NT) dirty_map[i] = 0u;
+        if (threadIdx.x == 0) misc->all_dirty = p.app_tokens > kDirtyMaxTokens;
+        if (threadIdx.x < p.app_tokens) first_slot = __ldg(p.slot_mapping + threadIdx.x);
+        if (!p.app_local) {
+            append_slice(threadIdx.x, NT);
             fence_proxy_async_global();
             __threadfence();
             __syncthreads();
@@ -1351,6 +1394,15 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
         v_mine = v;
         incl_mine = incl;
     }
+    if (APPEND && p.app_tokens <= kDirtyMaxTokens) {
+        auto mark = [&](int32_t slot) {
+            if (slot < 0) return;
+            const uint32_t bit = uint32_t(slot / BS) & uint32_t(kDirtyWords * 32 - 1);
+            atomicOr(&dirty_map[bit >> 5], 1u << (bit & 31));
+        };
+        mark(first_slot);
+        for (int t = threadIdx.x + NT; t < p.app_tokens; t += NT) mark(__ldg(p.slot_mapping + t));
+    }
     // A decode launched right after prefix_kernel (programmatic dependent
     // launch) has done the set-up above meanwhile; the prefix partials and
     // the rows that kernel appended are read only after this wait (a no-op
@@ -1359,6 +1411,7 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
     const int64_t want = (Wt + p.min_pages - 1) / p.min_pages;
     const int64_t grid_eff = want < int64_t(gridDim.x) ? want : int64_t(gridDim.x);
     if (Wt == 0 || int64_t(blockIdx.x) >= grid_eff) {  // no share: read no page
+        if (APPEND && p.app_local) append_slice(threadIdx.x, NT);
         if (APPEND && !p.app_local && threadIdx.x == 0) depart_grid(p);
         if (p.num_groups > 0) {
             asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -1463,24 +1516,52 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
                             blk = 0;
                         }
                     }
+                    bool patch_page = false;  // this lane's stage: the consumers write the new row
                     if (APPEND && p.app_local) {
-                        // the new rows of each marked page of the batch (its first
-                        // stage's lane stands for it), this head group's heads
+                        // Each marked page of the batch (its first stage's lane stands
+                        // for it): when its only new row is token b's, at the last
+                        // position of b, in b's last page, the consumers write that row
+                        // into the staged tiles; otherwise the new rows are written to
+                        // the cache here before the page is loaded.
                         const bool marked = lane < n && ((c0 + lane) & (SPL - 1)) == 0 &&
                                             block_marked(dirty_map, kDirtyWords, blk);
                         unsigned pages_hit = __ballot_sync(0xffffffffu, marked);
-                        if (pages_hit) {
-                            while (pages_hit) {
-                                const int src = __ffs(pages_hit) - 1;
-                                pages_hit &= pages_hit - 1;
-                                const int32_t bk = __shfl_sync(0xffffffffu, blk, src);
+                        unsigned by_consumers = 0u;
+                        bool wrote = false;
+                        while (pages_hit) {
+                            const int src = __ffs(pages_hit) - 1;
+                            pages_hit &= pages_hit - 1;
+                            const int32_t bk = __shfl_sync(0xffffffffu, blk, src);
+                            int cnt = 0, t_first = -1;
+                            int32_t s_first = 0;
+#pragma unroll
+                            for (int k = 0; k < kLocalMaxTokens / 32; ++k) {
+                                const unsigned h = __ballot_sync(0xffffffffu, my_slots[k] >= 0 && my_slots[k] / BS == bk);
+                                if (h && t_first < 0) {
+                                    const int tl = __ffs(h) - 1;
+                                    t_first = 32 * k + tl;
+                                    s_first = __shfl_sync(0xffffffffu, my_slots[k], tl);
+                                }
+                                cnt += __popc(h);
+                            }
+                            const int page = j + ((c0 + src) >> p.SPL_LOG);
+                            if (kConsumerPatch && cnt == 1 && t_first == b && page == (Lb - 1) / BS &&
+                                s_first % BS == (Lb - 1) % BS) {
+                                by_consumers |= 1u << src;
+                            } else if (cnt > 0) {
                                 write_block_rows<D, BS, Math<D, G, BS>::kElemBytes>(p, my_slots, bk, tile0, HG,
                                                                                      lane);
+                                wrote = true;
                             }
+                        }
+                        if (wrote) {
                             fence_proxy_async_global();
                             __syncwarp();
                             fence_proxy_async_global();
                         }
+                        // every stage of a page follows its first stage's lane
+                        const int lead = lane & ~(SPL - 1);
+                        patch_page = (by_consumers >> lead) & 1u;
                     } else if (APPEND && !rows_ready) {
                         const bool marked =
                             lane < n && (misc->all_dirty || block_marked(dirty_map, kDirtyWords, blk));
@@ -1501,6 +1582,7 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
                         if (use > 0) lane_ok = mbar_wait(&empty[slot], (use - 1) & 1, abort);
                         if (lane_ok) {
                             uint8_t* st = ring + slot * Cfg::kStage;
+                            if (APPEND) misc->patch[slot] = patch_page ? 1 : 0;
                             mbar_arrive_expect_tx(&full[slot], stage_tx);
                             const int tile = blk * p.Hkv + tile0 + sub * HS;
                             tma_load_4d(st, &p.tmap_k, 0, 0, 0, tile, &full[slot], pol);
@@ -1549,6 +1631,7 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
         }
         return;
     }
+    if (APPEND && p.app_local) append_slice(threadIdx.x, NW * 32);  // warps 0 .. NW-1
     if (warp >= HG) return;
 
     // ========================= consumer warps =========================
@@ -1607,6 +1690,13 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
         if (early && staged) stage_ranges();
         else if (early) st.piece_load(piece, p.prefix_o + row * D, p.prefix_ml + row, lane);
 
+        // fused append, local: token b's new row of this warp's head, written
+        // over the staged tiles of the stages the producer flags
+        NewRow<D> nrow;
+        if constexpr (kConsumerPatch)
+            if (p.app_local && (d.j0 + d.npg) * BS >= d.L && d.b < p.app_tokens) nrow.load(p, d.b, g, lane);
+        const int noff = (d.L - 1) % BS;  // the new row's place in the last page
+
         // (R is a multiple of SPL, so the stages of each warp recur in the
         // same slots and every parity wait is exact)
         if constexpr (MathT::kPairPages) {
@@ -1622,6 +1712,7 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
                 const int nr0 = d.L - (d.j0 + k) * BS, nr1 = d.L - (d.j0 + k + 1) * BS;
                 const int nv0 = nr0 < BS ? nr0 : BS;
                 const int nv1 = two ? (nr1 < BS ? nr1 : BS) : 0;
+
                 st.page2(kt0, kt0 + Cfg::kStageK, nv0, kt1, kt1 + Cfg::kStageK, nv1, lane);
                 __syncwarp();
                 if (lane == 0) {
@@ -1638,6 +1729,13 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
             uint8_t* vt = kt + Cfg::kStageK;
             const int nv_raw = d.L - (d.j0 + k) * BS;
             const int nv = nv_raw < BS ? nv_raw : BS;
+            bool wrote = false;
+            if constexpr (kConsumerPatch) {
+                if (p.app_local && misc->patch[slot]) {
+                    nrow.patch(kt, vt, noff, lane);
+                    wrote = true;
+                }
+            }
             if (MathT::kZeroMaskedV && nv < BS) {
                 // rows past the context may hold anything (NaN included): clear
                 // them in this head's V tile so that 0 * row stays 0 in the tensor core
@@ -1648,6 +1746,9 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
                     const int t = nv + (rem >> 3), cch = rem & 7;
                     *reinterpret_cast<uint4*>(vt + pn * Cfg::kPanel + t * 128 + cch * 16) = make_uint4(0, 0, 0, 0);
                 }
+                wrote = true;
+            }
+            if (wrote) {  // before the page math, and before the stage is refilled by TMA
                 __syncwarp();
                 fence_proxy_async_smem();
             }
