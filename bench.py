@@ -209,10 +209,15 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+HOLD = True  # untimed runs around the timed regions, for the clock samples (off with --no-clocks)
+
+
 def hold_load(call, seconds: float, dev, between=None):
     """Runs `call` back to back, untimed, for about `seconds` of wall time
     (in bursts of 50, synchronised), so that the clock samples taken around
     a short timed region see the same load."""
+    if not HOLD:
+        return
     t0 = time.time()
     while time.time() - t0 < seconds:
         for _ in range(50):
@@ -922,7 +927,9 @@ def run_prefill(args, ws, rank, local, reference: bool):
 
 
 def main():
+    global HOLD
     args = _args()
+    HOLD = not args.no_clocks
     ws, rank, local = _dist()
     try:
         if args.mode == "prefill":

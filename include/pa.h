@@ -145,17 +145,25 @@ PA_API pa_status pa_decode(const void* q, const void* k_cache, const void* v_cac
 /*
  * One decode step in one launch: the slot-mapped append of the step's new
  * K/V rows (pa_cache_append) and then paged decode attention over the
- * caches including those rows (pa_decode), fused.  Each CTA writes a slice
- * of the rows and arrives at a grid barrier (a cooperative launch, so all
- * CTAs are resident); a CTA waits there only before it reads a block that
- * the step's rows go to (blocks marked in a hashed bitmap of the slots), so
- * for a decode step, whose new rows sit in each sequence's last page, the
- * wait is off the critical path.  Arguments as for the two calls; the
- * workspace as for pa_decode.  Compared with the two calls it saves the
- * append's launch and its latency (miniVLLM docs index, "What is
- * miniVLLM?": low-latency decode; the append and the decode of one step).
- * After a call that set PA_DEVERR_TIMEOUT the workspace must be zero-filled
- * again.
+ * caches including those rows (pa_decode), fused.  Every CTA writes a slice
+ * of the rows to the caches and marks the blocks they go to in a hashed
+ * bitmap; what a CTA does before reading a marked block depends on
+ * num_tokens:
+ *   - up to 256 (a decode step has one per sequence): no CTA waits for
+ *     another.  When a block's only new row is token b's, at the last
+ *     position of sequence b, the CTA reading it patches that row into its
+ *     staged copy of the page (bf16 caches); otherwise it writes the block's
+ *     new rows to the caches itself before loading it (the same bytes as the
+ *     slice owner).  An ordinary launch.
+ *   - more: the CTAs meet at a grid barrier (a cooperative launch, so all
+ *     are resident), and a CTA waits there only before its first marked
+ *     block.
+ * Arguments as for the two calls; the workspace as for pa_decode.  Compared
+ * with the two calls it saves the append's launch and its latency
+ * (miniVLLM docs index, "What is miniVLLM?": low-latency decode; the append
+ * and the decode of one step).  Two tokens mapped to one slot: which lands,
+ * and which one a sequence reading that slot sees, is unspecified.  After a
+ * call that set PA_DEVERR_TIMEOUT the workspace must be zero-filled again.
  */
 PA_API pa_status pa_append_decode(const void* k_new, const void* v_new, const int32_t* slot_mapping,
                                   int32_t num_tokens, const void* q, void* k_cache, void* v_cache,
@@ -245,12 +253,15 @@ PA_API pa_status pa_decode_static_ws(const void* q, const void* k_cache, const v
  *     does not begin with the group's first member's P_i block ids (the
  *     output of such members is unspecified).
  *   - num_tokens > 0 also appends k_new/v_new at slot_mapping first (as
- *     pa_cache_append), inside the prefix pass's launch (or, with no groups,
- *     fused into the decode as in pa_append_decode); slots must not fall in
- *     the shared blocks, which the prefix pass reads meanwhile.
+ *     pa_cache_append): fused into the decode as in pa_append_decode (up to
+ *     256 tokens), or inside the prefix pass's launch (more); slots must not
+ *     fall in the shared blocks, which the prefix pass reads meanwhile.
  *     num_tokens = 0 skips the append (k_new, v_new, slot_mapping unused).
  *   - Two launches: the prefix pass, then the decode as its programmatic
- *     dependent, so that the decode's set-up overlaps the pass's end.
+ *     dependent.  With up to 256 new tokens the decode streams the members'
+ *     own pages while the prefix pass runs and waits for the pass only
+ *     before it reads the pass's partials; with more, it waits for the pass
+ *     before reading any page (the pass wrote the new rows).
  *   - Supported shapes and alignment as for pa_decode.  The workspace must
  *     be at least pa_decode_shared_prefix_workspace_bytes(dims, num_groups,
  *     max_group_size) bytes, zero-filled before its first use, and is left
@@ -303,12 +314,13 @@ PA_API pa_status pa_decode_fp8(const void* q, const void* k_cache, const void* v
 /*
  * One fp8 decode step in one launch: pa_cache_append_fp8 of the step's new
  * bf16 rows into the fp8 caches, then pa_decode_fp8 over the caches
- * including them, fused as pa_append_decode fuses the bf16 calls (a
- * cooperative launch; a CTA waits at the grid barrier only before reading a
- * block the new rows go to).  Arguments, codes and results as for the two
- * calls; the workspace as for pa_decode.  Graph-capturable like every call
- * here (no allocation, no synchronisation).  After a call that set
- * PA_DEVERR_TIMEOUT the workspace must be zero-filled again.
+ * including them, fused as pa_append_decode fuses the bf16 calls (up to 256
+ * tokens: a CTA writes the encoded new rows of a block to the caches itself
+ * before loading it; more: a grid barrier of a cooperative launch).
+ * Arguments, codes and results as for the two calls; the workspace as for
+ * pa_decode.  Graph-capturable like every call here (no allocation, no
+ * synchronisation).  After a call that set PA_DEVERR_TIMEOUT the workspace
+ * must be zero-filled again.
  */
 PA_API pa_status pa_append_decode_fp8(const void* k_new, const void* v_new, const int32_t* slot_mapping,
                                       int32_t num_tokens, const void* q, void* k_cache, void* v_cache,
