@@ -1692,10 +1692,16 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
 
         // fused append, local: token b's new row of this warp's head, written
         // over the staged tiles of the stages the producer flags
+        // (only the segment's last page, when it is b's last page, can carry
+        // the row: the flag is read there alone, so other pages pay nothing)
         NewRow<D> nrow;
-        if constexpr (kConsumerPatch)
-            if (p.app_local && (d.j0 + d.npg) * BS >= d.L && d.b < p.app_tokens) nrow.load(p, d.b, g, lane);
-        const int noff = (d.L - 1) % BS;  // the new row's place in the last page
+        int patch_k = -1;  // the page of this segment that may take the row
+        if constexpr (kConsumerPatch) {
+            if (p.app_local && (d.j0 + d.npg) * BS >= d.L && d.b < p.app_tokens) {
+                nrow.load(p, d.b, g, lane);
+                patch_k = d.npg - 1;
+            }
+        }
 
         // (R is a multiple of SPL, so the stages of each warp recur in the
         // same slots and every parity wait is exact)
@@ -1731,8 +1737,8 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
             const int nv = nv_raw < BS ? nv_raw : BS;
             bool wrote = false;
             if constexpr (kConsumerPatch) {
-                if (p.app_local && misc->patch[slot]) {
-                    nrow.patch(kt, vt, noff, lane);
+                if (k == patch_k && misc->patch[slot]) {
+                    nrow.patch(kt, vt, (d.L - 1) % BS, lane);
                     wrote = true;
                 }
             }
