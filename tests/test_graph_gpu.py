@@ -89,6 +89,30 @@ def test_graph_fused_append_decode(pa, oracle_lib):
     _run(pa, oracle_lib, w, step)
 
 
+def test_graph_fused_append_decode_barrier_mode(pa, oracle_lib):
+    # more than 256 new rows (the last 3 positions of each of 128 sequences):
+    # the fused step's CTAs meet at a grid barrier, a cooperative launch,
+    # captured and replayed; every replay must leave the barrier at zero
+    from paged_kv_attention_36_b200 import workloads
+    w = workloads.make("llama32", poison=True)
+    B = w.q.shape[0]
+    seq = torch.arange(B).repeat(3)
+    pos = w.context_lens.to(torch.int64)[seq] - 1 - torch.arange(3).repeat_interleave(B)
+    w.slot_mapping = workloads.slots_for_positions(w.block_tables[seq], pos, 16)
+    g0 = torch.Generator().manual_seed(79)
+    w.k_new = torch.randn((3 * B,) + tuple(w.k_new.shape[1:]), generator=g0).to(torch.bfloat16)
+    w.v_new = torch.randn((3 * B,) + tuple(w.v_new.shape[1:]), generator=g0).to(torch.bfloat16)
+
+    def step(t, out):
+        dims = pa.make_dims(t["q"], t["k_cache"], t["block_tables"])
+        if not hasattr(step, "ws"):
+            step.ws = pa.alloc_workspace(dims)
+        pa.pa_append_decode(t["k_new"], t["v_new"], t["slot_mapping"], t["q"], t["k_cache"], t["v_cache"],
+                            t["block_tables"], t["context_lens"], w.scale, out, workspace=step.ws)
+    _run(pa, oracle_lib, w, step, replays=2)
+    assert int(step.ws[-256:].view(torch.int32).abs().sum()) == 0
+
+
 def test_graph_two_call_step(pa, oracle_lib):
     from paged_kv_attention_36_b200 import workloads
     w = workloads.make("longskew", poison=True)
