@@ -130,6 +130,30 @@ def test_fp8_fused_reads_rows_written_by_other_ctas(pa, oracle_lib):
     assert pa.pa_device_errors(clear=True) == 0
 
 
+def test_fp8_fused_large_batch(pa, oracle_lib):
+    # 700 sequences (a tenth empty): more than a decode CTA's 288 threads, so
+    # the share scan runs in chunks, and 700 new rows (the grid-barrier mode)
+    from paged_kv_attention_36_b200 import workloads
+    g = torch.Generator().manual_seed(77)
+    lens = torch.randint(1, 201, (700,), generator=g)
+    lens[torch.rand(700, generator=g) < 0.1] = 0
+    w = workloads.make("qwen3", poison=True, context_lens=lens, seed=77)
+    ks, vs = _scales(w.k_cache.shape[1])
+    k8, v8, gk8, gv8, tks, tvs = _quantize_both(pa, oracle_lib, w.k_cache, w.v_cache, ks, vs)
+    oracle_lib.append_fp8(paging.bits(w.k_new), paging.bits(w.v_new), w.slot_mapping.numpy(), k8, v8, ks, vs)
+    ref = oracle_lib.decode_fp8(paging.bits(w.q), k8, v8, ks, vs, w.block_tables.numpy(),
+                                w.context_lens.numpy(), w.scale)
+    d = torch.device("cuda")
+    q = w.q.to(d)
+    out = torch.full_like(q, float("nan"))
+    pa.pa_append_decode_fp8(w.k_new.to(d), w.v_new.to(d), w.slot_mapping.to(d), q, gk8, gv8, tks, tvs,
+                            w.block_tables.to(d), w.context_lens.to(d), w.scale, out)
+    torch.cuda.synchronize()
+    assert np.array_equal(gk8.cpu().numpy(), k8) and np.array_equal(gv8.cpu().numpy(), v8)
+    _close(out, ref)
+    assert pa.pa_device_errors(clear=True) == 0
+
+
 @pytest.mark.parametrize("name", ["qwen3", "llama32"])
 def test_fp8_fused_multi_token_append(pa, oracle_lib, name):
     # the last 3 positions of every sequence appended in one step: 180 tokens

@@ -395,6 +395,36 @@ def test_fused_multi_token_append(pa, oracle_lib, name, per_seq):
     assert pa.pa_device_errors(clear=True) == 0
 
 
+def _large_batch(name, B, hi, seed):
+    """B sequences of U[1, hi] tokens, a tenth of them empty."""
+    from paged_kv_attention_36_b200 import workloads
+    g = torch.Generator().manual_seed(seed)
+    lens = torch.randint(1, hi + 1, (B,), generator=g)
+    lens[torch.rand(B, generator=g) < 0.1] = 0
+    return workloads.make(name, poison=True, context_lens=lens, seed=seed)
+
+
+@pytest.mark.parametrize("name,B,hi", [("tiny", 1000, 120), ("qwen3", 600, 300)])
+def test_large_batch_scans_in_chunks(pa, oracle_lib, name, B, hi):
+    # more sequences than a decode CTA has threads (288): the scan of the
+    # work line and the search for each CTA's first sequence run over
+    # several chunks; fused, the B new rows take the grid-barrier mode
+    _skip_unbuilt_workload(name)
+    w = _large_batch(name, B, hi, seed=B + hi)
+    kb, vb, ref = _oracle_step(oracle_lib, w)
+    t = _to_dev(w)
+    _assert_close(_gpu_step(pa, t, w.scale), ref)
+    _assert_caches_equal(t, kb, vb)
+    t = _to_dev(w)
+    out = torch.full_like(t["q"], float("nan"))
+    pa.pa_append_decode(t["k_new"], t["v_new"], t["slot_mapping"], t["q"], t["k_cache"], t["v_cache"],
+                        t["block_tables"], t["context_lens"], w.scale, out)
+    torch.cuda.synchronize()
+    _assert_caches_equal(t, kb, vb)
+    _assert_close(out, ref)
+    assert pa.pa_device_errors(clear=True) == 0
+
+
 def test_fused_reports_bad_slot(pa):
     d = torch.device("cuda")
     q = torch.randn((2, 8, 64), device=d).to(torch.bfloat16)

@@ -130,6 +130,38 @@ def test_group_shapes(pa, oracle_lib, heads):
     assert pa.pa_device_errors(clear=True) == 0
 
 
+@pytest.mark.parametrize("fused", [False, True])
+def test_large_grouped_batch(pa, oracle_lib, fused):
+    # 330 members in two groups plus 30 sequences in none: more sequences
+    # than a decode CTA's 288 threads (the share scan runs in chunks); fused,
+    # the 360 new rows are more than the decode appends itself, so the
+    # prefix pass writes them and the decode waits for it (their slots are
+    # past the shared blocks: a private suffix of at least one token)
+    from paged_kv_attention_36_b200 import workloads
+    g = torch.Generator().manual_seed(91)
+    suffix = torch.randint(1 if fused else 0, 60, (330,), generator=g).tolist()
+    tails = torch.randint(0, 90, (30,), generator=g).tolist()
+    w = workloads.make_grouped("tiny", [(150, 3), (180, 2)], suffix, tail_lens=tails, poison=True)
+    t = _dev(w)
+    if fused:
+        kb, vb = paging.bits(w.k_cache).copy(), paging.bits(w.v_cache).copy()
+        oracle_lib.append(paging.bits(w.k_new), paging.bits(w.v_new), w.slot_mapping.numpy(), kb, vb)
+        ref = oracle_lib.decode(paging.bits(w.q), kb, vb, w.block_tables.numpy(), w.context_lens.numpy(),
+                                w.scale)
+        out = torch.full_like(t["q"], float("nan"))
+        pa.pa_decode_shared_prefix(t["q"], t["k_cache"], t["v_cache"], t["block_tables"], t["context_lens"],
+                                   w.scale, t["group_offsets"], t["group_prefix_pages"], w.max_group_size, out,
+                                   k_new=t["k_new"], v_new=t["v_new"], slot_mapping=t["slot_mapping"])
+        torch.cuda.synchronize()
+        assert torch.equal(t["k_cache"].view(torch.int16).cpu(), torch.from_numpy(kb.view(np.int16)))
+        assert torch.equal(t["v_cache"].view(torch.int16).cpu(), torch.from_numpy(vb.view(np.int16)))
+    else:
+        ref = _ref(oracle_lib, w)
+        out = _decode(pa, t, w)
+    _assert_close(out, ref)
+    assert pa.pa_device_errors(clear=True) == 0
+
+
 def test_members_whose_context_is_the_prefix(pa, oracle_lib):
     # suffix 0: no own pages, the output is the prefix partials merged alone
     from paged_kv_attention_36_b200 import workloads
