@@ -267,8 +267,11 @@ PA_API pa_status pa_decode_static_ws(const void* q, const void* k_cache, const v
  *     max_group_size) bytes, zero-filled before its first use, and is left
  *     ready for the next call; calls that share it must not overlap.
  *   - The prefix pass splits each group's shared pages into key ranges
- *     (enough CTAs for one wave; PA_PREFIX_SPLITS=n, 1..16, read at the
- *     first call, overrides); the decode folds one partial per range.
+ *     (enough CTAs for half a wave; PA_PREFIX_SPLITS=n, 1..16, read at the
+ *     first call, overrides); the decode folds one partial per range.  The
+ *     decode CTAs that start on the SMs the pass leaves free take a larger
+ *     share of the members' own pages (sized by the longest prefix); the
+ *     result does not depend on the shares.
  *   - num_groups = 0 is pa_decode / pa_append_decode with this workspace.
  */
 PA_API size_t pa_decode_shared_prefix_workspace_bytes(const pa_dims* dims, int32_t num_groups,

@@ -113,6 +113,11 @@ struct DecodeParams {
     const int32_t* group_prefix_pages;  // [num_groups]
     int32_t num_groups, max_group_size;
     int32_t prefix_splits;              // key ranges of the prefix partials
+    // CTAs 0 .. early_ctas-1 start on SMs the prefix pass leaves free and take
+    // the units one CTA streams while the pass runs more than the others:
+    // early_units_per_ms * (early_ns + early_ns_per_page * pages of a key range) / 1e6
+    int32_t early_ctas;
+    int32_t early_ns, early_ns_per_page, early_units_per_ms;
     int32_t defer_dep;                  // 1: the decode owns the step's append, so it waits for the
                                         // prefix pass (griddepcontrol.wait) only before reading its
                                         // partials; 0: before reading anything (the pass appended)
@@ -136,12 +141,28 @@ struct SegDesc {
 static_assert(sizeof(SegDesc) == 64, "descriptor size");
 
 // Equal split of W pages over `grid` CTAs: CTA k gets [start(k), start(k+1)).
+// The CTAs' shares of the line: equal shares of the line minus E * extra
+// units (the first rem of them one unit longer), and the first E CTAs extra
+// units more each.  CTA k's share starts at
+//     start(k) = k * per + min(k, rem) + min(k, E) * extra;
+// owner(u) is the CTA whose share holds unit u.  E = 0 is the plain equal
+// split; E > 0 serves a decode whose first E CTAs start while the other SMs
+// still run the shared-prefix pass.
 struct Split {
     int64_t per, rem;
-    __device__ __forceinline__ int64_t start(int64_t k) const { return k * per + (k < rem ? k : rem); }
+    int64_t E = 0, extra = 0;
+    __device__ __forceinline__ int64_t start(int64_t k) const {
+        return k * per + (k < rem ? k : rem) + (k < E ? k : E) * extra;
+    }
     __device__ __forceinline__ int32_t owner(int64_t pg) const {
+        if (pg < start(E)) {  // the first E shares: per + extra units (+1 for the first rem)
+            const int64_t pe = per + extra, r = rem < E ? rem : E;
+            const int64_t big = r * (pe + 1);
+            return int32_t(pg < big ? pg / (pe + 1) : r + (pg - big) / pe);
+        }
+        const int64_t v = pg - E * extra;
         const int64_t big = rem * (per + 1);
-        return int32_t(pg < big ? pg / (per + 1) : rem + (pg - big) / per);
+        return int32_t(v < big ? v / (per + 1) : rem + (v - big) / per);
     }
 };
 
@@ -150,6 +171,8 @@ struct Misc {
     int abort;
     int all_dirty;       // fused append: every page counts as written this step
     int b0;              // sequence where the share starts
+    int L0, P0, np0;     // its context length, shared-prefix pages and own pages
+    int pmax;            // the longest shared prefix, in pages (early CTAs only)
     long long pre0;      // weighted position of b0's first unit
     long long red[16];  // block reductions, one slot per warp (<= 16 warps)
     unsigned char patch[32];  // fused append, local: per ring stage, the consumers write the new row
@@ -976,23 +999,41 @@ struct SeqPages {
     int32_t L, P, np;
 };
 
+constexpr int kFewGroups = 4;  // group tables read whole, in one round of loads
+
 template <int BS>
 __device__ __forceinline__ SeqPages seq_pages(const DecodeParams& p, int b, bool report) {
     SeqPages s;
     s.L = clamp_len<BS>(p, b, report);
     s.P = 0;
     if (p.num_groups > 0) {
+        // group i holds b when off[i] <= b < off[i+1]
         const int32_t* off = p.group_offsets;
-        if (b >= __ldg(off) && b < __ldg(off + p.num_groups)) {
-            int lo = 0, hi = p.num_groups;  // off[lo] <= b < off[hi]
+        const int ng = p.num_groups;
+        int32_t P = 0, beg = 0;
+        if (ng <= kFewGroups) {
+            int32_t o[kFewGroups + 1], pp[kFewGroups];
+#pragma unroll
+            for (int i = 0; i <= kFewGroups; ++i) o[i] = i <= ng ? __ldg(off + i) : 0;
+#pragma unroll
+            for (int i = 0; i < kFewGroups; ++i) pp[i] = i < ng ? __ldg(p.group_prefix_pages + i) : 0;
+#pragma unroll
+            for (int i = 0; i < kFewGroups; ++i)
+                if (i < ng && o[i] <= b && b < o[i + 1]) {
+                    P = pp[i];
+                    beg = o[i];
+                }
+        } else if (b >= __ldg(off) && b < __ldg(off + ng)) {
+            int lo = 0, hi = ng;  // off[lo] <= b < off[hi]
             while (hi - lo > 1) {
                 const int mid = (lo + hi) >> 1;
                 if (__ldg(off + mid) <= b) lo = mid;
                 else hi = mid;
             }
-            const int32_t P = __ldg(p.group_prefix_pages + lo);
-            if (P > 0 && int64_t(P) * BS <= s.L && b - __ldg(off + lo) < p.max_group_size) s.P = P;
+            P = __ldg(p.group_prefix_pages + lo);
+            beg = __ldg(off + lo);
         }
+        if (P > 0 && int64_t(P) * BS <= s.L && b - beg < p.max_group_size) s.P = P;
     }
     s.np = (s.L + BS - 1) / BS - s.P;
     return s;
@@ -1308,6 +1349,21 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
     // more than it saved: the producer writes the row to the cache first)
     constexpr bool kConsumerPatch = APPEND && Math<D, G, BS>::kElemBytes == 2;
 
+    // The producer's reads that need nothing computed here start now and
+    // land during the set-up and the share scan: its tensor maps, and (fused
+    // append, local) the step's slots, lane l holding tokens l, l+32, ...
+    constexpr int kSlotRegs = kLocalMaxTokens / 32;
+    int32_t my_slots[kSlotRegs];
+#pragma unroll
+    for (int k = 0; k < kSlotRegs; ++k) {
+        const int t = 32 * k + lane;
+        my_slots[k] = (APPEND && warp == NW && p.app_local && t < p.app_tokens) ? __ldg(p.slot_mapping + t) : -1;
+    }
+    if (warp == NW && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_k)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_v)) : "memory");
+    }
+
     if (threadIdx.x == 0) {
         for (int r = 0; r < R; ++r) {
             mbar_init(&full[r], 1);
@@ -1319,6 +1375,15 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
         }
         misc->abort = 0;
         fence_mbar_init();
+    }
+    if (p.early_ctas > 0 && warp == 0) {
+        // the longest shared prefix sets how long the prefix pass holds its
+        // SMs (published to the CTA by the scan's first barrier)
+        int32_t pm = 0;
+        for (int i = lane; i < p.num_groups; i += 32) pm = max(pm, __ldg(p.group_prefix_pages + i));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) pm = max(pm, __shfl_xor_sync(0xffffffffu, pm, off));
+        if (lane == 0) misc->pmax = pm;
     }
 
     // Fused append: this CTA's slice of the step's new rows (the bit copy of
@@ -1377,11 +1442,13 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
     // fits in one chunk the same scan also locates the share's start. ----
     const bool one_chunk = p.B <= NT;
     long long v_mine = 0, incl_mine = 0, Wt = 0;
+    SeqPages sp_mine{0, 0, 0};
     for (int base = 0; base < p.B; base += NT) {
         const int b = base + threadIdx.x;
         long long v = 0;
         if (b < p.B) {
             const SeqPages sp = seq_pages<BS>(p, b, blockIdx.x == 0);
+            sp_mine = sp;
             v = (long long)(sp.np > 0 ? sp.np + p.seg_weight : 0) * p.NG;
             if (sp.L == 0 && (b % int(gridDim.x)) == int(blockIdx.x)) {
                 uint4* o = reinterpret_cast<uint4*>(p.out + int64_t(b) * p.Hq * D);
@@ -1419,32 +1486,49 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
         }
         return;
     }
-    const Split split{Wt / grid_eff, Wt % grid_eff};
+    Split split{Wt / grid_eff, Wt % grid_eff};
+    if (p.early_ctas > 0 && misc->pmax > 0) {
+        // the early CTAs' extra units, keeping at least min_pages per share
+        const int64_t E = p.early_ctas < grid_eff ? p.early_ctas : grid_eff;
+        const int64_t ns = p.early_ns + int64_t(p.early_ns_per_page) * prefix_split_pages(misc->pmax, p.prefix_splits);
+        const int64_t want_x = ns * p.early_units_per_ms / 1000000;
+        const int64_t room = (Wt - grid_eff * int64_t(p.min_pages)) / E;
+        const int64_t x = want_x < room ? want_x : room;
+        if (x > 0) {
+            const int64_t Wr = Wt - E * x;
+            split = Split{Wr / grid_eff, Wr % grid_eff, E, x};
+        }
+    }
     const int64_t p_start = split.start(blockIdx.x);
     const int64_t p_end = split.start(int64_t(blockIdx.x) + 1);
 
-    // ---- the sequence where the share starts ----
-    auto locate = [&](int b, long long v, long long incl) {
+    // ---- the sequence where the share starts (with its page counts, so the
+    // producer starts without reading them again) ----
+    auto locate = [&](int b, long long v, long long incl, const SeqPages& sp) {
         const long long lo = incl - v;
         if (v > 0 && lo <= p_start && p_start < incl) {
             misc->b0 = b;
+            misc->L0 = sp.L;
+            misc->P0 = sp.P;
+            misc->np0 = sp.np;
             misc->pre0 = lo;
         }
     };
     if (one_chunk) {
-        locate(threadIdx.x, v_mine, incl_mine);
+        locate(threadIdx.x, v_mine, incl_mine, sp_mine);
     } else {
         long long carry = 0;
         for (int base = 0; base < p.B; base += NT) {
             const int b = base + threadIdx.x;
             long long v = 0;
+            SeqPages sp{0, 0, 0};
             if (b < p.B) {
-                const int32_t npb = seq_pages<BS>(p, b, false).np;
-                v = (long long)(npb > 0 ? npb + p.seg_weight : 0) * p.NG;
+                sp = seq_pages<BS>(p, b, false);
+                v = (long long)(sp.np > 0 ? sp.np + p.seg_weight : 0) * p.NG;
             }
             long long chunk_total;
             const long long incl = carry + block_incl_scan<NT>(v, misc->red, chunk_total);
-            locate(b, v, incl);
+            locate(b, v, incl, sp);
             carry += chunk_total;
         }
     }
@@ -1452,28 +1536,16 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
 
     if (warp == NW) {
         // ======================= producer warp =======================
-        if (lane == 0) {
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_k)) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_v)) : "memory");
-        }
         uint32_t stage_i = 0, seg_i = 0;
         constexpr int C = R < 32 ? R : 32;
         bool ok = true;
         bool rows_ready = !APPEND;  // fused append, barrier: every CTA's rows are visible
-        // fused append, local: the step's slots, lane l holding tokens l, l+32, ...
-        constexpr int kSlotRegs = kLocalMaxTokens / 32;
-        int32_t my_slots[kSlotRegs];
-#pragma unroll
-        for (int k = 0; k < kSlotRegs; ++k) {
-            const int t = 32 * k + lane;
-            my_slots[k] = (APPEND && p.app_local && t < p.app_tokens) ? __ldg(p.slot_mapping + t) : -1;
-        }
         const uint64_t pol = PA_EVICT_FIRST ? policy_evict_first() : policy_evict_normal();
         const uint32_t stage_tx = uint32_t(2 * HS * Cfg::kTile);
 
         // walk the (b, hg) whose units meet the share [p_start, p_end)
         int b = misc->b0;
-        SeqPages sp = seq_pages<BS>(p, b, false);
+        SeqPages sp{misc->L0, misc->P0, misc->np0};
         int32_t Lb = sp.L, Pb = sp.P, np = sp.np;  // the line holds b's pages Pb .. Pb+np-1
         int64_t unit = np + p.seg_weight;
         int hg = int((p_start - misc->pre0) / unit);

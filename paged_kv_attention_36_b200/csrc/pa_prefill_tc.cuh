@@ -162,6 +162,20 @@ __device__ __forceinline__ void tc_attention_tile(const Params& p) {
     const int pages = (nkeys + 15) / 16;
     const int nblk = (nkeys + BN - 1) / BN;
 
+    // Loads in flight while the barriers and TMEM are set up: the page ids of
+    // block 0 (producer lanes) and this thread's Q row (softmax warps).
+    const int32_t blk_first = (warp == 0 && lane < Cfg::kPages && lane < pages) ? __ldg(bt + lane) : 0;
+    uint4 qv[D / 8];
+    if (warp >= 2) {
+        const int r = row0 + (warp & 3) * 32 + lane;
+        const bool valid = r < nrows;
+        const int64_t qrow = int64_t(PREFIX ? first : q0) + r / G;
+        const int64_t orow = valid ? (qrow * p.Hq + g * G + r % G) * D : 0;
+        const uint4* src = reinterpret_cast<const uint4*>(p.q + orow * 2);
+#pragma unroll
+        for (int ch = 0; ch < D / 8; ++ch) qv[ch] = valid ? __ldg(src + ch) : make_uint4(0u, 0u, 0u, 0u);
+    }
+
     if (threadIdx.x == 0) {
         mbar_init(q_full, 128);
         for (int s = 0; s < KS; ++s) {
@@ -230,7 +244,7 @@ __device__ __forceinline__ void tc_attention_tile(const Params& p) {
         };
         // K runs one block ahead of V: V_j is read one softmax step after K_j
         int nk = 0, nv = 0;  // blocks whose K (V) copies were issued
-        int32_t blk_cur = page_of(0), blk_prev = 0;
+        int32_t blk_cur = blk_first, blk_prev = 0;
         for (int t = 0; t <= nblk; ++t) {
             const int32_t blk_next = page_of(t + 1);
             if (t < nblk) {
@@ -313,20 +327,16 @@ __device__ __forceinline__ void tc_attention_tile(const Params& p) {
         const uint32_t lanes = uint32_t(qw * 32) << 16;
         const int r = row0 + row;
         const bool valid = r < nrows;
-        // keys 0 .. lim-1 are visible to this row; its query and output row
+        // keys 0 .. lim-1 are visible to this row; its query row
         const int lim = PREFIX ? nkeys : (valid ? first_pos + r / G + 1 : 1);
         const int64_t qrow = int64_t(PREFIX ? first : q0) + r / G;
-        const int64_t orow = valid ? (qrow * p.Hq + g * G + r % G) * D : 0;
 
         // Q row into shared memory (128-byte swizzle: 16-byte chunk c of row t at c ^ (t % 8))
         {
-            const uint4* src = reinterpret_cast<const uint4*>(p.q + orow * 2);
 #pragma unroll
-            for (int ch = 0; ch < D / 8; ++ch) {
-                const uint4 v = valid ? __ldg(src + ch) : make_uint4(0u, 0u, 0u, 0u);
+            for (int ch = 0; ch < D / 8; ++ch)
                 *reinterpret_cast<uint4*>(qs + (ch >> 3) * Cfg::kPanelQ + row * 128 + (((ch & 7) ^ (row & 7)) << 4)) =
-                    v;
-            }
+                    qv[ch];
             fence_proxy_async_smem();
             mbar_arrive(q_full);
         }
@@ -493,21 +503,21 @@ __device__ __forceinline__ void tc_attention_tile(const Params& p) {
             }
         }
         if constexpr (PREFIX) {
-            // checks of the caller's grouping (kv head 0 only): each member of
-            // the tile holds the split's prefix blocks in its own table and
-            // its context covers the whole prefix
-            if (g == 0) {
-                const int npg = nkeys / 16;
-                const int m_lo = row0 / G;
-                const int m_hi = ((row0 + Cfg::kBM < nrows ? row0 + Cfg::kBM : nrows) + G - 1) / G;
-                for (int x = gt; x < (m_hi - m_lo) * npg; x += 128) {
-                    const int mem = first + m_lo + x / npg;
-                    const int j = pg0 + x % npg;
-                    if (__ldg(p.block_tables + int64_t(mem) * p.M + j) != __ldg(bt + (j - pg0)))
-                        raise_error(PA_DEVERR_PREFIX);
-                    if (x % npg == 0 && int64_t(__ldg(p.context_lens + mem)) < int64_t(P) * 16)
-                        raise_error(PA_DEVERR_PREFIX);
-                }
+            // checks of the caller's grouping: each member of the tile holds
+            // the split's prefix blocks in its own table and its context covers
+            // the whole prefix.  The (member, page) pairs are dealt out over the
+            // Hkv CTAs of the tile and split (kv head g takes every Hkv-th run
+            // of 128), so no CTA carries them all at its end.
+            const int npg = nkeys / 16;
+            const int m_lo = row0 / G;
+            const int m_hi = ((row0 + Cfg::kBM < nrows ? row0 + Cfg::kBM : nrows) + G - 1) / G;
+            for (int x = g * 128 + gt; x < (m_hi - m_lo) * npg; x += 128 * p.Hkv) {
+                const int mem = first + m_lo + x / npg;
+                const int j = pg0 + x % npg;
+                if (__ldg(p.block_tables + int64_t(mem) * p.M + j) != __ldg(bt + (j - pg0)))
+                    raise_error(PA_DEVERR_PREFIX);
+                if (x % npg == 0 && int64_t(__ldg(p.context_lens + mem)) < int64_t(P) * 16)
+                    raise_error(PA_DEVERR_PREFIX);
             }
         }
     }

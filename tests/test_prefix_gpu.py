@@ -162,6 +162,35 @@ def test_large_grouped_batch(pa, oracle_lib, fused):
     assert pa.pa_device_errors(clear=True) == 0
 
 
+@pytest.mark.parametrize("fused", [False, True])
+def test_many_groups(pa, oracle_lib, fused):
+    # ten groups, one of them empty and one sharing nothing: more groups than
+    # the decode reads in one round, so sequences find theirs by bisection
+    from paged_kv_attention_36_b200 import workloads
+    g = torch.Generator().manual_seed(93)
+    groups = [(2, 1), (3, 2), (1, 1), (0, 2), (4, 3), (2, 0), (1, 1), (3, 1), (2, 2), (5, 1)]
+    n = sum(m for m, _ in groups)
+    suffix = torch.randint(1, 50, (n,), generator=g).tolist()
+    w = workloads.make_grouped("tiny", groups, suffix, tail_lens=[9, 0], poison=True)
+    t = _dev(w)
+    if fused:
+        kb, vb = paging.bits(w.k_cache).copy(), paging.bits(w.v_cache).copy()
+        oracle_lib.append(paging.bits(w.k_new), paging.bits(w.v_new), w.slot_mapping.numpy(), kb, vb)
+        ref = oracle_lib.decode(paging.bits(w.q), kb, vb, w.block_tables.numpy(), w.context_lens.numpy(),
+                                w.scale)
+        out = torch.full_like(t["q"], float("nan"))
+        pa.pa_decode_shared_prefix(t["q"], t["k_cache"], t["v_cache"], t["block_tables"], t["context_lens"],
+                                   w.scale, t["group_offsets"], t["group_prefix_pages"], w.max_group_size, out,
+                                   k_new=t["k_new"], v_new=t["v_new"], slot_mapping=t["slot_mapping"])
+        torch.cuda.synchronize()
+        assert torch.equal(t["k_cache"].view(torch.int16).cpu(), torch.from_numpy(kb.view(np.int16)))
+    else:
+        ref = _ref(oracle_lib, w)
+        out = _decode(pa, t, w)
+    _assert_close(out, ref)
+    assert pa.pa_device_errors(clear=True) == 0
+
+
 def test_members_whose_context_is_the_prefix(pa, oracle_lib):
     # suffix 0: no own pages, the output is the prefix partials merged alone
     from paged_kv_attention_36_b200 import workloads
