@@ -60,6 +60,7 @@
 #include "pa_append.cuh"
 #include "pa_device.cuh"
 #include "pa_prefix.cuh"
+#include "pa_split.cuh"
 
 #ifndef PA_EVICT_FIRST
 #define PA_EVICT_FIRST 1  // K/V pages are read once: first candidates for L2 eviction
@@ -140,31 +141,6 @@ struct SegDesc {
 };
 static_assert(sizeof(SegDesc) == 64, "descriptor size");
 
-// Equal split of W pages over `grid` CTAs: CTA k gets [start(k), start(k+1)).
-// The CTAs' shares of the line: equal shares of the line minus E * extra
-// units (the first rem of them one unit longer), and the first E CTAs extra
-// units more each.  CTA k's share starts at
-//     start(k) = k * per + min(k, rem) + min(k, E) * extra;
-// owner(u) is the CTA whose share holds unit u.  E = 0 is the plain equal
-// split; E > 0 serves a decode whose first E CTAs start while the other SMs
-// still run the shared-prefix pass.
-struct Split {
-    int64_t per, rem;
-    int64_t E = 0, extra = 0;
-    __device__ __forceinline__ int64_t start(int64_t k) const {
-        return k * per + (k < rem ? k : rem) + (k < E ? k : E) * extra;
-    }
-    __device__ __forceinline__ int32_t owner(int64_t pg) const {
-        if (pg < start(E)) {  // the first E shares: per + extra units (+1 for the first rem)
-            const int64_t pe = per + extra, r = rem < E ? rem : E;
-            const int64_t big = r * (pe + 1);
-            return int32_t(pg < big ? pg / (pe + 1) : r + (pg - big) / pe);
-        }
-        const int64_t v = pg - E * extra;
-        const int64_t big = rem * (per + 1);
-        return int32_t(v < big ? v / (per + 1) : rem + (v - big) / per);
-    }
-};
 
 // Shared scalars.
 struct Misc {
@@ -1486,19 +1462,13 @@ __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, 1) decode_kernel(cons
         }
         return;
     }
-    Split split{Wt / grid_eff, Wt % grid_eff};
+    // the early CTAs' extra units: what one CTA streams while the prefix pass runs
+    int64_t want_x = 0;
     if (p.early_ctas > 0 && misc->pmax > 0) {
-        // the early CTAs' extra units, keeping at least min_pages per share
-        const int64_t E = p.early_ctas < grid_eff ? p.early_ctas : grid_eff;
         const int64_t ns = p.early_ns + int64_t(p.early_ns_per_page) * prefix_split_pages(misc->pmax, p.prefix_splits);
-        const int64_t want_x = ns * p.early_units_per_ms / 1000000;
-        const int64_t room = (Wt - grid_eff * int64_t(p.min_pages)) / E;
-        const int64_t x = want_x < room ? want_x : room;
-        if (x > 0) {
-            const int64_t Wr = Wt - E * x;
-            split = Split{Wr / grid_eff, Wr % grid_eff, E, x};
-        }
+        want_x = ns * p.early_units_per_ms / 1000000;
     }
+    const Split split = make_split(Wt, grid_eff, p.early_ctas, want_x, p.min_pages);
     const int64_t p_start = split.start(blockIdx.x);
     const int64_t p_end = split.start(int64_t(blockIdx.x) + 1);
 
