@@ -696,8 +696,9 @@ def run_pa(args, ws, rank, local):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                      "kernel": (("pa::prefix_kernel" if os.environ.get("PA_PREFILL_MMA") == "sync"
-                                 else "pa::prefix_tc_kernel (tcgen05; carries the append)")
-                                + " + pa::decode_kernel<...> (pa_decode_shared_prefix)"
+                                 else "pa::prefix_tc_kernel (tcgen05)")
+                                + " + pa::decode_kernel<..., APPEND> (pa_decode_shared_prefix; the decode"
+                                  " appends up to 256 new rows itself, the prefix launch any more)"
                                 if grouped else "pa::decode_kernel<..., APPEND> (pa_append_decode)"),
                      "traffic": _traffic(args.workload),
                      "algorithmic_bytes_per_launch": step_bytes},
